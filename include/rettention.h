@@ -1,0 +1,196 @@
+/*
+ * rettention.h -- C ABI of the B200 (sm_100a) Re-ttention attention library.
+ *
+ * Re-ttention ("Re-ttention: Ultra Sparse Visual Generation via Attention
+ * Statistical Reshape", project page) keeps only a few percent of the keys in
+ * each DiT attention step and corrects the sparse result with statistics
+ * cached at an earlier full-attention denoising step: the ratio between the
+ * full and the sparse softmax denominators, and the residual contribution of
+ * the masked-out tokens (project page, teaser and mechanism highlight).
+ *
+ * Three calls make up one attention layer's denoising cycle:
+ *   rt_build_block_mask     which key blocks each query block keeps;
+ *   rt_attn_full_capture    full attention at a capture step, plus the cache;
+ *   rt_attn_sparse_reshape  block-sparse attention reshaped with the cache.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Q, K, V and the attention output are bf16 tensors [B, H, N, D],
+ *    contiguous, in device memory.  Only the first d = head_dim columns carry
+ *    data; columns d..D-1 (D = head_dim_padded) must be zero on input and are
+ *    written as zero on output.  The softmax scale is passed by the caller
+ *    (normally 1/sqrt(d)).
+ *  - Tokens are grouped into blocks of block_size tokens, for queries and
+ *    keys alike; n_blocks = ceil(N / block_size) and the last block may be
+ *    short (ragged tail).
+ *  - The kept-block list is a CSR over the B*H*n_blocks query blocks
+ *    (row index (b*H + h)*n_blocks + query_block): row_ptr int32
+ *    [B*H*n_blocks + 1] holds global offsets into col_idx, col_idx int32 holds
+ *    head-local key-block indices, each row sorted ascending without
+ *    duplicates.
+ *  - Statistics are fp32: stat_m, stat_zfull, stat_zkept [B, H, N] and
+ *    stat_u [B, H, N, D] (columns d..D-1 zero).
+ *  - Every pointer argument except the shape is device memory, 16-byte
+ *    aligned, owned by the caller and never freed or retained by the library.
+ *    Calls are asynchronous on `stream` (NULL = the legacy default stream);
+ *    nothing is synchronised.
+ *  - Supported: head_dim_padded in {64, 80}, 1 <= head_dim <= head_dim_padded,
+ *    block_size in {64, 128}, n_blocks <= 2048.
+ *
+ * Errors
+ * ------
+ * Arguments are validated on the host before any CUDA call: a null pointer,
+ * a negative or zero size, a bad keep count or a misaligned pointer gives
+ * RT_ERR_INVALID_ARGUMENT, a head dim or block size outside the supported set
+ * gives RT_ERR_UNSUPPORTED, and nothing is launched.  A failed launch gives
+ * RT_ERR_CUDA.  Kernels never trap: every wait inside a kernel is bounded;
+ * when one runs out the kernel records RT_ERR_TIMEOUT in a device status word
+ * (read it with rt_take_device_error), leaves its outputs unspecified and
+ * returns.  A malformed CSR (indices out of range, unsorted rows) never makes
+ * a kernel read or write out of bounds; its results are unspecified.
+ */
+#ifndef RETTENTION_H
+#define RETTENTION_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RT_ABI_VERSION 1
+
+typedef enum rt_status {
+    RT_OK = 0,
+    RT_ERR_INVALID_ARGUMENT = 1,
+    RT_ERR_UNSUPPORTED = 2,
+    RT_ERR_CUDA = 3,
+    RT_ERR_TIMEOUT = 4
+} rt_status;
+
+/* Same type as cudaStream_t, spelled without the CUDA headers. */
+typedef struct CUstream_st *rt_stream_t;
+
+/* Problem shape, passed by host pointer. */
+typedef struct rt_shape {
+    int32_t batch;            /* B */
+    int32_t heads;            /* H */
+    int32_t seq_len;          /* N tokens */
+    int32_t head_dim;         /* d: logical head dim */
+    int32_t head_dim_padded;  /* D: stored head dim, >= d */
+    int32_t block_size;       /* tokens per query block and per key block */
+} rt_shape;
+
+/*
+ * rt_build_block_mask -- choose the key blocks each query block keeps.
+ *
+ * The project page's Abstract describes sparse attention as including "only a
+ * subset of tokens or patches", down to 3.1% of them; it does not say how the
+ * subset is chosen.  This call uses block mean pooling and a per-query-block
+ * top-k:
+ *   pooled_q[b,h,qb] = mean of q over the real tokens of query block qb
+ *                      (logical columns only); pooled_k likewise;
+ *   score[qb,kb]     = scale * <pooled_q[qb], pooled_k[kb]>;
+ *   kept(qb)         = every key block overlapping tokens [0, forced_prefix_tokens)
+ *                      plus the keep_blocks - |forced| other blocks with the
+ *                      largest score (equal scores: lower block index first),
+ *                      written sorted ascending.
+ *
+ * q, k          bf16 [B,H,N,D] device.
+ * scale         softmax scale used for the block scores.
+ * keep_blocks   kept key blocks per query block, 1..n_blocks, and at least
+ *               the number of forced blocks.
+ * forced_prefix_tokens  >= 0; 0 forces nothing.
+ * row_ptr       out, int32 [B*H*n_blocks + 1] device; row r starts at r*keep_blocks.
+ * col_idx       out, int32 [B*H*n_blocks*keep_blocks] device.
+ * block_scores  optional out (may be NULL), fp32 [B,H,n_blocks,n_blocks] device:
+ *               the scores the selection used.
+ * Takes a transient device workspace of 2*B*H*n_blocks*d*4 bytes from the
+ * stream-ordered allocator on `stream` and returns it on the same stream.
+ */
+rt_status rt_build_block_mask(const rt_shape *shape, const void *q, const void *k, float scale,
+                              int32_t keep_blocks, int32_t forced_prefix_tokens,
+                              int32_t *row_ptr, int32_t *col_idx, float *block_scores,
+                              rt_stream_t stream);
+
+/*
+ * rt_attn_full_capture -- full attention at a capture step, and the cache.
+ *
+ * The teaser reshapes sparse attention "with cached statistics across
+ * denoising steps"; the mechanism highlight names the cached quantities: the
+ * stable ratio between sparse and full softmax denominators and the residual
+ * contribution of the masked-out tokens.  For every query row i, with
+ * s_ij = scale * q_i . k_j over all keys j < N and K(i) the keys of the blocks
+ * that i's query block keeps:
+ *   m_i      = max_j s_ij
+ *   Z_full_i = sum_j exp(s_ij - m_i)
+ *   Z_kept_i = sum_{j in K(i)} exp(s_ij - m_i)
+ *   U_i      = sum_{j not in K(i)} exp(s_ij - m_i) * v_j
+ *   out_i    = sum_j exp(s_ij - m_i) * v_j / Z_full_i       (full attention, bf16)
+ *
+ * q, k, v       bf16 [B,H,N,D] device.
+ * row_ptr, col_idx  CSR of kept blocks (for example from rt_build_block_mask).
+ * out           out, bf16 [B,H,N,D] device.
+ * stat_m, stat_zfull, stat_zkept  out, fp32 [B,H,N] device.
+ * stat_u        out, fp32 [B,H,N,D] device.
+ */
+rt_status rt_attn_full_capture(const rt_shape *shape, const void *q, const void *k, const void *v,
+                               float scale, const int32_t *row_ptr, const int32_t *col_idx,
+                               void *out, float *stat_m, float *stat_zfull, float *stat_zkept,
+                               float *stat_u, rt_stream_t stream);
+
+/*
+ * rt_attn_sparse_reshape -- block-sparse attention with the statistical reshape.
+ *
+ * The Abstract reshapes the sparse attention scores with the prior softmax
+ * distribution history to overcome the normalisation shift of a softmax over
+ * a subset of keys; the mechanism highlight reconstructs the full
+ * distribution from the reused denominator ratio and the cached residual.
+ * For every query row i, over the kept keys K(i) of the current Q, K, V:
+ *   m'_i = max_{j in K(i)} s_ij,  Z'_i = sum_{K(i)} exp(s_ij - m'_i),
+ *   N'_i = sum_{K(i)} exp(s_ij - m'_i) * v_j
+ *   out_i = (N'_i + exp(m_i - m'_i) * U_i) / (Z'_i * Z_full_i / Z_kept_i)
+ * with m, Z_full, Z_kept, U from the latest capture step (same CSR).  If all
+ * four statistics pointers are NULL the call computes plain block-sparse
+ * attention out_i = N'_i / Z'_i.  A row whose query block keeps no key block
+ * gets out_i = 0.
+ *
+ * q, k, v       bf16 [B,H,N,D] device (the current step's inputs).
+ * row_ptr, col_idx  the CSR used at the capture step.
+ * stat_*        fp32 statistics written by rt_attn_full_capture, or all NULL.
+ * out           out, bf16 [B,H,N,D] device.
+ */
+rt_status rt_attn_sparse_reshape(const rt_shape *shape, const void *q, const void *k,
+                                 const void *v, float scale, const int32_t *row_ptr,
+                                 const int32_t *col_idx, const float *stat_m,
+                                 const float *stat_zfull, const float *stat_zkept,
+                                 const float *stat_u, void *out, rt_stream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *rt_status_string(rt_status status);
+
+/* RT_ABI_VERSION of the loaded library. */
+int32_t rt_abi_version(void);
+
+/*
+ * rt_take_device_error -- read and clear the device status word of the
+ * current CUDA device.  Waits for all work on the device to finish first.
+ * *code receives RT_OK or the first error a kernel recorded (RT_ERR_TIMEOUT).
+ * While the word holds an error, this library's kernels return at once
+ * without touching their outputs, so clear it before going on.
+ */
+rt_status rt_take_device_error(int32_t *code);
+
+/*
+ * rt_selftest_wait_timeout -- failure-detection self test.  Launches one
+ * block that waits, bounded by timeout_ns nanoseconds, on a barrier that
+ * nothing completes; the kernel then records RT_ERR_TIMEOUT in the device
+ * status word and returns.  Faults nothing and leaves the context usable.
+ */
+rt_status rt_selftest_wait_timeout(int64_t timeout_ns, rt_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RETTENTION_H */

@@ -1,0 +1,99 @@
+"""The C-ABI library builds for sm_100a, loads, exports what the header
+declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import ultra_sparse_attention_b200 as usa
+from ultra_sparse_attention_b200 import RtShape
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "rettention.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rt_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_three_calls():
+    names = _declared_functions()
+    for n in ("rt_build_block_mask", "rt_attn_full_capture", "rt_attn_sparse_reshape", "rt_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = usa.load_library()
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version():
+    assert usa.rt_abi_version() == 1
+    for code in range(5):
+        s = usa.rt_status_string(code)
+        assert s.startswith("RT_")
+    assert usa.rt_status_string(99) == "unknown rt_status"
+
+
+# Fake, never-dereferenced device addresses: validation must reject before use.
+A16 = ctypes.c_void_p(0x10000)
+A4 = ctypes.c_void_p(0x10004)
+MIS = ctypes.c_void_p(0x10002)
+
+
+def _mask(lib, shape, q=A16, k=A16, scale=0.125, keep=2, forced=0, rp=A16, ci=A16, sc=None):
+    return lib.rt_build_block_mask(ctypes.byref(shape) if shape is not None else None, q, k, scale, keep, forced,
+                                   rp, ci, sc, None)
+
+
+def _sparse(lib, shape, stats=(None, None, None, None), out=A16, scale=0.125):
+    return lib.rt_attn_sparse_reshape(ctypes.byref(shape), A16, A16, A16, scale, A16, A16, *stats, out, None)
+
+
+def _capture(lib, shape, u=A16, m=A16):
+    return lib.rt_attn_full_capture(ctypes.byref(shape), A16, A16, A16, 0.125, A16, A16, A16, m, A16, A16, u,
+                                    None)
+
+
+def test_mask_argument_validation():
+    lib = usa.load_library()
+    ok = RtShape(1, 2, 512, 64, 64, 64)
+    assert _mask(lib, None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _mask(lib, RtShape(1, 2, 512, 64, 96, 64)) == usa.RT_ERR_UNSUPPORTED      # D
+    assert _mask(lib, RtShape(1, 2, 512, 64, 64, 32)) == usa.RT_ERR_UNSUPPORTED      # block size
+    assert _mask(lib, RtShape(1, 2, 512, 81, 80, 64)) == usa.RT_ERR_INVALID_ARGUMENT  # d > D
+    assert _mask(lib, RtShape(0, 2, 512, 64, 64, 64)) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _mask(lib, RtShape(1, 1, 64 * 4097, 64, 64, 64)) == usa.RT_ERR_UNSUPPORTED  # too many blocks
+    assert _mask(lib, ok, q=None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _mask(lib, ok, q=MIS) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _mask(lib, ok, rp=MIS) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _mask(lib, ok, keep=0) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _mask(lib, ok, keep=9) == usa.RT_ERR_INVALID_ARGUMENT                     # > n_blocks
+    assert _mask(lib, ok, keep=2, forced=130) == usa.RT_ERR_INVALID_ARGUMENT          # 3 forced > keep
+    assert _mask(lib, ok, forced=-1) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _mask(lib, ok, scale=0.0) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _mask(lib, ok, scale=float("nan")) == usa.RT_ERR_INVALID_ARGUMENT
+
+
+def test_attention_argument_validation():
+    lib = usa.load_library()
+    ok = RtShape(2, 3, 1000, 72, 80, 64)
+    assert _sparse(lib, ok, stats=(A16, None, None, None)) == usa.RT_ERR_INVALID_ARGUMENT  # partial stats
+    assert _sparse(lib, ok, stats=(A4, A4, A4, A4)) == usa.RT_ERR_INVALID_ARGUMENT        # U misaligned
+    assert _sparse(lib, ok, out=None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _sparse(lib, ok, scale=-1.0) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _sparse(lib, RtShape(2, 3, 1000, 72, 72, 64)) == usa.RT_ERR_UNSUPPORTED
+    assert _capture(lib, ok, u=None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _capture(lib, ok, u=A4) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _capture(lib, ok, m=MIS) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _capture(lib, RtShape(2, 3, 1000, 72, 80, 256)) == usa.RT_ERR_UNSUPPORTED
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        usa.rt_build_block_mask(q, q, head_dim=64, block_size=64, scale=0.125, keep_blocks=1)

@@ -1,0 +1,230 @@
+"""GPU parity: the CUDA path against the fp64 oracle, element by element.
+
+Sizes are chosen so the oracle finishes in seconds while the kernels still
+see several 128-row query tiles, several 64-key tiles and a ragged tail.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ultra_sparse_attention_b200 as usa
+from ultra_sparse_attention_b200.workloads import Workload, denoising_inputs
+
+from parity import (check_mask, compare_out, compare_stats, random_csr, score_tol, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+def _wl(N, d, D, bs, B=2, H=3, std=1.0, seed=0, drift=0.05):
+    return Workload(name="case", batch=B, heads=H, seq_len=N, head_dim=d, head_dim_padded=D, block_size=bs,
+                    keep=(Fraction(1, 4),), forced_prefix_tokens=0, steps=2, capture_every=2, drift_sigma=drift,
+                    kind="iid", iid_std=std, seed=seed)
+
+
+def _inputs(w, device):
+    steps = list(denoising_inputs(w, 2))
+    host = [s[1:] for s in steps]
+    dev = [tuple(x.to(device) for x in s) for s in host]
+    return host, dev
+
+
+def _stats_to_dev(st, shape, device):
+    B, H, N, D = shape
+    u = np.zeros((B * H * N, D))
+    u[:, :st["u"].shape[1]] = st["u"]
+    f = lambda a: torch.as_tensor(a, dtype=torch.float32).reshape(B, H, N).to(device)
+    return usa.Stats(f(st["m"]), f(st["zfull"]), f(st["zkept"]),
+                     torch.as_tensor(u, dtype=torch.float32).reshape(B, H, N, D).to(device))
+
+
+def _abs_v(v):
+    return v.abs()
+
+
+CASES = [
+    # N, d, D, bs
+    (1000, 64, 64, 64),     # 16 blocks, last one 40 tokens; 8 query tiles
+    (1000, 72, 80, 64),
+    (1000, 72, 80, 128),    # 8 blocks, last one 104 tokens
+    (896, 64, 64, 128),     # exact multiple of the block size
+    (200, 64, 64, 64),      # one ragged query tile, odd number of blocks (4: 64,64,64,8)
+]
+
+
+# ------------------------------------------------------------------ mask builder
+@pytest.mark.parametrize("N,d,D,bs", CASES)
+@pytest.mark.parametrize("keep_frac", [Fraction(1, 4), Fraction(1, 1)])
+def test_mask_matches_oracle(cuda_device, N, d, D, bs, keep_frac):
+    w = _wl(N, d, D, bs, std=1.0, seed=N + d)
+    (h0, _), (d0, _) = _inputs(w, cuda_device)
+    nb = w.n_blocks
+    keep = w.keep_blocks(keep_frac)
+    forced = 70 if keep >= 2 else 0
+    rp, ci, sc = usa.rt_build_block_mask(d0[0], d0[1], head_dim=d, block_size=bs, scale=w.scale, keep_blocks=keep,
+                                         forced_prefix_tokens=forced, block_scores=True)
+    torch.cuda.synchronize()
+    _, _, s64 = oracle.build_block_mask(h0[0], h0[1], d, bs, w.scale, keep, forced, return_scores=True)
+    tol = score_tol(s64)
+    s32 = sc.double().cpu().numpy().reshape(s64.shape)
+    assert np.max(np.abs(s32 - s64)) <= tol
+    differ = check_mask(rp.cpu().numpy(), ci.cpu().numpy(), s64, keep, bs, forced, tol)
+    assert differ <= max(1, (w.batch * w.heads * nb) // 100)
+
+
+def test_mask_exact_scores_and_ties_bit_exact(cuda_device):
+    """Inputs whose block scores are exact in fp32 and fp64 (multiples of 2^-k),
+    with duplicated key blocks: the GPU CSR must equal the oracle's everywhere,
+    ties included (lower block index wins)."""
+    B, H, N, d, bs = 1, 2, 1024, 64, 64
+    g = torch.Generator().manual_seed(3)
+    q = (torch.randint(-1, 2, (B, H, N, d), generator=g).float() / 4).to(torch.bfloat16)
+    k = (torch.randint(-1, 2, (B, H, N, d), generator=g).float() / 4).to(torch.bfloat16)
+    k[:, :, 5 * bs:6 * bs] = k[:, :, 3 * bs:4 * bs]      # block 5 duplicates block 3
+    k[:, :, 9 * bs:10 * bs] = k[:, :, 12 * bs:13 * bs]   # block 9 duplicates block 12
+    scale = 0.125
+    for keep, forced in ((1, 0), (3, 0), (4, 64), (7, 130), (16, 0)):
+        rp, ci = usa.rt_build_block_mask(q.to(cuda_device), k.to(cuda_device), head_dim=d, block_size=bs,
+                                         scale=scale, keep_blocks=keep, forced_prefix_tokens=forced)
+        rp_o, ci_o = oracle.build_block_mask(q, k, d, bs, scale, keep, forced)
+        assert np.array_equal(rp.cpu().numpy(), rp_o)
+        assert np.array_equal(ci.cpu().numpy(), ci_o), (keep, forced)
+
+
+# ------------------------------------------------------------------ capture step
+@pytest.mark.parametrize("N,d,D,bs", CASES)
+@pytest.mark.parametrize("keep_frac", [Fraction(1, 4), Fraction(1, 1)])
+def test_capture_matches_oracle(cuda_device, N, d, D, bs, keep_frac):
+    w = _wl(N, d, D, bs, std=1.2, seed=7 * N + d)
+    (h0, _), (d0, _) = _inputs(w, cuda_device)
+    bh, nb = w.batch * w.heads, w.n_blocks
+    keep = w.keep_blocks(keep_frac)
+    rp, ci = random_csr(bh, nb, keep, seed=N)
+    out, st = usa.rt_attn_full_capture(*d0, head_dim=d, block_size=bs, scale=w.scale,
+                                       row_ptr=to_dev(rp, cuda_device), col_idx=to_dev(ci, cuda_device))
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    orc = oracle.full_capture(*h0, d, bs, w.scale, rp, ci)
+    orc_abs = oracle.full_capture(h0[0], h0[1], h0[2].abs(), d, bs, w.scale, rp, ci)["u"]
+    compare_out(out.reshape(-1, D), orc["o"], d, "capture O")
+    compare_stats(st, np.arange(bh * N), orc, orc_abs, d, "capture stats")
+    if keep == nb:
+        assert torch.all(st.u == 0)
+
+
+# ------------------------------------------------------------------ sparse step (oracle mask + oracle stats)
+@pytest.mark.parametrize("N,d,D,bs", CASES)
+@pytest.mark.parametrize("keep_frac", [Fraction(1, 4), Fraction(1, 2)])
+@pytest.mark.parametrize("with_stats", [True, False])
+def test_sparse_matches_oracle(cuda_device, N, d, D, bs, keep_frac, with_stats):
+    w = _wl(N, d, D, bs, std=1.2, seed=11 * N + d, drift=0.05)
+    (h0, h1), (d0, d1) = _inputs(w, cuda_device)
+    bh, nb = w.batch * w.heads, w.n_blocks
+    keep = w.keep_blocks(keep_frac)
+    rp, ci = random_csr(bh, nb, keep, seed=N + 1)
+    st_o = oracle.full_capture(*h0, d, bs, w.scale, rp, ci) if with_stats else None
+    st_d = _stats_to_dev(st_o, d0[0].shape, cuda_device) if with_stats else None
+    out = usa.rt_attn_sparse_reshape(*d1, head_dim=d, block_size=bs, scale=w.scale, row_ptr=to_dev(rp, cuda_device),
+                                     col_idx=to_dev(ci, cuda_device), stats=st_d)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp, ci, st_o)
+    compare_out(out.reshape(-1, D), want, d, "sparse O")
+
+
+# ------------------------------------------------------------------ invariants the pages fix
+@pytest.mark.parametrize("N,d,D,bs", [(1000, 72, 80, 64), (1000, 64, 64, 128)])
+def test_reshape_keep_all_equals_full_attention(cuda_device, N, d, D, bs):
+    """Keep ratio 100%: the reshaped sparse step is full attention of its own inputs."""
+    w = _wl(N, d, D, bs, std=1.2, seed=5, drift=0.2)
+    (h0, h1), (d0, d1) = _inputs(w, cuda_device)
+    nb = w.n_blocks
+    rp, ci = usa.rt_build_block_mask(d0[0], d0[1], head_dim=d, block_size=bs, scale=w.scale, keep_blocks=nb)
+    _, st = usa.rt_attn_full_capture(*d0, head_dim=d, block_size=bs, scale=w.scale, row_ptr=rp, col_idx=ci)
+    out = usa.rt_attn_sparse_reshape(*d1, head_dim=d, block_size=bs, scale=w.scale, row_ptr=rp, col_idx=ci, stats=st)
+    torch.cuda.synchronize()
+    rpo, cio = oracle.build_block_mask(h0[0], h0[1], d, bs, w.scale, nb, 0)
+    want = oracle.full_capture(*h1, d, bs, w.scale, rpo, cio)["o"]
+    compare_out(out.reshape(-1, D), want, d, "keep-all reshape vs full attention")
+
+
+@pytest.mark.parametrize("N,d,D,bs", [(1000, 72, 80, 64), (1000, 64, 64, 128)])
+def test_reshape_unchanged_inputs_recover_capture(cuda_device, N, d, D, bs):
+    """Inputs unchanged since the capture step: reshape recovers full attention at 1/8 keep."""
+    w = _wl(N, d, D, bs, std=1.5, seed=6)
+    (h0, _), (d0, _) = _inputs(w, cuda_device)
+    keep = w.keep_blocks(Fraction(1, 8))
+    rp, ci = usa.rt_build_block_mask(d0[0], d0[1], head_dim=d, block_size=bs, scale=w.scale, keep_blocks=keep)
+    _, st = usa.rt_attn_full_capture(*d0, head_dim=d, block_size=bs, scale=w.scale, row_ptr=rp, col_idx=ci)
+    out = usa.rt_attn_sparse_reshape(*d0, head_dim=d, block_size=bs, scale=w.scale, row_ptr=rp, col_idx=ci, stats=st)
+    torch.cuda.synchronize()
+    want = oracle.full_capture(*h0, d, bs, w.scale, rp.cpu().numpy(), ci.cpu().numpy())["o"]
+    compare_out(out.reshape(-1, D), want, d, "unchanged-input reshape vs capture")
+
+
+def test_sparse_empty_rows_give_zero(cuda_device):
+    N, d, D, bs = 512, 64, 64, 64
+    w = _wl(N, d, D, bs, B=1, H=1, seed=2)
+    (h0, _), (d0, _) = _inputs(w, cuda_device)
+    # query blocks 0 and 5 keep nothing; block 1 keeps nothing while its tile partner 0 also keeps nothing
+    sets = [[], [], [2], [0, 7], [3], [], [6], [1, 2]]
+    rp = np.array([0] + list(np.cumsum([len(s) for s in sets])), np.int32)
+    ci = np.array([x for s in sets for x in s], np.int32)
+    for with_stats in (False, True):
+        st_o = oracle.full_capture(*h0, d, bs, w.scale, rp, ci) if with_stats else None
+        st_d = _stats_to_dev(st_o, d0[0].shape, cuda_device) if with_stats else None
+        out = usa.rt_attn_sparse_reshape(*d0, head_dim=d, block_size=bs, scale=w.scale, row_ptr=to_dev(rp, cuda_device),
+                                         col_idx=to_dev(ci, cuda_device), stats=st_d)
+        torch.cuda.synchronize()
+        want = oracle.sparse_reshape(*h0, d, bs, w.scale, rp, ci, st_o)
+        o = out.reshape(-1, D)
+        assert torch.all(o[:2 * bs] == 0) and torch.all(o[5 * bs:6 * bs] == 0)
+        compare_out(o, want, d, "empty rows")
+
+
+def test_malformed_csr_stays_in_bounds(cuda_device):
+    """Out-of-range and duplicated block indices are skipped; the call completes
+    and writes only its output (checked with canary-padded buffers)."""
+    N, d, D, bs = 256, 64, 64, 64
+    w = _wl(N, d, D, bs, B=1, H=1, seed=4)
+    (_, _), (d0, _) = _inputs(w, cuda_device)
+    ci = np.array([0, 0, 9, -3, 1, 2, 2, 1000, 3], np.int32)
+    rp = np.array([0, 4, 5, 8, 9], np.int32)
+    big = torch.full((3 * N * D,), 7.0, dtype=torch.bfloat16, device=cuda_device)
+    out = big[N * D:2 * N * D].view(1, 1, N, D)
+    usa.rt_attn_sparse_reshape(*d0, head_dim=d, block_size=bs, scale=w.scale, row_ptr=to_dev(rp, cuda_device),
+                               col_idx=to_dev(ci, cuda_device), stats=None, out=out)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    assert torch.all(big[:N * D] == 7.0) and torch.all(big[2 * N * D:] == 7.0)
+    assert torch.isfinite(out.float()).all()
+
+
+# ------------------------------------------------------------------ whole cycle (GPU mask -> capture -> sparse)
+@pytest.mark.parametrize("N,d,D,bs", [(1000, 72, 80, 64), (1000, 72, 80, 128), (1000, 64, 64, 64)])
+def test_denoising_cycle_matches_oracle_chain(cuda_device, N, d, D, bs):
+    w = _wl(N, d, D, bs, std=1.2, seed=9, drift=0.05)
+    (h0, h1), (d0, d1) = _inputs(w, cuda_device)
+    keep = w.keep_blocks(Fraction(1, 4))
+    rp, ci = usa.rt_build_block_mask(d0[0], d0[1], head_dim=d, block_size=bs, scale=w.scale, keep_blocks=keep)
+    o0, st = usa.rt_attn_full_capture(*d0, head_dim=d, block_size=bs, scale=w.scale, row_ptr=rp, col_idx=ci)
+    o1 = usa.rt_attn_sparse_reshape(*d1, head_dim=d, block_size=bs, scale=w.scale, row_ptr=rp, col_idx=ci, stats=st)
+    torch.cuda.synchronize()
+    rpo, cio = oracle.build_block_mask(h0[0], h0[1], d, bs, w.scale, keep, 0)
+    assert np.array_equal(ci.cpu().numpy(), cio)
+    st_o = oracle.full_capture(*h0, d, bs, w.scale, rpo, cio)
+    compare_out(o0.reshape(-1, D), st_o["o"], d, "cycle capture O")
+    want = oracle.sparse_reshape(*h1, d, bs, w.scale, rpo, cio, st_o)
+    compare_out(o1.reshape(-1, D), want, d, "cycle sparse O")
+
+
+def test_timeout_self_test_reports_and_recovers(cuda_device):
+    """A bounded wait that runs out records RT_ERR_TIMEOUT; the context stays usable."""
+    assert usa.rt_take_device_error() == 0
+    usa.rt_selftest_wait_timeout(20_000_000)   # 20 ms
+    assert usa.rt_take_device_error() == usa.RT_ERR_TIMEOUT
+    assert usa.rt_take_device_error() == 0
+    x = torch.ones(4, device=cuda_device)
+    assert float(x.sum()) == 4.0

@@ -1,0 +1,223 @@
+"""Python binding of librettention.so: Re-ttention's attention path on B200.
+
+Argument marshalling only.  Every step of the path (pooling, block scores,
+top-k, full attention with the statistics cache, sparse attention with the
+reshape) runs in the library's CUDA kernels; PyTorch only supplies device
+memory and the current stream.  There is no CPU fallback: if the library
+cannot be built or loaded, every call raises.
+
+The functions carry the C ABI's names (see include/rettention.h):
+
+    rt_build_block_mask(q, k, ...)      -> (row_ptr, col_idx)
+    rt_attn_full_capture(q, k, v, ...)  -> (out, stats)
+    rt_attn_sparse_reshape(q, k, v, ...) -> out
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+from dataclasses import dataclass
+
+import torch
+
+from . import build as _build
+
+__all__ = [
+    "RtError",
+    "Stats",
+    "library_path",
+    "load_library",
+    "rt_build_block_mask",
+    "rt_attn_full_capture",
+    "rt_attn_sparse_reshape",
+    "rt_status_string",
+    "rt_abi_version",
+    "rt_take_device_error",
+    "rt_selftest_wait_timeout",
+]
+
+RT_OK = 0
+RT_ERR_INVALID_ARGUMENT = 1
+RT_ERR_UNSUPPORTED = 2
+RT_ERR_CUDA = 3
+RT_ERR_TIMEOUT = 4
+
+
+class RtError(RuntimeError):
+    """A librettention call returned a status other than RT_OK."""
+
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {rt_status_string(status)}")
+
+
+class RtShape(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_int32) for name in
+                ("batch", "heads", "seq_len", "head_dim", "head_dim_padded", "block_size")]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
+    """Load librettention.so, compiling it first if it is missing or stale."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if build_if_needed:
+                _build.build()
+            lib = ctypes.CDLL(_build.LIB)
+            vp, i32, f32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_int64
+            shp = ctypes.POINTER(RtShape)
+            lib.rt_build_block_mask.argtypes = [shp, vp, vp, f32, i32, i32, vp, vp, vp, vp]
+            lib.rt_attn_full_capture.argtypes = [shp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp]
+            lib.rt_attn_sparse_reshape.argtypes = [shp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp]
+            lib.rt_status_string.argtypes = [ctypes.c_int]
+            lib.rt_status_string.restype = ctypes.c_char_p
+            lib.rt_abi_version.argtypes = []
+            lib.rt_abi_version.restype = i32
+            lib.rt_take_device_error.argtypes = [ctypes.POINTER(i32)]
+            lib.rt_selftest_wait_timeout.argtypes = [i64, vp]
+            for fn in ("rt_build_block_mask", "rt_attn_full_capture", "rt_attn_sparse_reshape",
+                       "rt_take_device_error", "rt_selftest_wait_timeout"):
+                getattr(lib, fn).restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def rt_status_string(status: int) -> str:
+    return load_library().rt_status_string(int(status)).decode()
+
+
+def rt_abi_version() -> int:
+    return int(load_library().rt_abi_version())
+
+
+@dataclass
+class Stats:
+    """Statistics cache of a capture step (fp32, device)."""
+
+    m: torch.Tensor       # [B, H, N]   row max of the scaled scores
+    zfull: torch.Tensor   # [B, H, N]   full softmax denominator
+    zkept: torch.Tensor   # [B, H, N]   kept-key part of it
+    u: torch.Tensor       # [B, H, N, D] masked-out residual numerator
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device: torch.device, stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream))
+
+
+def _check_qkv(name: str, *xs: torch.Tensor) -> tuple[int, int, int, int]:
+    shape = None
+    for x in xs:
+        if not isinstance(x, torch.Tensor) or not x.is_cuda:
+            raise ValueError(f"{name}: Q/K/V must be CUDA tensors")
+        if x.dtype != torch.bfloat16 or x.dim() != 4 or not x.is_contiguous():
+            raise ValueError(f"{name}: Q/K/V must be contiguous bf16 [B, H, N, D]")
+        if shape is None:
+            shape = tuple(x.shape)
+        elif tuple(x.shape) != shape:
+            raise ValueError(f"{name}: Q/K/V shapes differ")
+    return shape
+
+
+def _shape(dims, head_dim: int, block_size: int) -> RtShape:
+    B, H, N, D = dims
+    return RtShape(B, H, N, head_dim, D, block_size)
+
+
+def _call(status: int, what: str):
+    if status != RT_OK:
+        raise RtError(status, what)
+
+
+def rt_build_block_mask(q: torch.Tensor, k: torch.Tensor, *, head_dim: int, block_size: int, scale: float,
+                        keep_blocks: int, forced_prefix_tokens: int = 0, row_ptr: torch.Tensor | None = None,
+                        col_idx: torch.Tensor | None = None, block_scores: torch.Tensor | bool | None = None,
+                        stream=None):
+    """Kept key blocks per query block (CSR).  Returns (row_ptr, col_idx[, block_scores])."""
+    dims = _check_qkv("rt_build_block_mask", q, k)
+    B, H, N, D = dims
+    nb = -(-N // block_size)
+    dev = q.device
+    if row_ptr is None:
+        row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        col_idx = torch.empty(B * H * nb * max(keep_blocks, 0), dtype=torch.int32, device=dev)
+    want_scores = block_scores is True
+    if want_scores:
+        block_scores = torch.empty(B, H, nb, nb, dtype=torch.float32, device=dev)
+    elif block_scores is False:
+        block_scores = None
+    shape = _shape(dims, head_dim, block_size)
+    _call(load_library().rt_build_block_mask(ctypes.byref(shape), _ptr(q), _ptr(k), float(scale), int(keep_blocks),
+                                             int(forced_prefix_tokens), _ptr(row_ptr), _ptr(col_idx),
+                                             _ptr(block_scores), _stream_handle(dev, stream)),
+          "rt_build_block_mask")
+    return (row_ptr, col_idx, block_scores) if want_scores else (row_ptr, col_idx)
+
+
+def rt_attn_full_capture(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, head_dim: int, block_size: int,
+                         scale: float, row_ptr: torch.Tensor, col_idx: torch.Tensor,
+                         out: torch.Tensor | None = None, stats: Stats | None = None, stream=None):
+    """Full attention at a capture step plus the statistics cache.  Returns (out, stats)."""
+    dims = _check_qkv("rt_attn_full_capture", q, k, v)
+    B, H, N, D = dims
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if stats is None:
+        stats = Stats(torch.empty(B, H, N, dtype=torch.float32, device=dev),
+                      torch.empty(B, H, N, dtype=torch.float32, device=dev),
+                      torch.empty(B, H, N, dtype=torch.float32, device=dev),
+                      torch.empty(B, H, N, D, dtype=torch.float32, device=dev))
+    shape = _shape(dims, head_dim, block_size)
+    _call(load_library().rt_attn_full_capture(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale),
+                                              _ptr(row_ptr), _ptr(col_idx), _ptr(out), _ptr(stats.m),
+                                              _ptr(stats.zfull), _ptr(stats.zkept), _ptr(stats.u),
+                                              _stream_handle(dev, stream)),
+          "rt_attn_full_capture")
+    return out, stats
+
+
+def rt_attn_sparse_reshape(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, head_dim: int, block_size: int,
+                           scale: float, row_ptr: torch.Tensor, col_idx: torch.Tensor, stats: Stats | None,
+                           out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Sparse step over the kept blocks, reshaped with ``stats`` (plain block-sparse if None)."""
+    dims = _check_qkv("rt_attn_sparse_reshape", q, k, v)
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    shape = _shape(dims, head_dim, block_size)
+    s = stats
+    _call(load_library().rt_attn_sparse_reshape(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale), _ptr(row_ptr), _ptr(col_idx),
+        _ptr(s.m if s else None), _ptr(s.zfull if s else None), _ptr(s.zkept if s else None),
+        _ptr(s.u if s else None), _ptr(out), _stream_handle(dev, stream)),
+        "rt_attn_sparse_reshape")
+    return out
+
+
+def rt_take_device_error() -> int:
+    """Read and clear the library's device status word (synchronises the device)."""
+    code = ctypes.c_int32(0)
+    _call(load_library().rt_take_device_error(ctypes.byref(code)), "rt_take_device_error")
+    return int(code.value)
+
+
+def rt_selftest_wait_timeout(timeout_ns: int, stream=None):
+    """Launch the bounded-wait self test (records RT_ERR_TIMEOUT in the status word)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _call(load_library().rt_selftest_wait_timeout(int(timeout_ns), _stream_handle(dev, stream)),
+          "rt_selftest_wait_timeout")

@@ -1,0 +1,184 @@
+// mask_builder.cuh -- which key blocks each query block keeps.
+//
+// Re-ttention project page, Abstract: the sparse step attends to "only a
+// subset of tokens or patches" (as few as 3.1%).  The subset rule used here:
+// mean-pool each block of Q and K, score every (query block, key block) pair
+// by the scaled dot product of the pooled vectors, keep the forced prefix
+// blocks plus the best-scoring others, ties to the lower block index, and
+// emit the kept set sorted ascending as a CSR row.
+//
+// Two kernels, both bound by memory or latency, not by arithmetic:
+//   pool_blocks_kernel   reads Q and K once (HBM-bound), writes fp32 block
+//                        means [BH, n_blocks, D] (pad columns zero);
+//   score_select_kernel  one warp per query block: scores against every key
+//                        block from shared memory, then k rounds of a warp
+//                        arg-max with a (score desc, index asc) order, then a
+//                        ballot scan that writes the row sorted ascending.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace rt {
+
+constexpr int kPoolRowGroups = 16;
+
+// grid (n_blocks, B*H, 2): z = 0 pools Q, z = 1 pools K.  D/8 * 16 threads.
+template <int D>
+__global__ void __launch_bounds__(D / 8 * kPoolRowGroups)
+    pool_blocks_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, int N, int d,
+                       int bs, float* __restrict__ pooled_q, float* __restrict__ pooled_k) {
+  constexpr int kChunks = D / 8;  // 16-byte chunks per row
+  __shared__ float partial[kPoolRowGroups][D];
+  __shared__ int skip;
+  if (threadIdx.x == 0) skip = device_status_set() ? 1 : 0;
+  __syncthreads();
+  if (skip) return;  // an earlier kernel failed (block-uniform)
+  const int b = blockIdx.x, bh = blockIdx.y;
+  const __nv_bfloat16* x = blockIdx.z == 0 ? q : k;
+  float* out = blockIdx.z == 0 ? pooled_q : pooled_k;
+  const int n_blocks = gridDim.x;
+  const int row0 = b * bs;
+  const int count = min(bs, N - row0);
+  const int t = threadIdx.x;
+  const int ch = t % kChunks, rg = t / kChunks;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  const uint4* base = reinterpret_cast<const uint4*>(x + (static_cast<size_t>(bh) * N + row0) * D) + ch;
+  for (int r = rg; r < count; r += kPoolRowGroups) {
+    uint4 u = __ldg(base + static_cast<size_t>(r) * kChunks);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] += bf16_lo_to_f32(w[i]);
+      acc[2 * i + 1] += bf16_hi_to_f32(w[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) partial[rg][ch * 8 + i] = acc[i];
+  __syncthreads();
+  for (int c = t; c < D; c += blockDim.x) {
+    float s = 0.f;
+#pragma unroll
+    for (int g = 0; g < kPoolRowGroups; ++g) s += partial[g][c];
+    out[(static_cast<size_t>(bh) * n_blocks + b) * D + c] = c < d ? s / static_cast<float>(count) : 0.f;
+  }
+}
+
+constexpr int kSelWarps = 8;      // query blocks per CTA
+constexpr int kSelChunk = 64;     // key blocks staged in shared memory at a time
+
+__host__ __device__ constexpr int select_words(int n_blocks) { return (n_blocks + 31) / 32; }
+
+template <int D>
+__host__ __device__ constexpr size_t score_select_smem_bytes(int n_blocks) {
+  return sizeof(float) * (static_cast<size_t>(kSelChunk) * (D + 1) + kSelWarps * D +
+                          static_cast<size_t>(kSelWarps) * n_blocks) +
+         sizeof(uint32_t) * kSelWarps * select_words(n_blocks);
+}
+
+// (score, index) order of the selection: higher score first, lower index on ties.
+__device__ __forceinline__ bool sel_better(float sa, int ka, float sb, int kb) {
+  return sa > sb || (sa == sb && ka < kb);
+}
+
+// grid (ceil(n_blocks / kSelWarps), B*H), 32*kSelWarps threads.
+template <int D>
+__global__ void __launch_bounds__(32 * kSelWarps)
+    score_select_kernel(const float* __restrict__ pooled_q, const float* __restrict__ pooled_k, int n_blocks,
+                        int bs, float scale, int keep, int forced_tokens, int32_t* __restrict__ row_ptr,
+                        int32_t* __restrict__ col_idx, float* __restrict__ block_scores) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* pk = reinterpret_cast<float*>(smem_raw);                 // [kSelChunk][D+1]
+  float* pq = pk + kSelChunk * (D + 1);                           // [kSelWarps][D]
+  float* sc = pq + kSelWarps * D;                                 // [kSelWarps][n_blocks]
+  uint32_t* taken = reinterpret_cast<uint32_t*>(sc + kSelWarps * n_blocks);  // [kSelWarps][words]
+  __shared__ int skip;
+  if (threadIdx.x == 0) skip = device_status_set() ? 1 : 0;
+  __syncthreads();
+  if (skip) return;  // an earlier kernel failed (block-uniform)
+
+  const int bh = blockIdx.y;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int qb = blockIdx.x * kSelWarps + warp;
+  const bool have_row = qb < n_blocks;
+  const int words = select_words(n_blocks);
+  const size_t head = static_cast<size_t>(bh) * n_blocks;
+
+  for (int i = threadIdx.x; i < kSelWarps * D; i += blockDim.x) {
+    const int w = i / D, c = i % D;
+    const int qq = blockIdx.x * kSelWarps + w;
+    pq[i] = qq < n_blocks ? pooled_q[(head + qq) * D + c] : 0.f;
+  }
+  for (int i = threadIdx.x; i < kSelWarps * words; i += blockDim.x) taken[i] = 0u;
+
+  float* my_sc = sc + warp * n_blocks;
+  for (int kb0 = 0; kb0 < n_blocks; kb0 += kSelChunk) {
+    __syncthreads();
+    const int nch = min(kSelChunk, n_blocks - kb0);
+    for (int i = threadIdx.x; i < nch * D; i += blockDim.x) {
+      const int r = i / D, c = i % D;
+      pk[r * (D + 1) + c] = pooled_k[(head + kb0 + r) * D + c];
+    }
+    __syncthreads();
+    if (have_row) {
+      const float* a = pq + warp * D;
+      for (int r = lane; r < nch; r += 32) {
+        const float* b = pk + r * (D + 1);
+        float acc = 0.f;
+#pragma unroll 16
+        for (int c = 0; c < D; ++c) acc = fmaf(a[c], b[c], acc);
+        float s = scale * acc;
+        if (s != s) s = -INFINITY;  // a NaN never wins
+        my_sc[kb0 + r] = s;
+      }
+    }
+  }
+  __syncwarp();
+  if (!have_row) return;
+
+  uint32_t* my_taken = taken + warp * words;
+  const int forced = min(n_blocks, forced_tokens > 0 ? (forced_tokens + bs - 1) / bs : 0);
+  for (int kb = lane; kb < forced; kb += 32) atomicOr(&my_taken[kb / 32], 1u << (kb % 32));
+  __syncwarp();
+  for (int round = forced; round < keep; ++round) {
+    float best_s = -INFINITY;
+    int best_k = n_blocks;  // sentinel: loses to every real block
+    for (int kb = forced + lane; kb < n_blocks; kb += 32) {
+      if ((my_taken[kb / 32] >> (kb % 32)) & 1u) continue;
+      const float s = my_sc[kb];
+      if (sel_better(s, kb, best_s, best_k)) { best_s = s; best_k = kb; }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float os = __shfl_xor_sync(0xffffffffu, best_s, off);
+      const int ok = __shfl_xor_sync(0xffffffffu, best_k, off);
+      if (sel_better(os, ok, best_s, best_k)) { best_s = os; best_k = ok; }
+    }
+    if (lane == 0 && best_k < n_blocks) my_taken[best_k / 32] |= 1u << (best_k % 32);
+    __syncwarp();
+  }
+
+  const size_t row = head + qb;
+  int32_t* out = col_idx + row * keep;
+  int written = 0;
+  for (int base = 0; base < n_blocks; base += 32) {
+    const int kb = base + lane;
+    const bool t = kb < n_blocks && ((my_taken[kb / 32] >> (kb % 32)) & 1u);
+    const uint32_t mask = __ballot_sync(0xffffffffu, t);
+    const int pos = written + __popc(mask & ((1u << lane) - 1u));
+    if (t && pos < keep) out[pos] = kb;
+    written += __popc(mask);
+  }
+  if (lane == 0) {
+    row_ptr[row] = static_cast<int32_t>(row * keep);
+    if (row + 1 == static_cast<size_t>(gridDim.y) * n_blocks)
+      row_ptr[row + 1] = static_cast<int32_t>((row + 1) * keep);
+  }
+  if (block_scores != nullptr)
+    for (int kb = lane; kb < n_blocks; kb += 32) block_scores[row * n_blocks + kb] = my_sc[kb];
+}
+
+}  // namespace rt

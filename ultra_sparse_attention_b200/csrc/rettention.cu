@@ -1,0 +1,287 @@
+// rettention.cu -- host side of the C ABI declared in include/rettention.h.
+//
+// Validates every argument before touching CUDA, encodes the TMA tensor maps,
+// and launches the kernels of mask_builder.cuh and attention.cuh on the
+// caller's stream.  All kernels live in this one translation unit so that the
+// device status word is a single symbol of one module.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "rettention.h"
+#include "ptx.cuh"
+#include "mask_builder.cuh"
+#include "attention.cuh"
+
+namespace {
+
+using rt::AttnArgs;
+
+constexpr int kMaxBlocks = 2048;
+
+// ------------------------------------------------------------------ validation
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Dims {
+  int64_t B, H, N, d, D, bs, n_blocks, bh;
+};
+
+rt_status check_shape(const rt_shape* s, Dims* out) {
+  if (s == nullptr) return RT_ERR_INVALID_ARGUMENT;
+  if (s->batch <= 0 || s->heads <= 0 || s->seq_len <= 0 || s->head_dim <= 0 || s->head_dim_padded <= 0 ||
+      s->block_size <= 0)
+    return RT_ERR_INVALID_ARGUMENT;
+  if (s->head_dim > s->head_dim_padded) return RT_ERR_INVALID_ARGUMENT;
+  if (s->head_dim_padded != 64 && s->head_dim_padded != 80) return RT_ERR_UNSUPPORTED;
+  if (s->block_size != 64 && s->block_size != 128) return RT_ERR_UNSUPPORTED;
+  Dims d;
+  d.B = s->batch;
+  d.H = s->heads;
+  d.N = s->seq_len;
+  d.d = s->head_dim;
+  d.D = s->head_dim_padded;
+  d.bs = s->block_size;
+  d.n_blocks = (d.N + d.bs - 1) / d.bs;
+  d.bh = d.B * d.H;
+  if (d.n_blocks > kMaxBlocks) return RT_ERR_UNSUPPORTED;
+  if (d.bh > 65535) return RT_ERR_UNSUPPORTED;                 // grid.y
+  if (d.bh * d.N > (int64_t(1) << 31) - 1) return RT_ERR_UNSUPPORTED;  // row ids stay in int32 range
+  *out = d;
+  return RT_OK;
+}
+
+bool scale_ok(float scale) { return std::isfinite(scale) && scale > 0.f; }
+
+// ------------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor [bh][N][D] viewed as 3-D (D, N, bh); box of `box_cols` x `box_rows` x 1.
+bool make_map(CUtensorMap* m, const void* base, const Dims& d, int box_cols, int box_rows, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d.D), static_cast<cuuint64_t>(d.N), static_cast<cuuint64_t>(d.bh)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d.D * 2), static_cast<cuuint64_t>(d.N * d.D * 2)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct Maps {
+  CUtensorMap q, q_tail, k, k_tail, v, v_tail;
+};
+
+bool make_maps(Maps* m, const Dims& d, const void* q, const void* k, const void* v) {
+  std::memset(m, 0, sizeof(*m));
+  bool ok = make_map(&m->q, q, d, 64, rt::kBM, true) && make_map(&m->k, k, d, 64, rt::kBN, true) &&
+            make_map(&m->v, v, d, 64, rt::kBN, true);
+  if (d.D == 80)
+    ok = ok && make_map(&m->q_tail, q, d, 16, rt::kBM, false) && make_map(&m->k_tail, k, d, 16, rt::kBN, false) &&
+         make_map(&m->v_tail, v, d, 16, rt::kBN, false);
+  else {
+    m->q_tail = m->q;
+    m->k_tail = m->k;
+    m->v_tail = m->v;
+  }
+  return ok;
+}
+
+rt_status launch_status() { return cudaGetLastError() == cudaSuccess ? RT_OK : RT_ERR_CUDA; }
+
+// ------------------------------------------------------------------ attention launch
+template <int D, int BS, bool kCapture>
+rt_status launch_attention(const Dims& d, const Maps& m, const AttnArgs& a, cudaStream_t stream) {
+  const int n_key_tiles = static_cast<int>((d.N + rt::kBN - 1) / rt::kBN);
+  size_t smem = rt::attn_smem_bytes<D>(static_cast<int>(d.n_blocks), n_key_tiles);
+  auto kernel = kCapture ? rt::full_capture_kernel<D, BS> : rt::sparse_reshape_kernel<D, BS>;
+  // The capture kernel holds all 512 TMEM columns: ask for enough shared
+  // memory that a second block can never share its SM.
+  if (kCapture && smem < 120 * 1024) smem = 120 * 1024;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return RT_ERR_CUDA;
+  dim3 grid(static_cast<unsigned>((d.N + rt::kBM - 1) / rt::kBM), static_cast<unsigned>(d.bh));
+  kernel<<<grid, rt::kAttnThreads, smem, stream>>>(m.q, m.q_tail, m.k, m.k_tail, m.v, m.v_tail, a);
+  return launch_status();
+}
+
+template <bool kCapture>
+rt_status dispatch_attention(const Dims& d, const Maps& m, const AttnArgs& a, cudaStream_t s) {
+  if (d.D == 64 && d.bs == 64) return launch_attention<64, 64, kCapture>(d, m, a, s);
+  if (d.D == 64 && d.bs == 128) return launch_attention<64, 128, kCapture>(d, m, a, s);
+  if (d.D == 80 && d.bs == 64) return launch_attention<80, 64, kCapture>(d, m, a, s);
+  if (d.D == 80 && d.bs == 128) return launch_attention<80, 128, kCapture>(d, m, a, s);
+  return RT_ERR_UNSUPPORTED;
+}
+
+// ------------------------------------------------------------------ mask launch
+template <int D>
+rt_status launch_mask(const Dims& d, const void* q, const void* k, float scale, int keep, int forced,
+                      int32_t* row_ptr, int32_t* col_idx, float* scores, float* pooled, cudaStream_t stream) {
+  float* pq = pooled;
+  float* pk = pooled + d.bh * d.n_blocks * D;
+  constexpr int kPoolThreads = D / 8 * rt::kPoolRowGroups;
+  dim3 pgrid(static_cast<unsigned>(d.n_blocks), static_cast<unsigned>(d.bh), 2);
+  rt::pool_blocks_kernel<D><<<pgrid, kPoolThreads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), static_cast<int>(d.N),
+      static_cast<int>(d.d), static_cast<int>(d.bs), pq, pk);
+  if (launch_status() != RT_OK) return RT_ERR_CUDA;
+  const size_t smem = rt::score_select_smem_bytes<D>(static_cast<int>(d.n_blocks));
+  if (cudaFuncSetAttribute(rt::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return RT_ERR_CUDA;
+  dim3 sgrid(static_cast<unsigned>((d.n_blocks + rt::kSelWarps - 1) / rt::kSelWarps), static_cast<unsigned>(d.bh));
+  rt::score_select_kernel<D><<<sgrid, 32 * rt::kSelWarps, smem, stream>>>(
+      pq, pk, static_cast<int>(d.n_blocks), static_cast<int>(d.bs), scale, keep, forced, row_ptr, col_idx, scores);
+  return launch_status();
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* rt_status_string(rt_status status) {
+  switch (status) {
+    case RT_OK: return "RT_OK";
+    case RT_ERR_INVALID_ARGUMENT: return "RT_ERR_INVALID_ARGUMENT: bad pointer, size, keep count or alignment";
+    case RT_ERR_UNSUPPORTED: return "RT_ERR_UNSUPPORTED: head dim, block size or size outside the supported set";
+    case RT_ERR_CUDA: return "RT_ERR_CUDA: a CUDA call or kernel launch failed";
+    case RT_ERR_TIMEOUT: return "RT_ERR_TIMEOUT: a kernel wait ran out and the kernel stopped";
+  }
+  return "unknown rt_status";
+}
+
+int32_t rt_abi_version(void) { return RT_ABI_VERSION; }
+
+rt_status rt_build_block_mask(const rt_shape* shape, const void* q, const void* k, float scale, int32_t keep_blocks,
+                              int32_t forced_prefix_tokens, int32_t* row_ptr, int32_t* col_idx, float* block_scores,
+                              rt_stream_t stream) {
+  Dims d;
+  rt_status st = check_shape(shape, &d);
+  if (st != RT_OK) return st;
+  if (!q || !k || !row_ptr || !col_idx) return RT_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(row_ptr, 4) || !aligned(col_idx, 4) ||
+      !aligned(block_scores, 4))
+    return RT_ERR_INVALID_ARGUMENT;
+  if (!scale_ok(scale) || forced_prefix_tokens < 0) return RT_ERR_INVALID_ARGUMENT;
+  if (keep_blocks < 1 || keep_blocks > d.n_blocks) return RT_ERR_INVALID_ARGUMENT;
+  const int64_t forced = std::min<int64_t>(d.n_blocks, (int64_t(forced_prefix_tokens) + d.bs - 1) / d.bs);
+  if (forced > keep_blocks) return RT_ERR_INVALID_ARGUMENT;
+  if (d.bh * d.n_blocks * keep_blocks > (int64_t(1) << 31) - 1) return RT_ERR_UNSUPPORTED;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* pooled = nullptr;
+  const size_t bytes = sizeof(float) * 2 * d.bh * d.n_blocks * d.D;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&pooled), bytes, s) != cudaSuccess) return RT_ERR_CUDA;
+  st = d.D == 64 ? launch_mask<64>(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx,
+                                    block_scores, pooled, s)
+                 : launch_mask<80>(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx,
+                                    block_scores, pooled, s);
+  if (cudaFreeAsync(pooled, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
+  return st;
+}
+
+rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void* k, const void* v, float scale,
+                               const int32_t* row_ptr, const int32_t* col_idx, void* out, float* stat_m,
+                               float* stat_zfull, float* stat_zkept, float* stat_u, rt_stream_t stream) {
+  Dims d;
+  rt_status st = check_shape(shape, &d);
+  if (st != RT_OK) return st;
+  if (!q || !k || !v || !row_ptr || !col_idx || !out || !stat_m || !stat_zfull || !stat_zkept || !stat_u)
+    return RT_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(stat_u, 16) ||
+      !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(stat_m, 4) || !aligned(stat_zfull, 4) ||
+      !aligned(stat_zkept, 4))
+    return RT_ERR_INVALID_ARGUMENT;
+  if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
+  Maps m;
+  if (!make_maps(&m, d, q, k, v)) return RT_ERR_CUDA;
+  AttnArgs a{};
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.out_m = stat_m;
+  a.out_zfull = stat_zfull;
+  a.out_zkept = stat_zkept;
+  a.out_u = stat_u;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.N = static_cast<int>(d.N);
+  a.d = static_cast<int>(d.d);
+  a.n_blocks = static_cast<int>(d.n_blocks);
+  a.scale_log2 = scale * rt::kLog2e;
+  return dispatch_attention<true>(d, m, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+rt_status rt_attn_sparse_reshape(const rt_shape* shape, const void* q, const void* k, const void* v, float scale,
+                                 const int32_t* row_ptr, const int32_t* col_idx, const float* stat_m,
+                                 const float* stat_zfull, const float* stat_zkept, const float* stat_u, void* out,
+                                 rt_stream_t stream) {
+  Dims d;
+  rt_status st = check_shape(shape, &d);
+  if (st != RT_OK) return st;
+  if (!q || !k || !v || !row_ptr || !col_idx || !out) return RT_ERR_INVALID_ARGUMENT;
+  const int nstats = (stat_m != nullptr) + (stat_zfull != nullptr) + (stat_zkept != nullptr) + (stat_u != nullptr);
+  if (nstats != 0 && nstats != 4) return RT_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(stat_u, 16) ||
+      !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(stat_m, 4) || !aligned(stat_zfull, 4) ||
+      !aligned(stat_zkept, 4))
+    return RT_ERR_INVALID_ARGUMENT;
+  if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
+  Maps m;
+  if (!make_maps(&m, d, q, k, v)) return RT_ERR_CUDA;
+  AttnArgs a{};
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.stat_m = stat_m;
+  a.stat_zfull = stat_zfull;
+  a.stat_zkept = stat_zkept;
+  a.stat_u = stat_u;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.N = static_cast<int>(d.N);
+  a.d = static_cast<int>(d.d);
+  a.n_blocks = static_cast<int>(d.n_blocks);
+  a.scale_log2 = scale * rt::kLog2e;
+  return dispatch_attention<false>(d, m, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+rt_status rt_take_device_error(int32_t* code) {
+  if (code == nullptr) return RT_ERR_INVALID_ARGUMENT;
+  if (cudaDeviceSynchronize() != cudaSuccess) return RT_ERR_CUDA;
+  int32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, rt::g_device_status, sizeof(v)) != cudaSuccess) return RT_ERR_CUDA;
+  if (cudaMemcpyToSymbol(rt::g_device_status, &zero, sizeof(zero)) != cudaSuccess) return RT_ERR_CUDA;
+  *code = v;
+  return RT_OK;
+}
+
+rt_status rt_selftest_wait_timeout(int64_t timeout_ns, rt_stream_t stream) {
+  if (timeout_ns <= 0 || timeout_ns > 10000000000ll) return RT_ERR_INVALID_ARGUMENT;
+  rt::wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(timeout_ns));
+  return launch_status();
+}
+
+}  // extern "C"
