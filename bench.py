@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Benchmark of Re-ttention's attention path on B200.
+
+One step is one pass of the whole hot path on one batch of synthetic input:
+the capture step at t0 (block mask from Q0/K0, then full attention with the
+statistics cache) followed by the sparse step at t1 (kept blocks only, with
+the reshape) on drifted Q1/K1/V1 -- the video-DiT 5B workload's "one sparse
+step after a full-capture step".
+
+The headline metric is the sparse step: its device time, its dense-equivalent
+TFLOP/s (4*B*H*N^2*d over the sparse-step time) and the tensor-pipe share of
+the bf16 peak on the flops it executes.  ``value`` is the dense-equivalent
+TFLOP/s of the sparse step summed over all ranks (each rank runs one replica;
+weak scaling).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from ultra_sparse_attention_b200.workloads import WORKLOADS, denoising_inputs  # noqa: E402
+
+METRIC = "sparse-step ms & dense-equiv TFLOP/s; tensor-pipe % of BF16 peak (1xB200)"
+UNIT = "TFLOP/s (dense-equivalent, sparse step)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=60)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--workload", default="video5b", choices=sorted(WORKLOADS))
+    p.add_argument("--keep", default=None, help="keep ratio as a fraction, e.g. 1/32 (default: the workload's)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-rows", type=int, default=4096, help="rows in the oracle's bounded sample")
+    return p.parse_args()
+
+
+# --------------------------------------------------------------------------- plumbing
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.proc = None
+        self.gpu = gpu_index
+        self.period = period_ms
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", str(self.period)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def stored_traffic(kernel: str, workload: str):
+    """dram bytes per launch from the committed ncu summary, if it matches the current sources."""
+    from ultra_sparse_attention_b200 import build as _b
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    cur = _b.source_hash()
+    for ln in lines:
+        if ln.startswith("#") or "=" not in ln:
+            continue
+        kv = dict(x.split("=", 1) for x in ln.split())
+        if kv.get("kernel") == kernel and kv.get("workload") == workload and kv.get("src_hash") == cur:
+            return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+# --------------------------------------------------------------------------- work accounting
+def kept_work(row_ptr: np.ndarray, col_idx: np.ndarray, N: int, bs: int, bh: int):
+    """Executed sparse-step flop factor: sum over query blocks of rows(qb) * kept key columns."""
+    nb = -(-N // bs)
+    sizes = np.minimum(bs, N - np.arange(nb) * bs).astype(np.int64)
+    total = 0
+    for r in range(bh * nb):
+        kept = col_idx[row_ptr[r]:row_ptr[r + 1]]
+        total += int(sizes[r % nb]) * int(sizes[kept].sum())
+    return total
+
+
+def workload_numbers(w, keep: int, row_ptr, col_idx):
+    B, H, N, d, D = w.batch, w.heads, w.seq_len, w.head_dim, w.head_dim_padded
+    bh = B * H
+    dense = 4.0 * bh * N * N * d
+    executed = 4.0 * d * kept_work(row_ptr, col_idx, N, w.block_size, bh)
+    sparse_bytes = bh * N * (D * 2 * 2 + D * 4 + 12) + 2 * bh * N * D * 2  # Q, O, U, stats; K and V once
+    capture_bytes = 3 * bh * N * D * 2 + bh * N * (D * 2 + D * 4 + 12)     # Q, K, V; O, U, stats
+    mask_bytes = 2 * bh * N * D * 2                                       # Q and K read once
+    return {"dense_flops": dense, "executed_flops": executed, "sparse_bytes": sparse_bytes,
+            "capture_bytes": capture_bytes, "mask_bytes": mask_bytes}
+
+
+# --------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local):
+    import ultra_sparse_attention_b200 as usa
+
+    w = WORKLOADS[args.workload]
+    keep_ratio = Fraction(args.keep) if args.keep else w.keep[0]
+    keep = w.keep_blocks(keep_ratio)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    usa.load_library()
+    steps = list(denoising_inputs(w, 2))
+    host0, host1 = steps[0][1:], steps[1][1:]
+    q0, k0, v0 = (x.to(device) for x in host0)
+    q1, k1, v1 = (x.to(device) for x in host1)
+    kw = dict(head_dim=w.head_dim, block_size=w.block_size, scale=w.scale)
+    B, H, N, D = q0.shape
+    nb = w.n_blocks
+    row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=device)
+    col_idx = torch.empty(B * H * nb * keep, dtype=torch.int32, device=device)
+    out0, out1 = torch.empty_like(q0), torch.empty_like(q1)
+    stats = usa.Stats(torch.empty(B, H, N, device=device), torch.empty(B, H, N, device=device),
+                      torch.empty(B, H, N, device=device), torch.empty(B, H, N, D, device=device))
+    stream = torch.cuda.current_stream(device)
+    ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(2)] for k in ("mask", "capture", "sparse")}
+    times = {k: [] for k in ev}
+
+    def step(record: bool):
+        def mark(name, i):
+            if record:
+                ev[name][i].record(stream)
+        mark("mask", 0)
+        usa.rt_build_block_mask(q0, k0, keep_blocks=keep, forced_prefix_tokens=w.forced_prefix_tokens,
+                                row_ptr=row_ptr, col_idx=col_idx, **kw)
+        mark("mask", 1)
+        mark("capture", 0)
+        usa.rt_attn_full_capture(q0, k0, v0, row_ptr=row_ptr, col_idx=col_idx, out=out0, stats=stats, **kw)
+        mark("capture", 1)
+        mark("sparse", 0)
+        usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=row_ptr, col_idx=col_idx, stats=stats, out=out1, **kw)
+        mark("sparse", 1)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    if usa.rt_take_device_error() != 0:
+        raise RuntimeError("a kernel reported a device error during warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step(True)
+        # per-kernel durations are read after the loop; keep the events of every step
+        for k in ev:
+            times[k].append((ev[k][0], ev[k][1]))
+            ev[k] = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    per_kernel = {k: statistics.mean(a.elapsed_time(b) for a, b in times[k]) for k in times}
+    if usa.rt_take_device_error() != 0:
+        raise RuntimeError("a kernel reported a device error in the timed region")
+
+    rp, ci = row_ptr.cpu().numpy(), col_idx.cpu().numpy()
+    nums = workload_numbers(w, keep, rp, ci)
+
+    # e2e: the sparse step through the public API with host buffers (pinned), copies inside.
+    e2e = None
+    if not args.no_e2e:
+        h_in = [x.pin_memory() for x in host1]
+        h_out = torch.empty(out1.shape, dtype=out1.dtype, pin_memory=True)
+        d_in = [torch.empty_like(x, device=device) for x in host1]
+        for it in range(args.warmup + args.steps):
+            if it == args.warmup:
+                barrier()
+                torch.cuda.synchronize()
+                e_start = torch.cuda.Event(enable_timing=True)
+                e_end = torch.cuda.Event(enable_timing=True)
+                e_start.record(stream)
+            for dx, hx in zip(d_in, h_in):
+                dx.copy_(hx, non_blocking=True)
+            usa.rt_attn_sparse_reshape(*d_in, row_ptr=row_ptr, col_idx=col_idx, stats=stats, out=out1, **kw)
+            h_out.copy_(out1, non_blocking=True)
+        e_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = e_start.elapsed_time(e_end) / args.steps
+        e2e = {"ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in h_in)),
+               "d2h_bytes_per_step": int(h_out.numel() * h_out.element_size())}
+
+    # max over ranks of every time
+    vals = torch.tensor([total_ms, per_kernel["mask"], per_kernel["capture"], per_kernel["sparse"],
+                         e2e["ms_per_step"] if e2e else 0.0], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    total_ms, mask_ms, cap_ms, sp_ms, e2e_ms = vals.tolist()
+    return {"w": w, "keep": keep, "keep_ratio": keep_ratio, "total_ms": total_ms, "mask_ms": mask_ms,
+            "capture_ms": cap_ms, "sparse_ms": sp_ms, "e2e": e2e, "e2e_ms": e2e_ms, "clocks": clk, "nums": nums,
+            "host1": host1, "host0": host0}
+
+
+# --------------------------------------------------------------------------- oracle timing (CPU)
+class OracleSample:
+    """The fp64 oracle's sparse step on a bounded row sample of the workload.
+
+    Its block mask and the capture statistics of the sampled rows are computed
+    once, untimed; ``time_step`` then times one sparse step with the reshape."""
+
+    def __init__(self, w, keep: int, host0, host1, rows: int, seed: int = 0):
+        import oracle
+        self.oracle, self.w, self.keep, self.host1 = oracle, w, keep, host1
+        d, bs = w.head_dim, w.block_size
+        self.rp, self.ci = oracle.build_block_mask(host0[0], host0[1], d, bs, w.scale, keep, w.forced_prefix_tokens)
+        rng = np.random.default_rng(seed)
+        total = w.batch * w.heads * w.seq_len
+        self.rows = np.sort(rng.choice(total, size=min(rows, total), replace=False)).astype(np.int64)
+        self.threads = oracle.default_threads()
+        self.stats = oracle.full_capture(*host0, d, bs, w.scale, self.rp, self.ci, rows=self.rows, threads=self.threads)
+        self.dense_flops = 4.0 * w.seq_len * d * len(self.rows)
+        self.desc = (f"{len(self.rows)} query rows sampled uniformly (seed {seed}) of {total} of {w.name} at keep "
+                     f"{keep}/{w.n_blocks}: fp64 oracle sparse step with reshape on {self.threads} threads; its mask "
+                     f"and the capture statistics of those rows computed beforehand, untimed")
+
+    def time_step(self) -> float:
+        w = self.w
+        t0 = time.perf_counter()
+        self.oracle.sparse_reshape(*self.host1, w.head_dim, w.block_size, w.scale, self.rp, self.ci, self.stats,
+                                   rows=self.rows, threads=self.threads)
+        return time.perf_counter() - t0
+
+    def baseline(self, repeats: int = 3) -> dict:
+        secs = min(self.time_step() for _ in range(repeats))
+        return {"value": self.dense_flops / secs / 1e12, "unit": UNIT, "cores": self.threads, "kind": "oracle",
+                "sample": self.desc}
+
+
+def run_reference(args, rank, world):
+    """The base contract's reference arm: the fp64 oracle on the host cores."""
+    if rank != 0:
+        return None
+    w = WORKLOADS[args.workload]
+    keep_ratio = Fraction(args.keep) if args.keep else w.keep[0]
+    keep = w.keep_blocks(keep_ratio)
+    steps = list(denoising_inputs(w, 2))
+    sample = OracleSample(w, keep, steps[0][1:], steps[1][1:], args.cpu_rows)
+    for _ in range(args.warmup):
+        sample.time_step()
+    secs = sum(sample.time_step() for _ in range(args.steps))
+    value = sample.dense_flops * args.steps / secs / 1e12
+    cpu = {"value": value, "unit": UNIT, "cores": sample.threads, "kind": "oracle", "sample": sample.desc}
+    return {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _config(w, keep, keep_ratio, args.gpus),
+            "cpu_baseline": cpu, "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                                         "d2h_bytes_per_step": 0}}
+
+
+def _config(w, keep, keep_ratio, gpus):
+    return {"workload": (f"{w.name}: B={w.batch} H={w.heads} N={w.seq_len} d={w.head_dim} D={w.head_dim_padded} "
+                         f"block={w.block_size} keep={keep}/{w.n_blocks} ({keep_ratio})"),
+            "step": "mask + full capture at t0, sparse reshape at t1 (drifted inputs)",
+            "forced_prefix_tokens": w.forced_prefix_tokens,
+            "l2": "inputs larger than L2 (about 1.1 GB touched per step; no flush)",
+            "parallelism": f"replicas x{gpus}"}
+
+
+# --------------------------------------------------------------------------- main
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                             device_id=torch.device("cuda", local))
+    try:
+        r = run_ours(args, rank, world, local)
+    finally:
+        pass
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        w, nums = r["w"], r["nums"]
+        sp_s = r["sparse_ms"] / 1e3
+        value = world * nums["dense_flops"] / sp_s / 1e12
+        exec_tflops = nums["executed_flops"] / sp_s / 1e12
+        cap_tflops = nums["dense_flops"] / (r["capture_ms"] / 1e3) / 1e12
+        kernels = {
+            "rt_build_block_mask": {"ms": r["mask_ms"], "bound": "hbm",
+                                    "achieved_gbs": nums["mask_bytes"] / (r["mask_ms"] / 1e3) / 1e9},
+            "rt_attn_full_capture": {"ms": r["capture_ms"], "bound": "tensor", "achieved_tflops": cap_tflops,
+                                     "algorithmic_tflop": nums["dense_flops"] / 1e12,
+                                     "achieved_gbs": nums["capture_bytes"] / (r["capture_ms"] / 1e3) / 1e9},
+            "rt_attn_sparse_reshape": {"ms": r["sparse_ms"], "bound": "tensor+hbm",
+                                       "executed_tflops": exec_tflops,
+                                       "executed_tflop": nums["executed_flops"] / 1e12,
+                                       "dense_equiv_tflops": nums["dense_flops"] / sp_s / 1e12,
+                                       "tensor_frac_of_bf16_peak": exec_tflops / peaks["bf16_tflops"],
+                                       "achieved_gbs": nums["sparse_bytes"] / sp_s / 1e9,
+                                       "hbm_frac": nums["sparse_bytes"] / sp_s / 1e9 / peaks["hbm_gbs"],
+                                       "algorithmic_bytes": nums["sparse_bytes"]},
+        }
+        # dominant kernel of the step (by device time)
+        dom = max(("rt_attn_full_capture", r["capture_ms"]), ("rt_attn_sparse_reshape", r["sparse_ms"]),
+                  ("rt_build_block_mask", r["mask_ms"]), key=lambda t: t[1])[0]
+        wl_tag = f"{w.name}@{r['keep']}"
+        if dom == "rt_attn_full_capture":
+            ach = cap_tflops
+            roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                    "traffic": stored_traffic("full_capture_kernel", wl_tag),
+                    "peak_source": f"bf16_tflops ({peak_src}, burst)",
+                    "per_launch": f"{nums['dense_flops'] / 1e12:.3f} TFLOP algorithmic (4*B*H*N^2*d)"}
+        elif dom == "rt_attn_sparse_reshape":
+            ach = exec_tflops
+            roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                    "traffic": stored_traffic("sparse_reshape_kernel", wl_tag),
+                    "peak_source": f"bf16_tflops ({peak_src}, burst)"}
+        else:
+            ach = kernels["rt_build_block_mask"]["achieved_gbs"]
+            roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": f"hbm_gbs ({peak_src})"}
+        e2e = None
+        if r["e2e"]:
+            e2e = {"value": world * nums["dense_flops"] / (r["e2e_ms"] / 1e3) / 1e12, "unit": UNIT,
+                   "ms_per_step": r["e2e_ms"], "h2d_bytes_per_step": r["e2e"]["h2d_bytes_per_step"],
+                   "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"],
+                   "what": "sparse step through the public API: pinned host Q1/K1/V1 -> device, "
+                           "rt_attn_sparse_reshape, output -> pinned host"}
+        cpu = None
+        if not args.no_cpu_baseline and world >= 1:
+            cpu = OracleSample(w, r["keep"], r["host0"], r["host1"], args.cpu_rows).baseline()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": r["total_ms"] / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": _config(w, r["keep"], r["keep_ratio"], world),
+            "sparse_step_ms": r["sparse_ms"], "full_step_ms": r["mask_ms"] + r["capture_ms"],
+            "dense_equiv_tflops": nums["dense_flops"] / sp_s / 1e12, "executed_tflops": exec_tflops,
+            "tensor_pct_of_bf16_peak": 100.0 * exec_tflops / peaks["bf16_tflops"],
+            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 4 * args.steps, "clocks": r["clocks"],
+            "peaks": {**peaks, "source": peak_src},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
