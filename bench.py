@@ -139,6 +139,19 @@ def stored_traffic(kernel: str, workload: str):
     return None
 
 
+def max_over_ranks(values, device, world: int):
+    """Element-wise max of per-rank timings (every rank takes part; no-op at world 1)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(units_per_rank: float, world: int, slowest_ms: float) -> float:
+    """Whole-job TFLOP/s: the units of all ranks over the slowest rank's time."""
+    return world * units_per_rank / (slowest_ms / 1e3) / 1e12
+
+
 # --------------------------------------------------------------------------- work accounting
 def kept_work(row_ptr: np.ndarray, col_idx: np.ndarray, N: int, bs: int, bh: int):
     """Executed sparse-step flop factor: sum over query blocks of rows(qb) * kept key columns."""
@@ -264,12 +277,9 @@ def run_ours(args, rank, world, local):
                "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in h_in)),
                "d2h_bytes_per_step": int(h_out.numel() * h_out.element_size())}
 
-    # max over ranks of every time
-    vals = torch.tensor([total_ms, per_kernel["mask"], per_kernel["capture"], per_kernel["sparse"],
-                         e2e["ms_per_step"] if e2e else 0.0], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
-    total_ms, mask_ms, cap_ms, sp_ms, e2e_ms = vals.tolist()
+    total_ms, mask_ms, cap_ms, sp_ms, e2e_ms = max_over_ranks(
+        [total_ms, per_kernel["mask"], per_kernel["capture"], per_kernel["sparse"],
+         e2e["ms_per_step"] if e2e else 0.0], device, world)
     return {"w": w, "keep": keep, "keep_ratio": keep_ratio, "total_ms": total_ms, "mask_ms": mask_ms,
             "capture_ms": cap_ms, "sparse_ms": sp_ms, "e2e": e2e, "e2e_ms": e2e_ms, "clocks": clk, "nums": nums,
             "host1": host1, "host0": host0}
@@ -361,7 +371,7 @@ def main():
         peaks, peak_src = load_peaks()
         w, nums = r["w"], r["nums"]
         sp_s = r["sparse_ms"] / 1e3
-        value = world * nums["dense_flops"] / sp_s / 1e12
+        value = job_throughput(nums["dense_flops"], world, r["sparse_ms"])
         exec_tflops = nums["executed_flops"] / sp_s / 1e12
         cap_tflops = nums["dense_flops"] / (r["capture_ms"] / 1e3) / 1e12
         kernels = {
@@ -402,7 +412,7 @@ def main():
                     "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": f"hbm_gbs ({peak_src})"}
         e2e = None
         if r["e2e"]:
-            e2e = {"value": world * nums["dense_flops"] / (r["e2e_ms"] / 1e3) / 1e12, "unit": UNIT,
+            e2e = {"value": job_throughput(nums["dense_flops"], world, r["e2e_ms"]), "unit": UNIT,
                    "ms_per_step": r["e2e_ms"], "h2d_bytes_per_step": r["e2e"]["h2d_bytes_per_step"],
                    "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"],
                    "what": "sparse step through the public API: pinned host Q1/K1/V1 -> device, "
