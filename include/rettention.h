@@ -189,6 +189,39 @@ rt_status rt_take_device_error(int32_t *code);
  */
 rt_status rt_selftest_wait_timeout(int64_t timeout_ns, rt_stream_t stream);
 
+/*
+ * rt_build_block_mask_static -- rt_build_block_mask for callers that must not
+ * allocate device memory.
+ *
+ * The pages describe no such call; it exists for deployment.  Some callers
+ * cannot let a library call cudaMalloc or the stream-ordered allocator: code
+ * running under a framework that owns every byte of device memory through its
+ * own pool, real-time loops that must never block in an allocator, and
+ * processes whose memory budget is fixed up front.  This variant computes
+ * exactly what rt_build_block_mask computes (same arguments, same outputs,
+ * same kernels), but keeps its pooled-mean workspace in a fixed array that
+ * the library places in device memory when it is loaded, instead of taking a
+ * transient buffer from the allocator.
+ *
+ * Limit: the workspace holds 2*B*H*n_blocks*D fp32 values and is 8 MiB, so
+ * 2*B*H*n_blocks*D must not exceed 2097152 (the video 5B shape, 48 heads x 278
+ * blocks x 64, needs 1708032).  Larger shapes return RT_ERR_UNSUPPORTED and
+ * launch nothing.  Every GPU that loads the library holds those 8 MiB until the
+ * process exits.
+ *
+ * The first call on a device looks up the workspace's device address on that
+ * device (with the device current); make that first call before capturing
+ * the stream into a CUDA graph.  All calls on a device share the one
+ * workspace and it keeps the last call's contents; nothing in it needs to
+ * start at zero (every call overwrites what it reads).  Calls that overlap on
+ * the GPU (different streams, or different host threads, without ordering
+ * between them) race on the workspace and give wrong masks: serialise them.
+ */
+rt_status rt_build_block_mask_static(const rt_shape *shape, const void *q, const void *k, float scale,
+                                     int32_t keep_blocks, int32_t forced_prefix_tokens,
+                                     int32_t *row_ptr, int32_t *col_idx, float *block_scores,
+                                     rt_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

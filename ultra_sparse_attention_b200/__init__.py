@@ -34,7 +34,12 @@ __all__ = [
     "rt_abi_version",
     "rt_take_device_error",
     "rt_selftest_wait_timeout",
+    "rt_build_block_mask_static",
+    "STATIC_POOL_FLOATS",
 ]
+
+# Capacity of rt_build_block_mask_static's fixed workspace (fp32 values).
+STATIC_POOL_FLOATS = 2 * 1024 * 1024
 
 RT_OK = 0
 RT_ERR_INVALID_ARGUMENT = 1
@@ -83,6 +88,8 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.rt_abi_version.restype = i32
             lib.rt_take_device_error.argtypes = [ctypes.POINTER(i32)]
             lib.rt_selftest_wait_timeout.argtypes = [i64, vp]
+            lib.rt_build_block_mask_static.argtypes = [shp, vp, vp, f32, i32, i32, vp, vp, vp, vp]
+            lib.rt_build_block_mask_static.restype = ctypes.c_int
             for fn in ("rt_build_block_mask", "rt_attn_full_capture", "rt_attn_sparse_reshape",
                        "rt_take_device_error", "rt_selftest_wait_timeout"):
                 getattr(lib, fn).restype = ctypes.c_int
@@ -221,3 +228,35 @@ def rt_selftest_wait_timeout(timeout_ns: int, stream=None):
     dev = torch.device("cuda", torch.cuda.current_device())
     _call(load_library().rt_selftest_wait_timeout(int(timeout_ns), _stream_handle(dev, stream)),
           "rt_selftest_wait_timeout")
+
+
+def rt_build_block_mask_static(q: torch.Tensor, k: torch.Tensor, *, head_dim: int, block_size: int, scale: float,
+                               keep_blocks: int, forced_prefix_tokens: int = 0, row_ptr: torch.Tensor | None = None,
+                               col_idx: torch.Tensor | None = None, block_scores: torch.Tensor | None = None,
+                               stream=None):
+    """rt_build_block_mask without any device allocation inside the library.
+
+    For callers that cannot let the library allocate (a framework that owns all
+    device memory through its own pool, loops that must not block in an
+    allocator).  The workspace is a fixed 8 MiB array of the library, shared
+    by every call on a device: calls must not overlap on the GPU.  Pass
+    preallocated ``row_ptr`` / ``col_idx`` to avoid allocations on the Python
+    side as well.  Shapes with 2*B*H*n_blocks*D > STATIC_POOL_FLOATS raise.
+    """
+    dims = _check_qkv("rt_build_block_mask_static", q, k)
+    B, H, N, D = dims
+    nb = -(-N // block_size)
+    if 2 * B * H * nb * D > STATIC_POOL_FLOATS:
+        raise ValueError(f"rt_build_block_mask_static: workspace needs {2 * B * H * nb * D} fp32 values, "
+                         f"the fixed array holds {STATIC_POOL_FLOATS}")
+    dev = q.device
+    if row_ptr is None:
+        row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        col_idx = torch.empty(B * H * nb * max(keep_blocks, 0), dtype=torch.int32, device=dev)
+    shape = _shape(dims, head_dim, block_size)
+    _call(load_library().rt_build_block_mask_static(ctypes.byref(shape), _ptr(q), _ptr(k), float(scale),
+                                                    int(keep_blocks), int(forced_prefix_tokens), _ptr(row_ptr),
+                                                    _ptr(col_idx), _ptr(block_scores), _stream_handle(dev, stream)),
+          "rt_build_block_mask_static")
+    return row_ptr, col_idx

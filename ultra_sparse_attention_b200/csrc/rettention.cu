@@ -159,6 +159,30 @@ rt_status launch_mask(const Dims& d, const void* q, const void* k, float scale, 
   return launch_status();
 }
 
+// Fixed workspace of rt_build_block_mask_static: pooled Q and K means.  It is
+// placed in device memory when the module loads on a device, so the call that
+// uses it never allocates.
+constexpr size_t kStaticPoolFloats = size_t(2) * 1024 * 1024;  // 8 MiB
+static __device__ __align__(256) float g_static_pool[kStaticPoolFloats];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_pool_mutex;
+float* g_static_pool_addr[kMaxDevices] = {};
+
+// Device address of g_static_pool on the current device, looked up once per device.
+rt_status static_pool_address(float** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RT_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_pool_mutex);
+  if (g_static_pool_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_pool) != cudaSuccess || p == nullptr) return RT_ERR_CUDA;
+    g_static_pool_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_static_pool_addr[dev];
+  return RT_OK;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -265,6 +289,32 @@ rt_status rt_attn_sparse_reshape(const rt_shape* shape, const void* q, const voi
   a.n_blocks = static_cast<int>(d.n_blocks);
   a.scale_log2 = scale * rt::kLog2e;
   return dispatch_attention<false>(d, m, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+rt_status rt_build_block_mask_static(const rt_shape* shape, const void* q, const void* k, float scale,
+                                     int32_t keep_blocks, int32_t forced_prefix_tokens, int32_t* row_ptr,
+                                     int32_t* col_idx, float* block_scores, rt_stream_t stream) {
+  Dims d;
+  rt_status st = check_shape(shape, &d);
+  if (st != RT_OK) return st;
+  if (!q || !k || !row_ptr || !col_idx) return RT_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(row_ptr, 4) || !aligned(col_idx, 4) ||
+      !aligned(block_scores, 4))
+    return RT_ERR_INVALID_ARGUMENT;
+  if (!scale_ok(scale) || forced_prefix_tokens < 0) return RT_ERR_INVALID_ARGUMENT;
+  if (keep_blocks < 1 || keep_blocks > d.n_blocks) return RT_ERR_INVALID_ARGUMENT;
+  const int64_t forced = std::min<int64_t>(d.n_blocks, (int64_t(forced_prefix_tokens) + d.bs - 1) / d.bs);
+  if (forced > keep_blocks) return RT_ERR_INVALID_ARGUMENT;
+  if (d.bh * d.n_blocks * keep_blocks > (int64_t(1) << 31) - 1) return RT_ERR_UNSUPPORTED;
+  if (static_cast<size_t>(2 * d.bh * d.n_blocks * d.D) > kStaticPoolFloats) return RT_ERR_UNSUPPORTED;
+  float* pooled = nullptr;
+  st = static_pool_address(&pooled);
+  if (st != RT_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d.D == 64 ? launch_mask<64>(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx,
+                                      block_scores, pooled, s)
+                   : launch_mask<80>(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx,
+                                      block_scores, pooled, s);
 }
 
 rt_status rt_take_device_error(int32_t* code) {
