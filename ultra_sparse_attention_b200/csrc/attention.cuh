@@ -4,33 +4,34 @@
 //                          emits the statistics the later sparse steps reuse:
 //                          row max m, Z_full, Z_kept and the fp32 residual
 //                          numerator U of the masked-out keys (project page,
-//                          mechanism highlight: "reusing the stable ratio between
-//                          sparse and full softmax denominators and caching the
-//                          residual contributions from masked-out tokens").
+//                          mechanism highlight: the reused ratio of the sparse
+//                          and full softmax denominators, and the cached residual
+//                          contribution of the masked-out tokens).
 //   sparse_reshape_kernel  attention over the kept key blocks only, then the
 //                          reshape o = (N' + e^{m_c - m'} U) / (Z' * Z_full / Z_kept)
-//                          in the epilogue (teaser: "reshaping sparse attention
-//                          with cached statistics across denoising steps").
+//                          in the epilogue (teaser: sparse attention reshaped with
+//                          statistics cached across denoising steps).
 //
-// Shared design (one CTA = one 128-row query tile of one (batch, head)):
-//  * warp 0 issues TMA loads (Q once, then K/V 64-key tiles into a 4-stage
-//    ring), warp 1 issues tcgen05.mma, warps 2..5 own one query row per thread
-//    (TMEM lane = row) for the softmax and the epilogue.
-//  * S = Q K^T lands in TMEM (two 64-column buffers, so QK^T of tile j+1 runs
-//    while the softmax of tile j does); the softmax writes P as bf16 back into
-//    the first 32 columns of the same buffer and the PV product reads A = P
-//    straight from TMEM (no shared-memory round trip).
+// Shared design (a 128-row query tile of one (batch, head) at a time):
+//  * warp 0 issues TMA loads, warp 1 issues tcgen05.mma, warps 2..5 own one
+//    query row per thread (TMEM lane = row) for the softmax and the epilogue.
+//  * S = Q K^T lands in TMEM; the softmax writes P as bf16 back into the first
+//    32 columns of the same buffer and the PV product reads A = P straight from
+//    TMEM (no shared-memory round trip).
 //  * With 64-token blocks the 128-row tile holds two query blocks, each with
-//    its own kept list; the kernel walks the union of both lists and a row
-//    whose block does not keep a tile writes P = 0 for it.
+//    its own kept list; the sparse kernel walks the union of both lists and a
+//    row whose block does not keep a tile writes P = 0 for it.  (An M = 64 MMA
+//    per query block would halve the tensor rate; the union costs only the
+//    blocks the two lists do not share.)
 //  * Online softmax in base 2 (x = s * scale * log2 e) with a lazy reference:
-//    the O accumulator is rescaled only when the row max moves up by more than
-//    8 (or down by more than 64 in the sparse step, whose reference starts at
-//    the cached max), so the rescale path almost never runs.
+//    O is rescaled only when the row max moves up by more than 8 (or down by
+//    more than 64 in the sparse step, whose reference starts at the cached
+//    max), so the rescale path practically never runs.
 //  * Head dim 64 uses 128-byte swizzled tiles; head dim 80 adds a 16-column
 //    tail tile with 32-byte swizzle (one more K-step for QK^T, one N=16 MMA for PV).
-//  * Every barrier wait is bounded (see ptx.cuh); on a timeout the block stops,
-//    drains its own copies and MMAs, frees TMEM and returns.
+//  * Every barrier wait is bounded (see ptx.cuh) and its outcome is made
+//    warp-uniform; on a timeout the block stops, drains its own copies and
+//    MMAs, frees TMEM and returns.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -39,9 +40,8 @@
 
 namespace rt {
 
-constexpr int kBM = 128;            // query rows per CTA (tcgen05 M)
+constexpr int kBM = 128;            // query rows per tile (tcgen05 M)
 constexpr int kBN = 64;             // keys per tile
-constexpr int kStages = 4;          // K/V ring depth
 constexpr int kAttnThreads = 192;   // 6 warps
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -49,24 +49,21 @@ constexpr float kRescaleUp = 8.f;    // log2 units
 constexpr float kRescaleDown = 64.f; // log2 units
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 
+// Tile byte sizes for head dim D (bf16 Q/K/V tiles).  A K or V tile is the
+// 64-column part (128-byte swizzle) followed, for D = 80, by the 16-column
+// tail (32-byte swizzle).
 template <int D>
-struct Geom {
+struct Tiles {
   static_assert(D == 64 || D == 80, "head_dim_padded must be 64 or 80");
   static constexpr bool kTail = D == 80;
   static constexpr int kQMain = kBM * 128;
   static constexpr int kQTail = kTail ? kBM * 32 : 0;
+  static constexpr int kQBytes = kQMain + kQTail;
   static constexpr int kKVMain = kBN * 128;
   static constexpr int kKVTail = kTail ? kBN * 32 : 0;
-  static constexpr int kStageBytes = 2 * (kKVMain + kKVTail);
-  static constexpr int kQBytes = kQMain + kQTail;
+  static constexpr int kKVBytes = kKVMain + kKVTail;   // one K or one V tile
+  static constexpr int kStageBytes = 2 * kKVBytes;     // K tile then V tile
   static constexpr int kKSteps = D / 16;
-  // byte offsets from the 1024-aligned shared-memory base
-  static constexpr int kOffQMain = 0;
-  static constexpr int kOffQTail = kQMain;
-  static constexpr int kOffStage0 = kQMain + kQTail;  // multiple of 1024
-  static constexpr int kOffKMain = 0, kOffVMain = kKVMain, kOffKTail = 2 * kKVMain,
-                       kOffVTail = 2 * kKVMain + kKVTail;
-  static constexpr int kOffBarriers = kOffStage0 + kStages * kStageBytes;
 };
 
 struct AttnArgs {
@@ -86,118 +83,97 @@ struct AttnArgs {
   int N;
   int d;
   int n_blocks;
+  int n_heads;       // B*H
   float scale_log2;  // softmax scale * log2(e)
 };
 
-// Barriers and small shared state, placed after the tile buffers.
-struct alignas(8) AttnShared {
-  uint64_t q_full;
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t pv_done;
-  uint64_t o_full;
-  uint64_t drain;
-  uint32_t tmem_base;
-  int abort_flag;
-  int n_tiles;
-  int ok_any;   // capture: some tile is kept by some row
-  int ou_any;   // capture: some tile is masked for some row
-};
-
 __host__ __device__ constexpr int attn_words(int n_blocks) { return (n_blocks + 31) / 32; }
+__host__ __device__ constexpr int key_tiles(int N) { return (N + kBN - 1) / kBN; }
+__host__ __device__ constexpr int query_tiles(int N) { return (N + kBM - 1) / kBM; }
 
-// Shared bytes: tiles + AttnShared + two block bitmaps + the tile list, plus 1 KB for alignment.
+// ------------------------------------------------------------------ descriptors and MMA issue
 template <int D>
-__host__ __device__ constexpr size_t attn_smem_bytes(int n_blocks, int n_key_tiles) {
-  return 1024 + Geom<D>::kOffBarriers + sizeof(AttnShared) + 2 * sizeof(uint32_t) * attn_words(n_blocks) +
-         sizeof(uint32_t) * (n_key_tiles + 1);
-}
-
-// ------------------------------------------------------------------ pieces shared by both kernels
-template <int D>
-__device__ __forceinline__ uint64_t q_desc(uint32_t sbase, int ks) {
-  using G = Geom<D>;
-  return ks < 4 ? smem_desc(sbase + G::kOffQMain + ks * 32, 16, 1024, kSwizzle128B)
-                : smem_desc(sbase + G::kOffQTail, 16, 256, kSwizzle32B);
+__device__ __forceinline__ uint64_t q_desc(uint32_t q_base, int ks) {
+  return ks < 4 ? smem_desc(q_base + ks * 32, 16, 1024, kSwizzle128B)
+                : smem_desc(q_base + Tiles<D>::kQMain, 16, 256, kSwizzle32B);
 }
 template <int D>
-__device__ __forceinline__ uint64_t k_desc(uint32_t stage_base, int ks) {
-  using G = Geom<D>;
-  return ks < 4 ? smem_desc(stage_base + G::kOffKMain + ks * 32, 16, 1024, kSwizzle128B)
-                : smem_desc(stage_base + G::kOffKTail, 16, 256, kSwizzle32B);
+__device__ __forceinline__ uint64_t k_desc(uint32_t k_base, int ks) {
+  return ks < 4 ? smem_desc(k_base + ks * 32, 16, 1024, kSwizzle128B)
+                : smem_desc(k_base + Tiles<D>::kKVMain, 16, 256, kSwizzle32B);
 }
 // V as the N-major B operand of P V: key rows are K, head-dim columns are N.
 template <int D>
-__device__ __forceinline__ uint64_t v_desc_main(uint32_t stage_base, int ks) {
-  return smem_desc(stage_base + Geom<D>::kOffVMain + ks * 2048, Geom<D>::kKVMain, 1024, kSwizzle128B);
+__device__ __forceinline__ uint64_t v_desc_main(uint32_t v_base, int ks) {
+  return smem_desc(v_base + ks * 2048, Tiles<D>::kKVMain, 1024, kSwizzle128B);
 }
 template <int D>
-__device__ __forceinline__ uint64_t v_desc_tail(uint32_t stage_base, int ks) {
-  return smem_desc(stage_base + Geom<D>::kOffVTail + ks * 512, Geom<D>::kKVTail, 256, kSwizzle32B);
+__device__ __forceinline__ uint64_t v_desc_tail(uint32_t v_base, int ks) {
+  return smem_desc(v_base + Tiles<D>::kKVMain + ks * 512, Tiles<D>::kKVTail, 256, kSwizzle32B);
 }
 
 constexpr uint32_t kIdescQK = idesc_bf16(kBM, kBN, false, false);
 constexpr uint32_t kIdescPV64 = idesc_bf16(kBM, 64, false, true);
 constexpr uint32_t kIdescPV16 = idesc_bf16(kBM, 16, false, true);
 
-// QK^T of one key tile into the S buffer at `s_tmem`.
+// S = Q K^T for one key tile into TMEM at `s_tmem`.
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t sbase, uint32_t stage_base) {
+__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_base, uint32_t k_base) {
 #pragma unroll
-  for (int ks = 0; ks < Geom<D>::kKSteps; ++ks)
-    mma_ss(s_tmem, q_desc<D>(sbase, ks), k_desc<D>(stage_base, ks), kIdescQK, ks > 0 ? 1u : 0u);
+  for (int ks = 0; ks < Tiles<D>::kKSteps; ++ks)
+    mma_ss(s_tmem, q_desc<D>(q_base, ks), k_desc<D>(k_base, ks), kIdescQK, ks > 0 ? 1u : 0u);
 }
 
 // acc (+)= P V for one key tile; P is bf16 in TMEM at `p_tmem` (32 columns).
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t acc_tmem, uint32_t p_tmem, uint32_t stage_base, bool accumulate) {
+__device__ __forceinline__ void issue_pv(uint32_t acc_tmem, uint32_t p_tmem, uint32_t v_base, bool accumulate) {
 #pragma unroll
   for (int ks = 0; ks < kBN / 16; ++ks) {
     const uint32_t acc = (accumulate || ks > 0) ? 1u : 0u;
-    mma_ts(acc_tmem, p_tmem + ks * 8, v_desc_main<D>(stage_base, ks), kIdescPV64, acc);
-    if constexpr (Geom<D>::kTail) mma_ts(acc_tmem + 64, p_tmem + ks * 8, v_desc_tail<D>(stage_base, ks), kIdescPV16, acc);
+    mma_ts(acc_tmem, p_tmem + ks * 8, v_desc_main<D>(v_base, ks), kIdescPV64, acc);
+    if constexpr (Tiles<D>::kTail)
+      mma_ts(acc_tmem + 64, p_tmem + ks * 8, v_desc_tail<D>(v_base, ks), kIdescPV16, acc);
   }
 }
 
-// Producer: Q once, then the K/V tiles listed in `tiles` (entry >> 2 = key-tile index).
 template <int D>
-__device__ void produce(AttnShared& sh, unsigned char* smem, const CUtensorMap* tq, const CUtensorMap* tq_tail,
-                        const CUtensorMap* tk, const CUtensorMap* tk_tail, const CUtensorMap* tv,
-                        const CUtensorMap* tv_tail, const uint32_t* tiles, int n_tiles, int q_row0, int bh,
-                        bool all_tiles) {
-  using G = Geom<D>;
-  volatile int* abort_flag = &sh.abort_flag;
-  mbar_arrive_expect_tx(&sh.q_full, G::kQBytes);
-  tma_load_3d(smem + G::kOffQMain, tq, &sh.q_full, 0, q_row0, bh);
-  if constexpr (G::kTail) tma_load_3d(smem + G::kOffQTail, tq_tail, &sh.q_full, 64, q_row0, bh);
-  int issued = 0;
-  for (int j = 0; j < n_tiles; ++j) {
-    const int st = j % kStages;
-    if (j >= kStages && !mbar_wait(&sh.kv_empty[st], ((j / kStages) - 1) & 1, abort_flag)) break;
-    const int tile = all_tiles ? j : static_cast<int>(tiles[j] >> 2);
-    const int key_row0 = tile * kBN;
-    unsigned char* stage = smem + G::kOffStage0 + st * G::kStageBytes;
-    mbar_arrive_expect_tx(&sh.kv_full[st], G::kStageBytes);
-    tma_load_3d(stage + G::kOffKMain, tk, &sh.kv_full[st], 0, key_row0, bh);
-    tma_load_3d(stage + G::kOffVMain, tv, &sh.kv_full[st], 0, key_row0, bh);
-    if constexpr (G::kTail) {
-      tma_load_3d(stage + G::kOffKTail, tk_tail, &sh.kv_full[st], 64, key_row0, bh);
-      tma_load_3d(stage + G::kOffVTail, tv_tail, &sh.kv_full[st], 64, key_row0, bh);
-    }
-    issued = j + 1;
-  }
-  if (*abort_flag) {
-    // Let every copy this block started land before the block exits.
-    volatile int no_abort = 0;
-    mbar_wait(&sh.q_full, 0, &no_abort, kDrainLimitNs);
-    for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-      mbar_wait(&sh.kv_full[j % kStages], (j / kStages) & 1, &no_abort, kDrainLimitNs);
-  }
+__device__ __forceinline__ void load_q(unsigned char* dst, const CUtensorMap* tq, const CUtensorMap* tq_tail,
+                                       uint64_t* bar, int row0, int bh) {
+  mbar_arrive_expect_tx(bar, Tiles<D>::kQBytes);
+  tma_load_3d(dst, tq, bar, 0, row0, bh);
+  if constexpr (Tiles<D>::kTail) tma_load_3d(dst + Tiles<D>::kQMain, tq_tail, bar, 64, row0, bh);
 }
 
-// Rescale `ncols` fp32 columns of this thread's TMEM row by f (warp-collective).
+// One 64-key K or V tile (main + tail) into `dst`, completing on `bar`.
+template <int D>
+__device__ __forceinline__ void load_kv_tile(unsigned char* dst, const CUtensorMap* t, const CUtensorMap* t_tail,
+                                             uint64_t* bar, int row0, int bh) {
+  mbar_arrive_expect_tx(bar, Tiles<D>::kKVBytes);
+  tma_load_3d(dst, t, bar, 0, row0, bh);
+  if constexpr (Tiles<D>::kTail) tma_load_3d(dst + Tiles<D>::kKVMain, t_tail, bar, 64, row0, bh);
+}
+
+// K then V tile of one key tile into a combined stage, completing on one barrier.
+template <int D>
+__device__ __forceinline__ void load_kv(unsigned char* stage, const CUtensorMap* tk, const CUtensorMap* tk_tail,
+                                        const CUtensorMap* tv, const CUtensorMap* tv_tail, uint64_t* bar, int row0,
+                                        int bh) {
+  using T = Tiles<D>;
+  mbar_arrive_expect_tx(bar, T::kStageBytes);
+  tma_load_3d(stage, tk, bar, 0, row0, bh);
+  if constexpr (T::kTail) tma_load_3d(stage + T::kKVMain, tk_tail, bar, 64, row0, bh);
+  tma_load_3d(stage + T::kKVBytes, tv, bar, 0, row0, bh);
+  if constexpr (T::kTail) tma_load_3d(stage + T::kKVBytes + T::kKVMain, tv_tail, bar, 64, row0, bh);
+}
+
+// ------------------------------------------------------------------ softmax helpers
+// Bounded wait whose outcome is the same for every lane of the warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const bool ok = mbar_wait(bar, parity, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Rescale NCOLS fp32 columns of this thread's TMEM row by f (warp-collective).
 template <int NCOLS>
 __device__ __forceinline__ void tmem_row_scale(uint32_t taddr, float f) {
 #pragma unroll
@@ -216,6 +192,11 @@ __device__ __forceinline__ void tmem_st32_zero(uint32_t taddr) {
   const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
   tmem_st16(taddr, z);
   tmem_st16(taddr + 16, z);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&pk)[32]) {
+  tmem_st16(taddr, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+  tmem_st16(taddr + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
 }
 
 // Mask key columns at or beyond N (only the ragged last tile has any).
@@ -266,230 +247,465 @@ __device__ __forceinline__ float exp_inplace64(float (&s)[64], float C, float re
   return z0 + z1;
 }
 
-// Block bitmaps of the kept key blocks of the (up to two) query blocks of this CTA.
-__device__ __forceinline__ void load_block_bitmaps(uint32_t* bitmaps, int words, const AttnArgs& a, int bh,
-                                                   int qb0, int nqb) {
-  for (int g = 0; g < nqb; ++g) {
-    const int qb = qb0 + g;
-    if (qb >= a.n_blocks) break;
-    const size_t r = static_cast<size_t>(bh) * a.n_blocks + qb;
-    const int s = a.row_ptr[r], e = a.row_ptr[r + 1];
-    const int len = max(0, min(e - s, a.n_blocks));
-    for (int i = threadIdx.x; i < len; i += blockDim.x) {
-      const int kb = a.col_idx[s + i];
-      if (kb >= 0 && kb < a.n_blocks) atomicOr(&bitmaps[g * words + kb / 32], 1u << (kb % 32));
-    }
+__device__ __forceinline__ bool bitmap_has(const uint32_t* bm, int kb) { return (bm[kb / 32] >> (kb % 32)) & 1u; }
+
+// Set the bits of the kept key blocks of query block `qb` of head `bh` (threads `t0, t0+stride, ...`).
+__device__ __forceinline__ void mark_kept_blocks(uint32_t* bm, const AttnArgs& a, int bh, int qb, int t0,
+                                                 int stride) {
+  if (qb >= a.n_blocks) return;
+  const size_t r = static_cast<size_t>(bh) * a.n_blocks + qb;
+  const int s = a.row_ptr[r], e = a.row_ptr[r + 1];
+  const int len = max(0, min(e - s, a.n_blocks));
+  for (int i = t0; i < len; i += stride) {
+    const int kb = a.col_idx[s + i];
+    if (kb >= 0 && kb < a.n_blocks) atomicOr(&bm[kb / 32], 1u << (kb % 32));
   }
 }
 
-__device__ __forceinline__ bool bitmap_has(const uint32_t* bm, int kb) { return (bm[kb / 32] >> (kb % 32)) & 1u; }
+// ================================================================== sparse step (persistent)
+//
+// Kept key tiles of every 128-row query tile, precomputed from the CSR by
+// tile_lists_kernel: lists[t * cap] = count, lists[t * cap + 1 + j] =
+// tile << 2 | (kept by query block 0) | (kept by query block 1) << 1, the
+// union of the tile's query blocks' kept lists in ascending order.
+__host__ __device__ constexpr int tile_list_cap(int N) { return (key_tiles(N) + 1 + 7) / 8 * 8; }
 
-// ------------------------------------------------------------------ sparse step
+template <int BS>
+__global__ void __launch_bounds__(32) tile_lists_kernel(const AttnArgs a, uint16_t* __restrict__ lists) {
+  extern __shared__ uint32_t bm[];  // [2][words]
+  constexpr int kQB = kBM / BS;
+  const int lane = threadIdx.x;
+  if (__shfl_sync(0xffffffffu, device_status_set() ? 1 : 0, 0)) return;  // an earlier kernel failed
+  const int n_qt = query_tiles(a.N), t = blockIdx.x, bh = t / n_qt, qt = t % n_qt;
+  const int words = attn_words(a.n_blocks), n_kt = key_tiles(a.N), cap = tile_list_cap(a.N);
+  for (int w = lane; w < 2 * words; w += 32) bm[w] = 0u;
+  __syncwarp();
+  for (int q = 0; q < kQB; ++q) mark_kept_blocks(bm + q * words, a, bh, qt * kQB + q, lane, 32);
+  __syncwarp();
+  uint16_t* out = lists + static_cast<size_t>(t) * cap;
+  int count = 0;
+  for (int t0 = 0; t0 < n_kt; t0 += 32) {
+    const int tile = t0 + lane;
+    uint32_t flags = 0u;
+    if (tile < n_kt) {
+      const int kb = tile * kBN / BS;
+      flags = bitmap_has(bm, kb) ? 1u : 0u;
+      if (kQB == 2) flags |= bitmap_has(bm + words, kb) ? 2u : 0u;
+    }
+    const uint32_t mask = __ballot_sync(0xffffffffu, flags != 0u);
+    if (flags) out[1 + count + __popc(mask & ((1u << lane) - 1u))] = static_cast<uint16_t>((tile << 2) | flags);
+    count += __popc(mask);
+  }
+  if (lane == 0) out[0] = static_cast<uint16_t>(count);
+}
+
+// The sparse kernel.  Grid: up to two CTAs per SM, each walking query tiles
+// t = blockIdx.x, blockIdx.x + gridDim.x, ... in head-major order
+// (neighbouring CTAs share a head, so its K/V stay in L2).
+//
+// Measured on this part: a tcgen05.mma costs ~50 cycles to issue, a commit
+// ~90, an mbarrier test 100-200 even when the phase is complete, and a
+// hand-off between warps ~250.  The pipeline is built to keep those off the
+// per-key-tile path:
+//  * warp 0, lane 0 (producer): bulk-copies the precomputed list of tile i+2,
+//    loads Q(i) into one of two buffers, streams K(g) and V(g) of every key
+//    tile g into two rings under ONE barrier per key tile, and issues the TMA
+//    store of each finished tile (polled, so no warp ever waits on a store);
+//  * warp 1, lane 0 (MMA): step g issues PV(g-2), then QK^T(g), then one
+//    commit to step[g % 8] -- which tells the softmax that S(g) is ready and
+//    P[g & 1] (aliased into S) was consumed, and tells the producer that the
+//    K slot of g and the V slot of g-2 are free;
+//  * warps 2-5 (softmax + epilogue): one row per thread; P is written as bf16
+//    into the first 32 columns of S[g & 1].
+// TMEM (256 columns): S0 [0,64) S1 [64,128) O [128,128+D).
+// The epilogue releases O right after reading it, combines it with U (whose
+// row each thread prefetched into L2 a tile earlier), and writes bf16 rows
+// into the tile's Q buffer, which the producer then stores with one TMA store.
+template <int D>
+struct SparseLayout {
+  using T = Tiles<D>;
+  static constexpr int kNK = D == 64 ? 3 : 2;  // K ring
+  static constexpr int kNV = D == 64 ? 5 : 4;  // V ring
+  static_assert(kNV - 2 == kNK, "K(g) and V(g) load together once step g - kNK is done");
+  static constexpr int kNL = 3;                // tile-list buffers
+  static constexpr int kOffQ = 0;              // two Q / output staging buffers
+  static constexpr int kOffK = 2 * T::kQBytes;
+  static constexpr int kOffV = kOffK + kNK * T::kKVBytes;
+  static constexpr int kOffLists = kOffV + kNV * T::kKVBytes;
+};
+
+struct alignas(8) SparseShared {
+  uint64_t q_full[2];
+  uint64_t kv_full[8], step[8];
+  uint64_t p_full[2];
+  uint64_t o_full, o_empty;
+  uint64_t staged[2];
+  uint64_t list_full[3], list_empty[3];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+__host__ __device__ constexpr size_t sparse_smem_bytes(int N) {
+  return 1024 + SparseLayout<D>::kOffLists + SparseLayout<D>::kNL * 2 * tile_list_cap(N) + sizeof(SparseShared);
+}
+
 template <int D, int BS>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     sparse_reshape_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tq_tail,
                           const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tk_tail,
                           const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tv_tail,
-                          const AttnArgs a) {
-  using G = Geom<D>;
+                          const __grid_constant__ CUtensorMap to, const __grid_constant__ CUtensorMap to_tail,
+                          const AttnArgs a, const uint16_t* __restrict__ tile_lists) {
+  using T = Tiles<D>;
+  using L = SparseLayout<D>;
   static_assert(BS == 64 || BS == 128, "block size must be 64 or 128");
-  constexpr int kQBPerCta = kBM / BS;
-  constexpr uint32_t kTmemCols = 256;  // S0 [0,64) S1 [64,128) O [128,128+D)
+  constexpr int NK = L::kNK, NV = L::kNV, NL = L::kNL;
+  constexpr uint32_t kTmemCols = 256;
   constexpr uint32_t kOCol = 128;
 
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   unsigned char* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sbase = smem_u32(smem);
-  AttnShared& sh = *reinterpret_cast<AttnShared*>(smem + G::kOffBarriers);
-  const int words = attn_words(a.n_blocks);
-  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(&sh + 1);
-  uint32_t* tiles = bitmaps + 2 * words;
+  const int cap = tile_list_cap(a.N);
+  uint16_t* lists = reinterpret_cast<uint16_t*>(smem + L::kOffLists);  // [NL][cap]
+  SparseShared& sh = *reinterpret_cast<SparseShared*>(smem + L::kOffLists + NL * 2 * cap);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int bh = blockIdx.y;
-  const int q_row0 = blockIdx.x * kBM;
-  const int qb0 = blockIdx.x * kQBPerCta;
+  const int n_qt = query_tiles(a.N);
+  const int total = n_qt * a.n_heads;
+  const int n_mine = total > static_cast<int>(blockIdx.x) ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const bool has_stats = a.stat_m != nullptr;
 
   if (warp == 0) tmem_alloc(&sh.tmem_base, kTmemCols);
   if (threadIdx.x == 32) {
-    mbar_init(&sh.q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sh.kv_full[s], 1);
-      mbar_init(&sh.kv_empty[s], 1);
-    }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&sh.s_full[b], 1);
+      mbar_init(&sh.q_full[b], 1);
       mbar_init(&sh.p_full[b], 128);
+      mbar_init(&sh.staged[b], 128);
     }
-    mbar_init(&sh.pv_done, 1);
+    for (int s = 0; s < 8; ++s) {
+      mbar_init(&sh.kv_full[s], 1);
+      mbar_init(&sh.step[s], 1);
+    }
+    for (int s = 0; s < NL; ++s) {
+      mbar_init(&sh.list_full[s], 1);
+      mbar_init(&sh.list_empty[s], 5);  // the MMA thread + one lane of each softmax warp
+    }
     mbar_init(&sh.o_full, 1);
+    mbar_init(&sh.o_empty, 128);
     mbar_init(&sh.drain, 1);
     sh.abort_flag = device_status_set() ? 1 : 0;  // an earlier failure: do nothing
     fence_mbar_init();
-  }
-  for (int i = threadIdx.x; i < 2 * words; i += blockDim.x) bitmaps[i] = 0u;
-  __syncthreads();
-  const bool run = sh.abort_flag == 0;  // block-uniform
-  if (run) load_block_bitmaps(bitmaps, words, a, bh, qb0, kQBPerCta);
-  __syncthreads();
-  // Union of the kept lists as 64-key tiles: entry = tile << 2 | (kept by block 0) | (kept by block 1) << 1.
-  if (warp == 2) {
-    int count = 0;
-    const int n_key_tiles = (a.N + kBN - 1) / kBN;
-    for (int t0 = 0; t0 < n_key_tiles; t0 += 32) {
-      const int tile = t0 + lane;
-      uint32_t flags = 0u;
-      if (tile < n_key_tiles) {
-        const int kb = tile * kBN / BS;
-        flags = bitmap_has(bitmaps, kb) ? 1u : 0u;
-        if (kQBPerCta == 2) flags |= bitmap_has(bitmaps + words, kb) ? 2u : 0u;
-      }
-      const uint32_t mask = __ballot_sync(0xffffffffu, flags != 0u);
-      if (flags) tiles[count + __popc(mask & ((1u << lane) - 1u))] = (static_cast<uint32_t>(tile) << 2) | flags;
-      count += __popc(mask);
-    }
-    if (lane == 0) sh.n_tiles = count;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
-  const int T = sh.n_tiles;
   volatile int* abort_flag = &sh.abort_flag;
+  const bool run = sh.abort_flag == 0;  // block-uniform
+  auto tile_of = [&](int i) { return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x); };
 
   if (!run) {
     // an earlier kernel failed: leave the outputs untouched
   } else if (warp == 0) {
-    if (lane == 0 && T > 0) produce<D>(sh, smem, &tq, &tq_tail, &tk, &tk_tail, &tv, &tv_tail, tiles, T, q_row0, bh, false);
-  } else if (warp == 1) {
-    if (lane == 0 && T > 0) {
-      bool ok = mbar_wait(&sh.q_full, 0, abort_flag);
-      auto pv = [&](int i) -> bool {
-        if (!mbar_wait(&sh.p_full[i & 1], (i >> 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-        issue_pv<D>(tmem + kOCol, tmem + (i & 1) * 64, sbase + G::kOffStage0 + (i % kStages) * G::kStageBytes, i > 0);
-        mma_commit(&sh.kv_empty[i % kStages]);
-        mma_commit(&sh.pv_done);
+    // ---------------- producer (one thread)
+    if (lane == 0) {
+      int lists_issued = 0, stores_issued = 0, q_loads = 0, g = 0, kslot = 0, vslot = 0;
+      bool ok = true;
+      // Bring the list of tile `lists_issued` into its buffer; `block` waits for the buffer.
+      auto issue_list = [&](bool block) -> bool {
+        const int i = lists_issued, lb = i % NL;
+        if (i >= n_mine) return true;
+        if (i >= NL) {
+          const uint32_t par = ((i / NL) - 1) & 1;
+          if (block ? !mbar_wait(&sh.list_empty[lb], par, abort_flag) : !mbar_test(&sh.list_empty[lb], par))
+            return !block;
+        }
+        mbar_arrive_expect_tx(&sh.list_full[lb], 2 * cap);
+        bulk_load(lists + lb * cap, tile_lists + static_cast<size_t>(tile_of(i)) * cap, 2 * cap, &sh.list_full[lb]);
+        ++lists_issued;
         return true;
       };
-      for (int j = 0; ok && j < T; ++j) {
-        const int st = j % kStages;
-        if (!mbar_wait(&sh.kv_full[st], (j / kStages) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        issue_qk<D>(tmem + (j & 1) * 64, sbase, sbase + G::kOffStage0 + st * G::kStageBytes);
-        mma_commit(&sh.s_full[j & 1]);
-        if (j > 0 && !pv(j - 1)) ok = false;
+      // Store the output of tile `stores_issued` once its epilogue has staged it.
+      auto issue_store = [&](bool block) -> bool {
+        const int i = stores_issued;
+        const uint32_t par = (i >> 1) & 1;
+        if (block ? !mbar_wait(&sh.staged[i & 1], par, abort_flag) : !mbar_test(&sh.staged[i & 1], par))
+          return !block;
+        const int t = tile_of(i), bh = t / n_qt, qt = t % n_qt;
+        const unsigned char* stg = smem + L::kOffQ + (i & 1) * T::kQBytes;
+        tma_store_3d(&to, stg, 0, qt * kBM, bh);
+        if constexpr (T::kTail) tma_store_3d(&to_tail, stg + T::kQMain, 64, qt * kBM, bh);
+        bulk_commit_group();
+        ++stores_issued;
+        return true;
+      };
+      for (int i = 0; ok && i < n_mine; ++i) {
+        const int t = tile_of(i), bh = t / n_qt, qt = t % n_qt;
+        while (ok && lists_issued < i + 2 && lists_issued < n_mine) ok = issue_list(true);
+        if (!ok) break;
+        if (!mbar_wait(&sh.list_full[i % NL], (i / NL) & 1, abort_flag)) break;
+        const int count = lists[(i % NL) * cap];
+        const uint16_t* lst = lists + (i % NL) * cap + 1;
+        // Q(i) reuses the buffer of tile i-2 once its output store has read it.
+        if (i >= 2) {
+          while (ok && stores_issued <= i - 2) ok = issue_store(true);
+          if (!ok) break;
+          bulk_wait_group_read0();
+        }
+        load_q<D>(smem + L::kOffQ + (i & 1) * T::kQBytes, &tq, &tq_tail, &sh.q_full[i & 1], qt * kBM, bh);
+        ++q_loads;
+        for (int j = 0; j < count; ++j, ++g) {
+          if (g >= NK && !mbar_wait(&sh.step[(g - NK) & 7], ((g - NK) >> 3) & 1, abort_flag)) { ok = false; break; }
+          const int row0 = (lst[j] >> 2) * kBN;
+          uint64_t* bar = &sh.kv_full[g & 7];
+          mbar_arrive_expect_tx(bar, 2 * T::kKVBytes);
+          unsigned char* kd = smem + L::kOffK + kslot * T::kKVBytes;
+          unsigned char* vd = smem + L::kOffV + vslot * T::kKVBytes;
+          tma_load_3d(kd, &tk, bar, 0, row0, bh);
+          if constexpr (T::kTail) tma_load_3d(kd + T::kKVMain, &tk_tail, bar, 64, row0, bh);
+          tma_load_3d(vd, &tv, bar, 0, row0, bh);
+          if constexpr (T::kTail) tma_load_3d(vd + T::kKVMain, &tv_tail, bar, 64, row0, bh);
+          if (++kslot == NK) kslot = 0;
+          if (++vslot == NV) vslot = 0;
+          // Opportunistic work that must not wait: the next list, a finished tile's store.
+          if (lists_issued < n_mine) issue_list(false);
+          if (stores_issued < i) issue_store(false);
+        }
       }
-      if (ok && pv(T - 1)) mma_commit(&sh.o_full);
+      while (ok && stores_issued < n_mine) ok = issue_store(true);
+      bulk_wait_group0();
+      if (*abort_flag) {
+        // Let every copy this block started land before the block exits.
+        volatile int no_abort = 0;
+        for (int i = q_loads > 2 ? q_loads - 2 : 0; i < q_loads; ++i)
+          mbar_wait(&sh.q_full[i & 1], (i >> 1) & 1, &no_abort, kDrainLimitNs);
+        for (int h = g > 8 ? g - 8 : 0; h < g; ++h) mbar_wait(&sh.kv_full[h & 7], (h >> 3) & 1, &no_abort, kDrainLimitNs);
+        for (int i = lists_issued > NL ? lists_issued - NL : 0; i < lists_issued; ++i)
+          mbar_wait(&sh.list_full[i % NL], (i / NL) & 1, &no_abort, kDrainLimitNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (one thread)
+    if (lane == 0) {
+      struct Item { int j, T, e; bool valid; };
+      Item q0{0, 0, 0, false}, q1{0, 0, 0, false};  // key tiles g-2 and g-1
+      int g = 0, e = 0, kslot = 0, vslot = 0;
+      bool ok = true;
+      // PV of key tile h = g - 2 (or later in the drain).
+      auto pv = [&](const Item& it, int h) -> bool {
+        if (!mbar_wait(&sh.p_full[h & 1], (h >> 1) & 1, abort_flag)) return false;
+        if (it.j == 0 && it.e >= 1 && !mbar_wait(&sh.o_empty, (it.e - 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        issue_pv<D>(tmem + kOCol, tmem + (h & 1) * 64, sbase + L::kOffV + vslot * T::kKVBytes, it.j > 0);
+        if (++vslot == NV) vslot = 0;
+        if (it.j == it.T - 1) mma_commit(&sh.o_full);
+        return true;
+      };
+      for (int i = 0; ok && i < n_mine; ++i) {
+        if (!mbar_wait(&sh.list_full[i % NL], (i / NL) & 1, abort_flag)) { ok = false; break; }
+        const int Tn = lists[(i % NL) * cap];
+        mbar_arrive(&sh.list_empty[i % NL]);
+        if (Tn == 0) continue;
+        if (!mbar_wait(&sh.q_full[i & 1], (i >> 1) & 1, abort_flag)) { ok = false; break; }
+        const uint32_t q_base = sbase + L::kOffQ + (i & 1) * T::kQBytes;
+        for (int j = 0; j < Tn; ++j, ++g) {
+          if (q0.valid && !pv(q0, g - 2)) { ok = false; break; }
+          if (!mbar_wait(&sh.kv_full[g & 7], (g >> 3) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_qk<D>(tmem + (g & 1) * 64, q_base, sbase + L::kOffK + kslot * T::kKVBytes);
+          mma_commit(&sh.step[g & 7]);
+          if (++kslot == NK) kslot = 0;
+          q0 = q1;
+          q1 = Item{j, Tn, e, true};
+        }
+        ++e;
+      }
+      // Drain: the last two PVs, each closing a step of its own.
+      if (ok && q0.valid) ok = pv(q0, g - 2);
+      if (ok) mma_commit(&sh.step[g & 7]);
+      if (ok && q1.valid) ok = pv(q1, g - 1);
+      if (ok) mma_commit(&sh.step[(g + 1) & 7]);
       mma_commit(&sh.drain);
       volatile int no_abort = 0;
       mbar_wait(&sh.drain, 0, &no_abort, kDrainLimitNs);
     }
   } else {
-    // ---- softmax + epilogue: one query row per thread
+    // ---------------- softmax + epilogue: one query row per thread (warps 2..5)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const int g = r / BS;
-    const int i = q_row0 + r;
-    const bool valid = i < a.N;
-    const size_t row_g = static_cast<size_t>(bh) * a.N + (valid ? i : 0);
-    const bool has_stats = a.stat_m != nullptr;
+    const int grp = r / BS;
     const float C = a.scale_log2;
-    float m_run = -INFINITY, mc2 = 0.f, zf_c = 1.f, zk_c = 1.f;
-    if (has_stats) {
-      if (valid) {
-        mc2 = a.stat_m[row_g] * kLog2e;
-        zf_c = a.stat_zfull[row_g];
-        zk_c = a.stat_zkept[row_g];
+    const uint64_t C2 = f2_pack(C, C);
+    // Prefetch into L2 what the epilogue of tile i reads: this row's U and statistics.
+    auto prefetch_row = [&](int i) {
+      if (!has_stats || i >= n_mine) return;
+      const int t = tile_of(i), bh = t / n_qt, row = (t % n_qt) * kBM + r;
+      if (row >= a.N) return;
+      const size_t rg = static_cast<size_t>(bh) * a.N + row;
+      const unsigned char* u = reinterpret_cast<const unsigned char*>(a.stat_u + rg * D);
+#pragma unroll
+      for (int off = 0; off < D * 4; off += 128) prefetch_l2(u + off);
+      prefetch_l2(u + D * 4 - 4);
+      if ((r & 31) == 0) {
+        prefetch_l2(a.stat_m + rg);
+        prefetch_l2(a.stat_zfull + rg);
+        prefetch_l2(a.stat_zkept + rg);
       }
-      m_run = mc2;
-    }
-    float m_seen = -INFINITY, z = 0.f;
-    bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      if (!mbar_wait(&sh.s_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t e = tiles[j];
-      const bool active = (e >> g) & 1u;
-      const uint32_t pt = tmem + lane_off + (j & 1) * 64;
-      if (active) {
-        float s[64];
-        tmem_ld64(pt, s);
-        mask_tail(s, static_cast<int>(e >> 2) * kBN, a.N);
-        m_seen = fmaxf(m_seen, row_max64(s) * C);
-        float ref = m_run;
-        bool need = false;
-        if (m_run == -INFINITY) {
-          ref = m_seen;
-        } else if (m_seen > m_run + kRescaleUp || m_seen < m_run - kRescaleDown) {
-          need = true;
-          ref = m_seen;
+    };
+    prefetch_row(0);
+    int g = 0, e = 0;
+    for (int i = 0; i < n_mine; ++i) {
+      prefetch_row(i + 1);
+      const int t = tile_of(i), bh = t / n_qt, qt = t % n_qt;
+      const int row = qt * kBM + r;
+      const bool valid = row < a.N;
+      const size_t row_g = static_cast<size_t>(bh) * a.N + (valid ? row : 0);
+      float m_run = -INFINITY, mc2 = 0.f, zf_c = 1.f, zk_c = 1.f;
+      if (has_stats) {
+        if (valid) {
+          mc2 = __ldg(a.stat_m + row_g) * kLog2e;
+          zf_c = __ldg(a.stat_zfull + row_g);
+          zk_c = __ldg(a.stat_zkept + row_g);
         }
-        if (__any_sync(0xffffffffu, need)) {
-          if (j > 0 && !mbar_wait(&sh.pv_done, (j - 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const float f = need ? ex2_approx(m_run - ref) : 1.f;
-          tmem_row_scale<D>(tmem + lane_off + kOCol, f);
-          z *= f;
-        }
-        m_run = ref;
+        m_run = mc2;
+      }
+      const int lb = i % NL;
+      if (!warp_wait(&sh.list_full[lb], (i / NL) & 1, abort_flag)) break;
+      const int Tn = lists[lb * cap];
+      const uint16_t* lst = lists + lb * cap + 1;
+      float m_seen = -INFINITY, z = 0.f;
+      bool ok = true;
+      for (int j = 0; j < Tn; ++j, ++g) {
+        if (!warp_wait(&sh.step[g & 7], (g >> 3) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ent = lst[j];
+        const bool active = (ent >> grp) & 1u;  // warp-uniform
+        const uint32_t pt = tmem + lane_off + (g & 1) * 64;
         uint32_t pk[32];
-        if (m_run == -INFINITY) {
+        if (active) {
+          float s[64];
+          tmem_ld64(pt, s);
+          mask_tail(s, static_cast<int>(ent >> 2) * kBN, a.N);
+          float mx = fmax3(s[0], s[1], s[2]);
+#pragma unroll
+          for (int c = 3; c < 63; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
+          mx = fmaxf(mx, s[63]);
+          m_seen = fmaxf(m_seen, mx * C);
+          float ref = m_run;
+          bool need = false;
+          if (m_run == -INFINITY) {
+            ref = m_seen;
+          } else if (m_seen > m_run + kRescaleUp || m_seen < m_run - kRescaleDown) {
+            need = true;
+            ref = m_seen;
+          }
+          if (__any_sync(0xffffffffu, need)) {
+            // Rescaling O needs PV(g-1) done: step g+1 (the previous tile's O is already read when j == 0).
+            if (j > 0 && !warp_wait(&sh.step[(g + 1) & 7], ((g + 1) >> 3) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const float f = need ? ex2_approx(m_run - ref) : 1.f;
+            tmem_row_scale<D>(tmem + lane_off + kOCol, f);
+            z *= f;
+          }
+          m_run = ref;
+          if (m_run == -INFINITY) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pk[c] = 0u;
+          } else {
+            const uint64_t nref = f2_pack(-m_run, -m_run);
+            uint64_t zz = f2_pack(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), C2, nref), x0, x1);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              zz = f2_add(zz, f2_pack(p0, p1));
+              pk[c / 2] = pack_bf16x2(p0, p1);
+            }
+            float z0, z1;
+            f2_unpack(zz, z0, z1);
+            z += z0 + z1;
+          }
+        } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) pk[c] = 0u;
-        } else {
-          z += exp_pack64(s, C, m_run, pk);
         }
-        tmem_st16(pt, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-        tmem_st16(pt + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
-      } else {
-        tmem_st32_zero(pt);
+        tmem_st32(pt, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&sh.p_full[g & 1]);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&sh.p_full[j & 1]);
-    }
-    if (ok && T > 0) ok = mbar_wait(&sh.o_full, 0, abort_flag);
-    tc_fence_after();
-    if (ok) {
-      const float fu = has_stats ? ex2_approx(mc2 - m_run) : 0.f;
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.list_empty[lb]);
+
+      // ---- epilogue
+      float u[D];
+#pragma unroll
+      for (int c = 0; c < D; ++c) u[c] = 0.f;
+      float fu = 0.f;
+      if (has_stats && valid) {
+        // U is read before waiting for O so its latency overlaps the last PV.
+        const float4* up = reinterpret_cast<const float4*>(a.stat_u + row_g * D);
+#pragma unroll
+        for (int q4 = 0; q4 < D / 4; ++q4) {
+          const float4 x = __ldg(up + q4);
+          u[4 * q4 + 0] = x.x;
+          u[4 * q4 + 1] = x.y;
+          u[4 * q4 + 2] = x.z;
+          u[4 * q4 + 3] = x.w;
+        }
+        fu = ex2_approx(mc2 - m_run);
+      }
       const float denom = has_stats ? z * (zf_c / zk_c) : z;
       const float inv = z > 0.f ? 1.f / denom : 0.f;
+      unsigned char* stg = smem + L::kOffQ + (i & 1) * T::kQBytes;
+      if (Tn > 0) {
+        if (!warp_wait(&sh.o_full, e & 1, abort_flag)) break;
+        tc_fence_after();
+      } else {
+        // No key tile: the Q load of this tile must land before its buffer is reused.
+        if (!warp_wait(&sh.q_full[i & 1], (i >> 1) & 1, abort_flag)) break;
+      }
+      // O (16 columns at a time) + e^{m_c - m'} U, normalised, as bf16 into the tile's Q
+      // buffer in the 128B / 32B swizzled layouts the TMA store expects.
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 16) {
-        float o[16];
-        if (T > 0) {
-          tmem_ld16(tmem + lane_off + kOCol + c0, o);
+        float v[16];
+        if (Tn > 0) {
+          tmem_ld16(tmem + lane_off + kOCol + c0, v);
         } else {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) o[c] = 0.f;
+          for (int c = 0; c < 16; ++c) v[c] = 0.f;
         }
-        if (valid) {
-          if (has_stats) {
-            const float4* up = reinterpret_cast<const float4*>(a.stat_u + row_g * D + c0);
+        uint32_t w[8];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const float4 u = __ldg(up + q4);
-              o[4 * q4 + 0] = fmaf(fu, u.x, o[4 * q4 + 0]);
-              o[4 * q4 + 1] = fmaf(fu, u.y, o[4 * q4 + 1]);
-              o[4 * q4 + 2] = fmaf(fu, u.z, o[4 * q4 + 2]);
-              o[4 * q4 + 3] = fmaf(fu, u.w, o[4 * q4 + 3]);
-            }
-          }
-          uint32_t w[8];
+        for (int c = 0; c < 16; c += 2) {
+          const float v0 = (c0 + c < a.d) ? fmaf(fu, u[c0 + c], v[c]) * inv : 0.f;
+          const float v1 = (c0 + c + 1 < a.d) ? fmaf(fu, u[c0 + c + 1], v[c + 1]) * inv : 0.f;
+          w[c / 2] = pack_bf16x2(v0, v1);
+        }
 #pragma unroll
-          for (int c = 0; c < 16; c += 2) {
-            const float v0 = (c0 + c < a.d && z > 0.f) ? o[c] * inv : 0.f;
-            const float v1 = (c0 + c + 1 < a.d && z > 0.f) ? o[c + 1] * inv : 0.f;
-            w[c / 2] = pack_bf16x2(v0, v1);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(a.out + row_g * D + c0);
-          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        for (int h = 0; h < 2; ++h) {
+          const int c8 = c0 + 8 * h;
+          unsigned char* dst;
+          if (c8 < 64) dst = stg + r * 128 + (((c8 >> 3) ^ (r & 7)) << 4);
+          else dst = stg + T::kQMain + r * 32 + ((((c8 - 64) >> 3) ^ ((r >> 2) & 1)) << 4);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]);
         }
       }
+      if (Tn > 0) {
+        tc_fence_before();
+        mbar_arrive(&sh.o_empty);
+        ++e;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&sh.staged[i & 1]);
     }
   }
 
@@ -502,39 +718,79 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   }
 }
 
-// ------------------------------------------------------------------ capture step
+// ================================================================== capture step
+//
+// One CTA per 128-row query tile, every key tile in order.  Each key tile's
+// P V goes to O_kept (rows whose query block keeps the tile's block) and/or
+// to U (the other rows), where U takes P as a bf16 high part plus a bf16
+// residual so the cached numerator keeps about 16 bits of P.  Head dim 64:
+// 256 TMEM columns (one S buffer) so two CTAs share an SM and two softmax
+// warps share each SM sub-partition.  Head dim 80: 512 columns (two S
+// buffers, one CTA per SM).
+template <int D>
+struct CaptureLayout {
+  using T = Tiles<D>;
+  static constexpr int kSBufs = D == 64 ? 1 : 2;
+  static constexpr uint32_t kTmemCols = D == 64 ? 256 : 512;
+  static constexpr uint32_t kPKCol = D == 64 ? 64 : 128;    // kept-rows P, 32 columns per buffer
+  static constexpr uint32_t kOKCol = D == 64 ? 128 : 256;   // O_kept accumulator
+  static constexpr uint32_t kOUCol = D == 64 ? 192 : 384;   // U accumulator
+  static constexpr int kStages = D == 64 ? 5 : 4;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffStage0 = T::kQBytes;
+  static constexpr int kOffShared = kOffStage0 + kStages * T::kStageBytes;
+  static constexpr size_t kMinSmem = D == 64 ? 0 : 120 * 1024;  // D = 80: keep one CTA per SM
+};
+
+struct alignas(8) CaptureShared {
+  uint64_t q_full;
+  uint64_t kv_full[8], kv_empty[8];
+  uint64_t s_full[2], p_full[2];
+  uint64_t pv_done, o_full, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int ok_any;  // some tile is kept by some row
+  int ou_any;  // some tile is masked for some row
+};
+
+template <int D>
+__host__ __device__ constexpr size_t capture_smem_bytes(int n_blocks) {
+  const size_t s = 1024 + CaptureLayout<D>::kOffShared + sizeof(CaptureShared) + 2 * sizeof(uint32_t) * attn_words(n_blocks);
+  return s < CaptureLayout<D>::kMinSmem ? CaptureLayout<D>::kMinSmem : s;
+}
+
 template <int D, int BS>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kAttnThreads, 2)
     full_capture_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tq_tail,
                         const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tk_tail,
                         const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tv_tail,
                         const AttnArgs a) {
-  using G = Geom<D>;
+  using T = Tiles<D>;
+  using L = CaptureLayout<D>;
   static_assert(BS == 64 || BS == 128, "block size must be 64 or 128");
-  constexpr int kQBPerCta = kBM / BS;
-  // S0 [0,64) S1 [64,128) PK0 [128,160) PK1 [160,192) O_kept [256,256+D) U [384,384+D)
-  constexpr uint32_t kTmemCols = 512;
-  constexpr uint32_t kPKCol = 128, kOKCol = 256, kOUCol = 384;
+  constexpr int kQB = kBM / BS;
+  constexpr int NS = L::kStages;
+  constexpr int SB = L::kSBufs;
 
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   unsigned char* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sbase = smem_u32(smem);
-  AttnShared& sh = *reinterpret_cast<AttnShared*>(smem + G::kOffBarriers);
+  CaptureShared& sh = *reinterpret_cast<CaptureShared*>(smem + L::kOffShared);
   const int words = attn_words(a.n_blocks);
   uint32_t* bitmaps = reinterpret_cast<uint32_t*>(&sh + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.y;
   const int q_row0 = blockIdx.x * kBM;
-  const int qb0 = blockIdx.x * kQBPerCta;
-  const int nqb_here = min(kQBPerCta, a.n_blocks - qb0);
-  const int T = (a.N + kBN - 1) / kBN;
+  const int qb0 = blockIdx.x * kQB;
+  const int nqb_here = min(kQB, a.n_blocks - qb0);
+  const int Tn = key_tiles(a.N);
 
-  if (warp == 0) tmem_alloc(&sh.tmem_base, kTmemCols);
+  if (warp == 0) tmem_alloc(&sh.tmem_base, L::kTmemCols);
   if (threadIdx.x == 32) {
     mbar_init(&sh.q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&sh.kv_full[s], 1);
       mbar_init(&sh.kv_empty[s], 1);
     }
@@ -553,16 +809,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   for (int i = threadIdx.x; i < 2 * words; i += blockDim.x) bitmaps[i] = 0u;
   __syncthreads();
   const bool run = sh.abort_flag == 0;  // block-uniform
-  if (run) load_block_bitmaps(bitmaps, words, a, bh, qb0, kQBPerCta);
+  if (run)
+    for (int g = 0; g < kQB; ++g) mark_kept_blocks(bitmaps + g * words, a, bh, qb0 + g, threadIdx.x, blockDim.x);
   __syncthreads();
-  // Which accumulators this CTA will touch at all.
-  for (int t = threadIdx.x; t < T; t += blockDim.x) {
-    const int kb = t * kBN / BS;
-    for (int g = 0; g < nqb_here; ++g) {
-      if (bitmap_has(bitmaps + g * words, kb)) sh.ok_any = 1;
-      else sh.ou_any = 1;
+  if (run)
+    for (int t = threadIdx.x; t < Tn; t += blockDim.x) {
+      const int kb = t * kBN / BS;
+      for (int g = 0; g < nqb_here; ++g) {
+        if (bitmap_has(bitmaps + g * words, kb)) sh.ok_any = 1;
+        else sh.ou_any = 1;
+      }
     }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -584,40 +841,58 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (!run) {
     // an earlier kernel failed: leave the outputs untouched
   } else if (warp == 0) {
-    if (lane == 0) produce<D>(sh, smem, &tq, &tq_tail, &tk, &tk_tail, &tv, &tv_tail, nullptr, T, q_row0, bh, true);
+    if (lane == 0) {
+      load_q<D>(smem + L::kOffQ, &tq, &tq_tail, &sh.q_full, q_row0, bh);
+      int issued = 0;
+      for (int j = 0; j < Tn; ++j) {
+        const int st = j % NS;
+        if (j >= NS && !mbar_wait(&sh.kv_empty[st], ((j / NS) - 1) & 1, abort_flag)) break;
+        load_kv<D>(smem + L::kOffStage0 + st * T::kStageBytes, &tk, &tk_tail, &tv, &tv_tail, &sh.kv_full[st],
+                   j * kBN, bh);
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        volatile int no_abort = 0;
+        mbar_wait(&sh.q_full, 0, &no_abort, kDrainLimitNs);
+        for (int j = issued > NS ? issued - NS : 0; j < issued; ++j)
+          mbar_wait(&sh.kv_full[j % NS], (j / NS) & 1, &no_abort, kDrainLimitNs);
+      }
+    }
   } else if (warp == 1) {
     if (lane == 0) {
       bool ok = mbar_wait(&sh.q_full, 0, abort_flag);
       bool ok_started = false, ou_started = false;
       auto pv = [&](int i) -> bool {
-        if (!mbar_wait(&sh.p_full[i & 1], (i >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(&sh.p_full[i % SB], (i / SB) & 1, abort_flag)) return false;
         tc_fence_after();
         bool kept_any, masked_any;
         tile_kind(i, kept_any, masked_any);
-        const uint32_t stage_base = sbase + G::kOffStage0 + (i % kStages) * G::kStageBytes;
+        const uint32_t v_base = sbase + L::kOffStage0 + (i % NS) * T::kStageBytes + T::kKVBytes;
         if (kept_any) {
-          issue_pv<D>(tmem + kOKCol, tmem + kPKCol + (i & 1) * 32, stage_base, ok_started);
+          issue_pv<D>(tmem + L::kOKCol, tmem + L::kPKCol + (i % SB) * 32, v_base, ok_started);
           ok_started = true;
         }
         if (masked_any) {
-          const uint32_t sbuf = tmem + (i & 1) * 64;
-          issue_pv<D>(tmem + kOUCol, sbuf, stage_base, ou_started);        // bf16(p)
-          issue_pv<D>(tmem + kOUCol, sbuf + 32, stage_base, true);         // p - bf16(p)
+          const uint32_t sbuf = tmem + (i % SB) * 64;
+          issue_pv<D>(tmem + L::kOUCol, sbuf, v_base, ou_started);   // bf16(p)
+          issue_pv<D>(tmem + L::kOUCol, sbuf + 32, v_base, true);    // p - bf16(p)
           ou_started = true;
         }
-        mma_commit(&sh.kv_empty[i % kStages]);
+        mma_commit(&sh.kv_empty[i % NS]);
         mma_commit(&sh.pv_done);
         return true;
       };
-      for (int j = 0; ok && j < T; ++j) {
-        const int st = j % kStages;
-        if (!mbar_wait(&sh.kv_full[st], (j / kStages) & 1, abort_flag)) { ok = false; break; }
+      for (int j = 0; ok && j < Tn; ++j) {
+        const int st = j % NS;
+        if (!mbar_wait(&sh.kv_full[st], (j / NS) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        issue_qk<D>(tmem + (j & 1) * 64, sbase, sbase + G::kOffStage0 + st * G::kStageBytes);
-        mma_commit(&sh.s_full[j & 1]);
-        if (j > 0 && !pv(j - 1)) ok = false;
+        // One S buffer: P(j-1) must be consumed before QK^T(j) overwrites it.
+        if (SB == 1 && j > 0 && !pv(j - 1)) { ok = false; break; }
+        issue_qk<D>(tmem + (j % SB) * 64, sbase + L::kOffQ, sbase + L::kOffStage0 + st * T::kStageBytes);
+        mma_commit(&sh.s_full[j % SB]);
+        if (SB == 2 && j > 0 && !pv(j - 1)) { ok = false; break; }
       }
-      if (ok && pv(T - 1)) mma_commit(&sh.o_full);
+      if (ok && pv(Tn - 1)) mma_commit(&sh.o_full);
       mma_commit(&sh.drain);
       volatile int no_abort = 0;
       mbar_wait(&sh.drain, 0, &no_abort, kDrainLimitNs);
@@ -626,21 +901,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const int g = r / BS;
+    const int grp = r / BS;
     const int i = q_row0 + r;
     const bool valid = i < a.N;
     const size_t row_g = static_cast<size_t>(bh) * a.N + (valid ? i : 0);
     const float C = a.scale_log2;
-    const uint32_t* my_bm = bitmaps + (g < nqb_here ? g : 0) * words;
+    const uint32_t* my_bm = bitmaps + (grp < nqb_here ? grp : 0) * words;
     float m_run = -INFINITY, m_seen = -INFINITY, zk = 0.f, zm = 0.f;
     bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      if (!mbar_wait(&sh.s_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+    for (int j = 0; j < Tn; ++j) {
+      if (!warp_wait(&sh.s_full[j % SB], (j / SB) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       bool kept_any, masked_any;
       tile_kind(j, kept_any, masked_any);
-      const bool kept = g < nqb_here && bitmap_has(my_bm, j * kBN / BS);
-      const uint32_t sbuf = tmem + lane_off + (j & 1) * 64;
+      const bool kept = grp < nqb_here && bitmap_has(my_bm, j * kBN / BS);  // warp-uniform
+      const uint32_t sbuf = tmem + lane_off + (j % SB) * 64;
       float s[64];
       tmem_ld64(sbuf, s);
       mask_tail(s, j * kBN, a.N);
@@ -650,11 +925,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (m_run == -INFINITY) ref = m_seen;
       else if (m_seen > m_run + kRescaleUp) { need = true; ref = m_seen; }
       if (__any_sync(0xffffffffu, need)) {
-        if (j > 0 && !mbar_wait(&sh.pv_done, (j - 1) & 1, abort_flag)) { ok = false; break; }
+        if (j > 0 && !warp_wait(&sh.pv_done, (j - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const float f = need ? ex2_approx(m_run - ref) : 1.f;
-        tmem_row_scale<D>(tmem + lane_off + kOKCol, f);
-        tmem_row_scale<D>(tmem + lane_off + kOUCol, f);
+        tmem_row_scale<D>(tmem + lane_off + L::kOKCol, f);
+        tmem_row_scale<D>(tmem + lane_off + L::kOUCol, f);
         zk *= f;
         zm *= f;
       }
@@ -663,14 +938,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) pk[c / 2] = pack_bf16x2(s[c], s[c + 1]);
-      if (kept) zk += zt; else zm += zt;
+      if (kept) zk += zt;
+      else zm += zt;
+      const uint32_t pkt = tmem + lane_off + L::kPKCol + (j % SB) * 32;
       if (kept_any) {
-        if (kept) {
-          tmem_st16(tmem + lane_off + kPKCol + (j & 1) * 32, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-          tmem_st16(tmem + lane_off + kPKCol + (j & 1) * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
-        } else {
-          tmem_st32_zero(tmem + lane_off + kPKCol + (j & 1) * 32);
-        }
+        if (kept) tmem_st32(pkt, pk);
+        else tmem_st32_zero(pkt);
       }
       if (masked_any) {
         if (!kept) {
@@ -678,10 +951,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int c = 0; c < 64; c += 2)
             lo[c / 2] = pack_bf16x2(s[c] - bf16_lo_to_f32(pk[c / 2]), s[c + 1] - bf16_hi_to_f32(pk[c / 2]));
-          tmem_st16(sbuf, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-          tmem_st16(sbuf + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
-          tmem_st16(sbuf + 32, *reinterpret_cast<const uint32_t(*)[16]>(&lo[0]));
-          tmem_st16(sbuf + 48, *reinterpret_cast<const uint32_t(*)[16]>(&lo[16]));
+          tmem_st32(sbuf, pk);
+          tmem_st32(sbuf + 32, lo);
         } else {
           tmem_st32_zero(sbuf);
           tmem_st32_zero(sbuf + 32);
@@ -689,9 +960,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&sh.p_full[j & 1]);
+      mbar_arrive(&sh.p_full[j % SB]);
     }
-    if (ok) ok = mbar_wait(&sh.o_full, 0, abort_flag);
+    if (ok) ok = warp_wait(&sh.o_full, 0, abort_flag);
     tc_fence_after();
     if (ok) {
       const float adj = ex2_approx(m_run - m_seen);  // <= 1: refer the cache to the true row max
@@ -700,12 +971,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 16) {
         float okv[16], ouv[16];
-        if (ok_any) tmem_ld16(tmem + lane_off + kOKCol + c0, okv);
+        if (ok_any) tmem_ld16(tmem + lane_off + L::kOKCol + c0, okv);
         else {
 #pragma unroll
           for (int c = 0; c < 16; ++c) okv[c] = 0.f;
         }
-        if (ou_any) tmem_ld16(tmem + lane_off + kOUCol + c0, ouv);
+        if (ou_any) tmem_ld16(tmem + lane_off + L::kOUCol + c0, ouv);
         else {
 #pragma unroll
           for (int c = 0; c < 16; ++c) ouv[c] = 0.f;
@@ -743,7 +1014,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 0) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 

@@ -91,49 +91,100 @@ bool make_map(CUtensorMap* m, const void* base, const Dims& d, int box_cols, int
 }
 
 struct Maps {
-  CUtensorMap q, q_tail, k, k_tail, v, v_tail;
+  CUtensorMap q, q_tail, k, k_tail, v, v_tail, o, o_tail;
 };
 
-bool make_maps(Maps* m, const Dims& d, const void* q, const void* k, const void* v) {
+bool make_maps(Maps* m, const Dims& d, const void* q, const void* k, const void* v, const void* out) {
   std::memset(m, 0, sizeof(*m));
   bool ok = make_map(&m->q, q, d, 64, rt::kBM, true) && make_map(&m->k, k, d, 64, rt::kBN, true) &&
-            make_map(&m->v, v, d, 64, rt::kBN, true);
+            make_map(&m->v, v, d, 64, rt::kBN, true) && make_map(&m->o, out, d, 64, rt::kBM, true);
   if (d.D == 80)
     ok = ok && make_map(&m->q_tail, q, d, 16, rt::kBM, false) && make_map(&m->k_tail, k, d, 16, rt::kBN, false) &&
-         make_map(&m->v_tail, v, d, 16, rt::kBN, false);
+         make_map(&m->v_tail, v, d, 16, rt::kBN, false) && make_map(&m->o_tail, out, d, 16, rt::kBM, false);
   else {
     m->q_tail = m->q;
     m->k_tail = m->k;
     m->v_tail = m->v;
+    m->o_tail = m->o;
   }
   return ok;
+}
+
+int sm_count() {
+  static int counts[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    counts[dev] = n;
+  }
+  return counts[dev];
 }
 
 rt_status launch_status() { return cudaGetLastError() == cudaSuccess ? RT_OK : RT_ERR_CUDA; }
 
 // ------------------------------------------------------------------ attention launch
-template <int D, int BS, bool kCapture>
-rt_status launch_attention(const Dims& d, const Maps& m, const AttnArgs& a, cudaStream_t stream) {
-  const int n_key_tiles = static_cast<int>((d.N + rt::kBN - 1) / rt::kBN);
-  size_t smem = rt::attn_smem_bytes<D>(static_cast<int>(d.n_blocks), n_key_tiles);
-  auto kernel = kCapture ? rt::full_capture_kernel<D, BS> : rt::sparse_reshape_kernel<D, BS>;
-  // The capture kernel holds all 512 TMEM columns: ask for enough shared
-  // memory that a second block can never share its SM.
-  if (kCapture && smem < 120 * 1024) smem = 120 * 1024;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-      cudaSuccess)
-    return RT_ERR_CUDA;
-  dim3 grid(static_cast<unsigned>((d.N + rt::kBM - 1) / rt::kBM), static_cast<unsigned>(d.bh));
+// Shared-memory size and the largest carveout, so two CTAs fit on an SM when their sizes allow.
+template <typename K>
+bool set_smem(K kernel, size_t smem) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) ==
+             cudaSuccess &&
+         cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              static_cast<int>(cudaSharedmemCarveoutMaxShared)) == cudaSuccess;
+}
+
+template <int D, int BS>
+rt_status launch_sparse(const Dims& d, const Maps& m, const AttnArgs& a, cudaStream_t stream) {
+  // Per-query-tile kept lists (transient, stream-ordered), then the persistent kernel.
+  const int N = static_cast<int>(d.N);
+  const int64_t tiles = rt::query_tiles(N) * d.bh;
+  const size_t list_bytes = sizeof(uint16_t) * static_cast<size_t>(tiles) * rt::tile_list_cap(N);
+  uint16_t* lists = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&lists), list_bytes, stream) != cudaSuccess) return RT_ERR_CUDA;
+  rt_status st = RT_OK;
+  const size_t bm_bytes = 2 * sizeof(uint32_t) * rt::attn_words(static_cast<int>(d.n_blocks));
+  rt::tile_lists_kernel<BS><<<static_cast<unsigned>(tiles), 32, bm_bytes, stream>>>(a, lists);
+  st = launch_status();
+  if (st == RT_OK) {
+    const size_t smem = rt::sparse_smem_bytes<D>(N);
+    auto kernel = rt::sparse_reshape_kernel<D, BS>;
+    if (!set_smem(kernel, smem)) {
+      st = RT_ERR_CUDA;
+    } else {
+      const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, 2 * sm_count()));
+      kernel<<<grid, rt::kAttnThreads, smem, stream>>>(m.q, m.q_tail, m.k, m.k_tail, m.v, m.v_tail, m.o, m.o_tail, a,
+                                                       lists);
+      st = launch_status();
+    }
+  }
+  if (cudaFreeAsync(lists, stream) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
+  return st;
+}
+
+template <int D, int BS>
+rt_status launch_capture(const Dims& d, const Maps& m, const AttnArgs& a, cudaStream_t stream) {
+  const size_t smem = rt::capture_smem_bytes<D>(static_cast<int>(d.n_blocks));
+  auto kernel = rt::full_capture_kernel<D, BS>;
+  if (!set_smem(kernel, smem)) return RT_ERR_CUDA;
+  dim3 grid(static_cast<unsigned>(rt::query_tiles(static_cast<int>(d.N))), static_cast<unsigned>(d.bh));
   kernel<<<grid, rt::kAttnThreads, smem, stream>>>(m.q, m.q_tail, m.k, m.k_tail, m.v, m.v_tail, a);
   return launch_status();
 }
 
 template <bool kCapture>
 rt_status dispatch_attention(const Dims& d, const Maps& m, const AttnArgs& a, cudaStream_t s) {
-  if (d.D == 64 && d.bs == 64) return launch_attention<64, 64, kCapture>(d, m, a, s);
-  if (d.D == 64 && d.bs == 128) return launch_attention<64, 128, kCapture>(d, m, a, s);
-  if (d.D == 80 && d.bs == 64) return launch_attention<80, 64, kCapture>(d, m, a, s);
-  if (d.D == 80 && d.bs == 128) return launch_attention<80, 128, kCapture>(d, m, a, s);
+  if (kCapture) {
+    if (d.D == 64 && d.bs == 64) return launch_capture<64, 64>(d, m, a, s);
+    if (d.D == 64 && d.bs == 128) return launch_capture<64, 128>(d, m, a, s);
+    if (d.D == 80 && d.bs == 64) return launch_capture<80, 64>(d, m, a, s);
+    if (d.D == 80 && d.bs == 128) return launch_capture<80, 128>(d, m, a, s);
+  } else {
+    if (d.D == 64 && d.bs == 64) return launch_sparse<64, 64>(d, m, a, s);
+    if (d.D == 64 && d.bs == 128) return launch_sparse<64, 128>(d, m, a, s);
+    if (d.D == 80 && d.bs == 64) return launch_sparse<80, 64>(d, m, a, s);
+    if (d.D == 80 && d.bs == 128) return launch_sparse<80, 128>(d, m, a, s);
+  }
   return RT_ERR_UNSUPPORTED;
 }
 
@@ -243,7 +294,7 @@ rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void*
     return RT_ERR_INVALID_ARGUMENT;
   if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
   Maps m;
-  if (!make_maps(&m, d, q, k, v)) return RT_ERR_CUDA;
+  if (!make_maps(&m, d, q, k, v, out)) return RT_ERR_CUDA;
   AttnArgs a{};
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
@@ -255,6 +306,7 @@ rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void*
   a.N = static_cast<int>(d.N);
   a.d = static_cast<int>(d.d);
   a.n_blocks = static_cast<int>(d.n_blocks);
+  a.n_heads = static_cast<int>(d.bh);
   a.scale_log2 = scale * rt::kLog2e;
   return dispatch_attention<true>(d, m, a, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -275,7 +327,7 @@ rt_status rt_attn_sparse_reshape(const rt_shape* shape, const void* q, const voi
     return RT_ERR_INVALID_ARGUMENT;
   if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
   Maps m;
-  if (!make_maps(&m, d, q, k, v)) return RT_ERR_CUDA;
+  if (!make_maps(&m, d, q, k, v, out)) return RT_ERR_CUDA;
   AttnArgs a{};
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
@@ -287,6 +339,7 @@ rt_status rt_attn_sparse_reshape(const rt_shape* shape, const void* q, const voi
   a.N = static_cast<int>(d.N);
   a.d = static_cast<int>(d.d);
   a.n_blocks = static_cast<int>(d.n_blocks);
+  a.n_heads = static_cast<int>(d.bh);
   a.scale_log2 = scale * rt::kLog2e;
   return dispatch_attention<false>(d, m, a, reinterpret_cast<cudaStream_t>(stream));
 }
