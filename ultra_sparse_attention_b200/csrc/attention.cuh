@@ -91,48 +91,39 @@ __host__ __device__ constexpr int attn_words(int n_blocks) { return (n_blocks + 
 __host__ __device__ constexpr int key_tiles(int N) { return (N + kBN - 1) / kBN; }
 __host__ __device__ constexpr int query_tiles(int N) { return (N + kBM - 1) / kBM; }
 
-// ------------------------------------------------------------------ descriptors and MMA issue
-template <int D>
-__device__ __forceinline__ uint64_t q_desc(uint32_t q_base, int ks) {
-  return ks < 4 ? smem_desc(q_base + ks * 32, 16, 1024, kSwizzle128B)
-                : smem_desc(q_base + Tiles<D>::kQMain, 16, 256, kSwizzle32B);
-}
-template <int D>
-__device__ __forceinline__ uint64_t k_desc(uint32_t k_base, int ks) {
-  return ks < 4 ? smem_desc(k_base + ks * 32, 16, 1024, kSwizzle128B)
-                : smem_desc(k_base + Tiles<D>::kKVMain, 16, 256, kSwizzle32B);
-}
-// V as the N-major B operand of P V: key rows are K, head-dim columns are N.
-template <int D>
-__device__ __forceinline__ uint64_t v_desc_main(uint32_t v_base, int ks) {
-  return smem_desc(v_base + ks * 2048, Tiles<D>::kKVMain, 1024, kSwizzle128B);
-}
-template <int D>
-__device__ __forceinline__ uint64_t v_desc_tail(uint32_t v_base, int ks) {
-  return smem_desc(v_base + Tiles<D>::kKVMain + ks * 512, Tiles<D>::kKVTail, 256, kSwizzle32B);
-}
-
+// ------------------------------------------------------------------ MMA issue
 constexpr uint32_t kIdescQK = idesc_bf16(kBM, kBN, false, false);
 constexpr uint32_t kIdescPV64 = idesc_bf16(kBM, 64, false, true);
 constexpr uint32_t kIdescPV16 = idesc_bf16(kBM, 16, false, true);
 
-// S = Q K^T for one key tile into TMEM at `s_tmem`.
+// S = Q K^T for one key tile into TMEM at `s_tmem`.  The descriptors are
+// built once and advanced by adding to their start-address field (16-byte
+// units): the per-MMA issue path is the critical resource of these kernels.
 template <int D>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_base, uint32_t k_base) {
+  const uint64_t qd = smem_desc(q_base, 16, 1024, kSwizzle128B);
+  const uint64_t kd = smem_desc(k_base, 16, 1024, kSwizzle128B);
+  mma_ss(s_tmem, qd, kd, kIdescQK, 0u);
 #pragma unroll
-  for (int ks = 0; ks < Tiles<D>::kKSteps; ++ks)
-    mma_ss(s_tmem, q_desc<D>(q_base, ks), k_desc<D>(k_base, ks), kIdescQK, ks > 0 ? 1u : 0u);
+  for (int ks = 1; ks < 4; ++ks) mma_ss(s_tmem, qd + 2 * ks, kd + 2 * ks, kIdescQK, 1u);
+  if constexpr (Tiles<D>::kTail)
+    mma_ss(s_tmem, smem_desc(q_base + Tiles<D>::kQMain, 16, 256, kSwizzle32B),
+           smem_desc(k_base + Tiles<D>::kKVMain, 16, 256, kSwizzle32B), kIdescQK, 1u);
 }
 
 // acc (+)= P V for one key tile; P is bf16 in TMEM at `p_tmem` (32 columns).
 template <int D>
 __device__ __forceinline__ void issue_pv(uint32_t acc_tmem, uint32_t p_tmem, uint32_t v_base, bool accumulate) {
+  const uint64_t vd = smem_desc(v_base, Tiles<D>::kKVMain, 1024, kSwizzle128B);
+  const uint32_t acc0 = accumulate ? 1u : 0u;
+  mma_ts(acc_tmem, p_tmem, vd, kIdescPV64, acc0);
 #pragma unroll
-  for (int ks = 0; ks < kBN / 16; ++ks) {
-    const uint32_t acc = (accumulate || ks > 0) ? 1u : 0u;
-    mma_ts(acc_tmem, p_tmem + ks * 8, v_desc_main<D>(v_base, ks), kIdescPV64, acc);
-    if constexpr (Tiles<D>::kTail)
-      mma_ts(acc_tmem + 64, p_tmem + ks * 8, v_desc_tail<D>(v_base, ks), kIdescPV16, acc);
+  for (int ks = 1; ks < kBN / 16; ++ks) mma_ts(acc_tmem, p_tmem + ks * 8, vd + 128 * ks, kIdescPV64, 1u);
+  if constexpr (Tiles<D>::kTail) {
+    const uint64_t vt = smem_desc(v_base + Tiles<D>::kKVMain, Tiles<D>::kKVTail, 256, kSwizzle32B);
+    mma_ts(acc_tmem + 64, p_tmem, vt, kIdescPV16, acc0);
+#pragma unroll
+    for (int ks = 1; ks < kBN / 16; ++ks) mma_ts(acc_tmem + 64, p_tmem + ks * 8, vt + 32 * ks, kIdescPV16, 1u);
   }
 }
 
