@@ -134,6 +134,34 @@ def test_sparse_matches_oracle(cuda_device, N, d, D, bs, keep_frac, with_stats):
     compare_out(out.reshape(-1, D), want, d, "sparse O")
 
 
+@pytest.mark.parametrize("N,d,D,bs", [(1000, 64, 64, 64), (1000, 72, 80, 64), (200, 64, 64, 64), (896, 64, 64, 128)])
+@pytest.mark.parametrize("gain", [3.0, 0.25])
+def test_sparse_reshape_with_rescales(cuda_device, N, d, D, bs, gain):
+    """Sparse step on Q scaled by `gain` against statistics of the unscaled step.
+
+    With gain 3 the running maxima exceed the cached ones by far more than the
+    lazy-rescale margin, so O is rescaled on the first kept tiles of most rows
+    (including while the previous query tile's output is still pending); with
+    gain 1/4 no rescale happens but e^{m_c - m'} is large.  The oracle evaluates
+    the same reshape formula on the same inputs."""
+    w = _wl(N, d, D, bs, std=1.2, seed=5 * N + d, drift=0.0)
+    (h0, _), (d0, _) = _inputs(w, cuda_device)
+    q1 = (h0[0].float() * gain).to(torch.bfloat16)
+    h1 = (q1, h0[1], h0[2])
+    d1 = (q1.to(cuda_device), d0[1], d0[2])
+    bh, nb = w.batch * w.heads, w.n_blocks
+    keep = w.keep_blocks(Fraction(1, 2))
+    rp, ci = random_csr(bh, nb, keep, seed=N + 7)
+    st_o = oracle.full_capture(*h0, d, bs, w.scale, rp, ci)
+    st_d = _stats_to_dev(st_o, d0[0].shape, cuda_device)
+    out = usa.rt_attn_sparse_reshape(*d1, head_dim=d, block_size=bs, scale=w.scale, row_ptr=to_dev(rp, cuda_device),
+                                     col_idx=to_dev(ci, cuda_device), stats=st_d)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp, ci, st_o)
+    compare_out(out.reshape(-1, D), want, d, f"sparse O (Q x {gain})")
+
+
 # ------------------------------------------------------------------ invariants the pages fix
 @pytest.mark.parametrize("N,d,D,bs", [(1000, 72, 80, 64), (1000, 64, 64, 128)])
 def test_reshape_keep_all_equals_full_attention(cuda_device, N, d, D, bs):

@@ -96,19 +96,45 @@ constexpr uint32_t kIdescQK = idesc_bf16(kBM, kBN, false, false);
 constexpr uint32_t kIdescPV64 = idesc_bf16(kBM, 64, false, true);
 constexpr uint32_t kIdescPV16 = idesc_bf16(kBM, 16, false, true);
 
-// S = Q K^T for one key tile into TMEM at `s_tmem`.  The descriptors are
-// built once and advanced by adding to their start-address field (16-byte
-// units): the per-MMA issue path is the critical resource of these kernels.
+// S = Q K^T for one key tile into TMEM at `s_tmem`, Q and K in shared memory.
+// The issue helpers below are warp-collective (one elected lane issues).  The
+// descriptors are built once and advanced by adding to their start-address
+// field (16-byte units).
 template <int D>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_base, uint32_t k_base) {
   const uint64_t qd = smem_desc(q_base, 16, 1024, kSwizzle128B);
   const uint64_t kd = smem_desc(k_base, 16, 1024, kSwizzle128B);
-  mma_ss(s_tmem, qd, kd, kIdescQK, 0u);
+  mma_ss_w(s_tmem, qd, kd, kIdescQK, 0u);
 #pragma unroll
-  for (int ks = 1; ks < 4; ++ks) mma_ss(s_tmem, qd + 2 * ks, kd + 2 * ks, kIdescQK, 1u);
+  for (int ks = 1; ks < 4; ++ks) mma_ss_w(s_tmem, qd + 2 * ks, kd + 2 * ks, kIdescQK, 1u);
   if constexpr (Tiles<D>::kTail)
-    mma_ss(s_tmem, smem_desc(q_base + Tiles<D>::kQMain, 16, 256, kSwizzle32B),
-           smem_desc(k_base + Tiles<D>::kKVMain, 16, 256, kSwizzle32B), kIdescQK, 1u);
+    mma_ss_w(s_tmem, smem_desc(q_base + Tiles<D>::kQMain, 16, 256, kSwizzle32B),
+             smem_desc(k_base + Tiles<D>::kKVMain, 16, 256, kSwizzle32B), kIdescQK, 1u);
+}
+
+// The same with Q resident in TMEM (D/2 columns of bf16 pairs): only K is
+// read from shared memory, which keeps an N = 64 tile at the full MMA rate
+// (with both operands in shared memory it is bound by the shared-memory
+// bandwidth: 6 KB per 32-cycle MMA).
+template <int D>
+__device__ __forceinline__ void issue_qk_tq(uint32_t s_tmem, uint32_t q_tmem, uint32_t k_base) {
+  const uint64_t kd = smem_desc(k_base, 16, 1024, kSwizzle128B);
+  mma_ts_w(s_tmem, q_tmem, kd, kIdescQK, 0u);
+#pragma unroll
+  for (int ks = 1; ks < 4; ++ks) mma_ts_w(s_tmem, q_tmem + ks * 8, kd + 2 * ks, kIdescQK, 1u);
+  if constexpr (Tiles<D>::kTail)
+    mma_ts_w(s_tmem, q_tmem + 32, smem_desc(k_base + Tiles<D>::kKVMain, 16, 256, kSwizzle32B), kIdescQK, 1u);
+}
+
+// Copy a 128-row bf16 Q tile (K-major: 128-byte swizzled main part, 32-byte
+// swizzled tail for D = 80) into D/2 TMEM columns.
+template <int D>
+__device__ __forceinline__ void copy_q_to_tmem(uint32_t q_tmem, uint32_t q_base) {
+  const uint64_t qd = smem_desc(q_base, 16, 1024, kSwizzle128B);
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) tmem_cp_128x256b_w(q_tmem + ks * 8, qd + 2 * ks);
+  if constexpr (Tiles<D>::kTail)
+    tmem_cp_128x256b_w(q_tmem + 32, smem_desc(q_base + Tiles<D>::kQMain, 16, 256, kSwizzle32B));
 }
 
 // acc (+)= P V for one key tile; P is bf16 in TMEM at `p_tmem` (32 columns).
@@ -116,14 +142,14 @@ template <int D>
 __device__ __forceinline__ void issue_pv(uint32_t acc_tmem, uint32_t p_tmem, uint32_t v_base, bool accumulate) {
   const uint64_t vd = smem_desc(v_base, Tiles<D>::kKVMain, 1024, kSwizzle128B);
   const uint32_t acc0 = accumulate ? 1u : 0u;
-  mma_ts(acc_tmem, p_tmem, vd, kIdescPV64, acc0);
+  mma_ts_w(acc_tmem, p_tmem, vd, kIdescPV64, acc0);
 #pragma unroll
-  for (int ks = 1; ks < kBN / 16; ++ks) mma_ts(acc_tmem, p_tmem + ks * 8, vd + 128 * ks, kIdescPV64, 1u);
+  for (int ks = 1; ks < kBN / 16; ++ks) mma_ts_w(acc_tmem, p_tmem + ks * 8, vd + 128 * ks, kIdescPV64, 1u);
   if constexpr (Tiles<D>::kTail) {
     const uint64_t vt = smem_desc(v_base + Tiles<D>::kKVMain, Tiles<D>::kKVTail, 256, kSwizzle32B);
-    mma_ts(acc_tmem + 64, p_tmem, vt, kIdescPV16, acc0);
+    mma_ts_w(acc_tmem + 64, p_tmem, vt, kIdescPV16, acc0);
 #pragma unroll
-    for (int ks = 1; ks < kBN / 16; ++ks) mma_ts(acc_tmem + 64, p_tmem + ks * 8, vt + 32 * ks, kIdescPV16, 1u);
+    for (int ks = 1; ks < kBN / 16; ++ks) mma_ts_w(acc_tmem + 64, p_tmem + ks * 8, vt + 32 * ks, kIdescPV16, 1u);
   }
 }
 
@@ -199,16 +225,18 @@ __device__ __forceinline__ void mask_tail(float (&s)[64], int key0, int N) {
   }
 }
 
+// Row max of 64 scores: four independent 3-input max chains (short dependency depth).
 __device__ __forceinline__ float row_max64(const float (&s)[64]) {
-  float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+  float m[4];
 #pragma unroll
-  for (int c = 4; c < 64; c += 4) {
-    m0 = fmaxf(m0, s[c]);
-    m1 = fmaxf(m1, s[c + 1]);
-    m2 = fmaxf(m2, s[c + 2]);
-    m3 = fmaxf(m3, s[c + 3]);
-  }
-  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+  for (int k = 0; k < 4; ++k) m[k] = fmax3(s[k], s[k + 4], s[k + 8]);
+#pragma unroll
+  for (int c = 12; c < 60; c += 8)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m[k] = fmax3(m[k], s[c + k], s[c + 4 + k]);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) m[k] = fmaxf(m[k], s[60 + k]);
+  return fmax3(m[0], m[1], fmaxf(m[2], m[3]));
 }
 
 // p = 2^(s*C - ref) for 64 columns, packed as bf16 pairs; returns the fp32 sum of p.
@@ -294,21 +322,23 @@ __global__ void __launch_bounds__(32) tile_lists_kernel(const AttnArgs a, uint16
 // t = blockIdx.x, blockIdx.x + gridDim.x, ... in head-major order
 // (neighbouring CTAs share a head, so its K/V stay in L2).
 //
-// Measured on this part: a tcgen05.mma costs ~50 cycles to issue, a commit
-// ~90, an mbarrier test 100-200 even when the phase is complete, and a
-// hand-off between warps ~250.  The pipeline is built to keep those off the
-// per-key-tile path:
+// Measured on this part: a tcgen05.mma issued by an elected lane of a
+// converged warp costs ~11 cycles, a commit ~50, a wait on a completed
+// mbarrier ~60 and a hand-off between warps ~110-150.  The pipeline:
 //  * warp 0, lane 0 (producer): bulk-copies the precomputed list of tile i+2,
 //    loads Q(i) into one of two buffers, streams K(g) and V(g) of every key
 //    tile g into two rings under ONE barrier per key tile, and issues the TMA
 //    store of each finished tile (polled, so no warp ever waits on a store);
-//  * warp 1, lane 0 (MMA): step g issues PV(g-2), then QK^T(g), then one
-//    commit to step[g % 8] -- which tells the softmax that S(g) is ready and
-//    P[g & 1] (aliased into S) was consumed, and tells the producer that the
-//    K slot of g and the V slot of g-2 are free;
+//  * warp 1 (MMA, warp-collective issue): at the first key tile of a query
+//    tile it copies Q into TMEM (head dim 64); step g issues PV(g-2), then
+//    QK^T(g), then one commit to step[g % 8] -- which tells the softmax that
+//    S(g) is ready and P[g & 1] (aliased into S) was consumed, and tells the
+//    producer that the K slot of g and the V slot of g-2 are free;
 //  * warps 2-5 (softmax + epilogue): one row per thread; P is written as bf16
 //    into the first 32 columns of S[g & 1].
-// TMEM (256 columns): S0 [0,64) S1 [64,128) O [128,128+D).
+// TMEM (256 columns): S0 [0,64) S1 [64,128) O [128,128+D); head dim 64 adds
+// two Q buffers [192,224) [224,256), so QK^T reads only K from shared memory
+// (with both operands there an N = 64 QK^T is bound by shared-memory bandwidth).
 // The epilogue releases O right after reading it, combines it with U (whose
 // row each thread prefetched into L2 a tile earlier), and writes bf16 rows
 // into the tile's Q buffer, which the producer then stores with one TMA store.
@@ -355,6 +385,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   constexpr int NK = L::kNK, NV = L::kNV, NL = L::kNL;
   constexpr uint32_t kTmemCols = 256;
   constexpr uint32_t kOCol = 128;
+  constexpr uint32_t kQCol = 192;             // head dim 64: two Q buffers of 32 columns
+  constexpr bool kQTmem = D == 64;
 
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -480,50 +512,56 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer (one thread)
-    if (lane == 0) {
-      struct Item { int j, T, e; bool valid; };
-      Item q0{0, 0, 0, false}, q1{0, 0, 0, false};  // key tiles g-2 and g-1
-      int g = 0, e = 0, kslot = 0, vslot = 0;
-      bool ok = true;
-      // PV of key tile h = g - 2 (or later in the drain).
-      auto pv = [&](const Item& it, int h) -> bool {
-        if (!mbar_wait(&sh.p_full[h & 1], (h >> 1) & 1, abort_flag)) return false;
-        if (it.j == 0 && it.e >= 1 && !mbar_wait(&sh.o_empty, (it.e - 1) & 1, abort_flag)) return false;
+    // ---------------- MMA issuer (the whole warp; one elected lane issues)
+    struct Item { int j, T, e; bool valid; };
+    Item q0{0, 0, 0, false}, q1{0, 0, 0, false};  // key tiles g-2 and g-1
+    int g = 0, e = 0, kslot = 0, vslot = 0;
+    bool ok = true;
+    // PV of key tile h = g - 2 (or later in the drain).
+    auto pv = [&](const Item& it, int h) -> bool {
+      if (!warp_wait(&sh.p_full[h & 1], (h >> 1) & 1, abort_flag)) return false;
+      if (it.j == 0 && it.e >= 1 && !warp_wait(&sh.o_empty, (it.e - 1) & 1, abort_flag)) return false;
+      tc_fence_after();
+      issue_pv<D>(tmem + kOCol, tmem + (h & 1) * 64, sbase + L::kOffV + vslot * T::kKVBytes, it.j > 0);
+      if (++vslot == NV) vslot = 0;
+      if (it.j == it.T - 1) mma_commit_w(&sh.o_full);
+      return true;
+    };
+    for (int i = 0; ok && i < n_mine; ++i) {
+      if (!warp_wait(&sh.list_full[i % NL], (i / NL) & 1, abort_flag)) { ok = false; break; }
+      const int Tn = lists[(i % NL) * cap];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.list_empty[i % NL]);
+      if (Tn == 0) continue;
+      if (!warp_wait(&sh.q_full[i & 1], (i >> 1) & 1, abort_flag)) { ok = false; break; }
+      const uint32_t q_base = sbase + L::kOffQ + (i & 1) * T::kQBytes;
+      const uint32_t q_tm = tmem + kQCol + (e & 1) * 32;  // head dim 64: Q of the e-th non-empty tile
+      for (int j = 0; j < Tn; ++j, ++g) {
+        if (q0.valid && !pv(q0, g - 2)) { ok = false; break; }
+        // P(g-2) consumed means every QK^T up to g-2 is done, in particular those of the
+        // non-empty tile e-2, the last reader of this Q buffer.
+        if (kQTmem && j == 0) copy_q_to_tmem<D>(q_tm, q_base);
+        if (!warp_wait(&sh.kv_full[g & 7], (g >> 3) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        issue_pv<D>(tmem + kOCol, tmem + (h & 1) * 64, sbase + L::kOffV + vslot * T::kKVBytes, it.j > 0);
-        if (++vslot == NV) vslot = 0;
-        if (it.j == it.T - 1) mma_commit(&sh.o_full);
-        return true;
-      };
-      for (int i = 0; ok && i < n_mine; ++i) {
-        if (!mbar_wait(&sh.list_full[i % NL], (i / NL) & 1, abort_flag)) { ok = false; break; }
-        const int Tn = lists[(i % NL) * cap];
-        mbar_arrive(&sh.list_empty[i % NL]);
-        if (Tn == 0) continue;
-        if (!mbar_wait(&sh.q_full[i & 1], (i >> 1) & 1, abort_flag)) { ok = false; break; }
-        const uint32_t q_base = sbase + L::kOffQ + (i & 1) * T::kQBytes;
-        for (int j = 0; j < Tn; ++j, ++g) {
-          if (q0.valid && !pv(q0, g - 2)) { ok = false; break; }
-          if (!mbar_wait(&sh.kv_full[g & 7], (g >> 3) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          issue_qk<D>(tmem + (g & 1) * 64, q_base, sbase + L::kOffK + kslot * T::kKVBytes);
-          mma_commit(&sh.step[g & 7]);
-          if (++kslot == NK) kslot = 0;
-          q0 = q1;
-          q1 = Item{j, Tn, e, true};
-        }
-        ++e;
+        const uint32_t k_base = sbase + L::kOffK + kslot * T::kKVBytes;
+        if constexpr (kQTmem) issue_qk_tq<D>(tmem + (g & 1) * 64, q_tm, k_base);
+        else issue_qk<D>(tmem + (g & 1) * 64, q_base, k_base);
+        mma_commit_w(&sh.step[g & 7]);
+        if (++kslot == NK) kslot = 0;
+        q0 = q1;
+        q1 = Item{j, Tn, e, true};
       }
-      // Drain: the last two PVs, each closing a step of its own.
-      if (ok && q0.valid) ok = pv(q0, g - 2);
-      if (ok) mma_commit(&sh.step[g & 7]);
-      if (ok && q1.valid) ok = pv(q1, g - 1);
-      if (ok) mma_commit(&sh.step[(g + 1) & 7]);
-      mma_commit(&sh.drain);
-      volatile int no_abort = 0;
-      mbar_wait(&sh.drain, 0, &no_abort, kDrainLimitNs);
+      ++e;
     }
+    // Drain: the last two PVs, each closing a step of its own.
+    if (ok && q0.valid) ok = pv(q0, g - 2);
+    if (ok) mma_commit_w(&sh.step[g & 7]);
+    if (ok && q1.valid) ok = pv(q1, g - 1);
+    if (ok) mma_commit_w(&sh.step[(g + 1) & 7]);
+    mma_commit_w(&sh.drain);
+    volatile int no_abort = 0;
+    mbar_wait(&sh.drain, 0, &no_abort, kDrainLimitNs);
+    __syncwarp();
   } else {
     // ---------------- softmax + epilogue: one query row per thread (warps 2..5)
     const int quad = warp & 3;
@@ -582,11 +620,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           float s[64];
           tmem_ld64(pt, s);
           mask_tail(s, static_cast<int>(ent >> 2) * kBN, a.N);
-          float mx = fmax3(s[0], s[1], s[2]);
-#pragma unroll
-          for (int c = 3; c < 63; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
-          mx = fmaxf(mx, s[63]);
-          m_seen = fmaxf(m_seen, mx * C);
+          m_seen = fmaxf(m_seen, row_max64(s) * C);
           float ref = m_run;
           bool need = false;
           if (m_run == -INFINITY) {
@@ -747,7 +781,7 @@ struct alignas(8) CaptureShared {
 template <int D>
 __host__ __device__ constexpr size_t capture_smem_bytes(int n_blocks) {
   const size_t s = 1024 + CaptureLayout<D>::kOffShared + sizeof(CaptureShared) + 2 * sizeof(uint32_t) * attn_words(n_blocks);
-  return s < CaptureLayout<D>::kMinSmem ? CaptureLayout<D>::kMinSmem : s;
+  return s > CaptureLayout<D>::kMinSmem ? s : CaptureLayout<D>::kMinSmem;
 }
 
 template <int D, int BS>
@@ -850,44 +884,44 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      bool ok = mbar_wait(&sh.q_full, 0, abort_flag);
-      bool ok_started = false, ou_started = false;
-      auto pv = [&](int i) -> bool {
-        if (!mbar_wait(&sh.p_full[i % SB], (i / SB) & 1, abort_flag)) return false;
-        tc_fence_after();
-        bool kept_any, masked_any;
-        tile_kind(i, kept_any, masked_any);
-        const uint32_t v_base = sbase + L::kOffStage0 + (i % NS) * T::kStageBytes + T::kKVBytes;
-        if (kept_any) {
-          issue_pv<D>(tmem + L::kOKCol, tmem + L::kPKCol + (i % SB) * 32, v_base, ok_started);
-          ok_started = true;
-        }
-        if (masked_any) {
-          const uint32_t sbuf = tmem + (i % SB) * 64;
-          issue_pv<D>(tmem + L::kOUCol, sbuf, v_base, ou_started);   // bf16(p)
-          issue_pv<D>(tmem + L::kOUCol, sbuf + 32, v_base, true);    // p - bf16(p)
-          ou_started = true;
-        }
-        mma_commit(&sh.kv_empty[i % NS]);
-        mma_commit(&sh.pv_done);
-        return true;
-      };
-      for (int j = 0; ok && j < Tn; ++j) {
-        const int st = j % NS;
-        if (!mbar_wait(&sh.kv_full[st], (j / NS) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        // One S buffer: P(j-1) must be consumed before QK^T(j) overwrites it.
-        if (SB == 1 && j > 0 && !pv(j - 1)) { ok = false; break; }
-        issue_qk<D>(tmem + (j % SB) * 64, sbase + L::kOffQ, sbase + L::kOffStage0 + st * T::kStageBytes);
-        mma_commit(&sh.s_full[j % SB]);
-        if (SB == 2 && j > 0 && !pv(j - 1)) { ok = false; break; }
+    // MMA issuer: the whole warp, one elected lane issues.
+    bool ok = warp_wait(&sh.q_full, 0, abort_flag);
+    bool ok_started = false, ou_started = false;
+    auto pv = [&](int i) -> bool {
+      if (!warp_wait(&sh.p_full[i % SB], (i / SB) & 1, abort_flag)) return false;
+      tc_fence_after();
+      bool kept_any, masked_any;
+      tile_kind(i, kept_any, masked_any);
+      const uint32_t v_base = sbase + L::kOffStage0 + (i % NS) * T::kStageBytes + T::kKVBytes;
+      if (kept_any) {
+        issue_pv<D>(tmem + L::kOKCol, tmem + L::kPKCol + (i % SB) * 32, v_base, ok_started);
+        ok_started = true;
       }
-      if (ok && pv(Tn - 1)) mma_commit(&sh.o_full);
-      mma_commit(&sh.drain);
-      volatile int no_abort = 0;
-      mbar_wait(&sh.drain, 0, &no_abort, kDrainLimitNs);
+      if (masked_any) {
+        const uint32_t sbuf = tmem + (i % SB) * 64;
+        issue_pv<D>(tmem + L::kOUCol, sbuf, v_base, ou_started);   // bf16(p)
+        issue_pv<D>(tmem + L::kOUCol, sbuf + 32, v_base, true);    // p - bf16(p)
+        ou_started = true;
+      }
+      mma_commit_w(&sh.kv_empty[i % NS]);
+      mma_commit_w(&sh.pv_done);
+      return true;
+    };
+    for (int j = 0; ok && j < Tn; ++j) {
+      const int st = j % NS;
+      if (!warp_wait(&sh.kv_full[st], (j / NS) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      // One S buffer: P(j-1) must be consumed before QK^T(j) overwrites it.
+      if (SB == 1 && j > 0 && !pv(j - 1)) { ok = false; break; }
+      issue_qk<D>(tmem + (j % SB) * 64, sbase + L::kOffQ, sbase + L::kOffStage0 + st * T::kStageBytes);
+      mma_commit_w(&sh.s_full[j % SB]);
+      if (SB == 2 && j > 0 && !pv(j - 1)) { ok = false; break; }
     }
+    if (ok && pv(Tn - 1)) mma_commit_w(&sh.o_full);
+    mma_commit_w(&sh.drain);
+    volatile int no_abort = 0;
+    mbar_wait(&sh.drain, 0, &no_abort, kDrainLimitNs);
+    __syncwarp();
   } else {
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
