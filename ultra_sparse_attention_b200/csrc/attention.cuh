@@ -748,30 +748,38 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 // One CTA per 128-row query tile, every key tile in order.  Each key tile's
 // P V goes to O_kept (rows whose query block keeps the tile's block) and/or
 // to U (the other rows), where U takes P as a bf16 high part plus a bf16
-// residual so the cached numerator keeps about 16 bits of P.  Head dim 64:
-// 256 TMEM columns (one S buffer) so two CTAs share an SM and two softmax
-// warps share each SM sub-partition.  Head dim 80: 512 columns (two S
-// buffers, one CTA per SM).
+// residual so the cached numerator keeps about 16 bits of P.
+//
+// S is double-buffered in TMEM, so QK^T(j+1) runs while the softmax works on
+// tile j: the MMA warp issues QK^T(j+1) as soon as PV(j-1) -- the last reader
+// of that buffer -- is issued, then waits for P(j) and issues PV(j).
+// A tile that is kept by some rows and masked for others ("mixed"; a few per
+// cent of the tiles) needs P twice: the masked rows' high/low parts stay in
+// the S buffer (kept rows zero) for the U products, and the kept rows' P goes
+// to a shared-memory tile (masked rows zero) read by one SS product into
+// O_kept.
+// TMEM: S0 [0,64) S1 [64,128) O_kept [128,128+D) U at kOUCol.  Head dim 64
+// fits in 256 columns, so two CTAs share an SM (two softmax warps per SM
+// sub-partition); head dim 80 takes 512 columns and one CTA per SM.
 template <int D>
 struct CaptureLayout {
   using T = Tiles<D>;
-  static constexpr int kSBufs = D == 64 ? 1 : 2;
   static constexpr uint32_t kTmemCols = D == 64 ? 256 : 512;
-  static constexpr uint32_t kPKCol = D == 64 ? 64 : 128;    // kept-rows P, 32 columns per buffer
-  static constexpr uint32_t kOKCol = D == 64 ? 128 : 256;   // O_kept accumulator
-  static constexpr uint32_t kOUCol = D == 64 ? 192 : 384;   // U accumulator
-  static constexpr int kStages = D == 64 ? 5 : 4;
+  static constexpr uint32_t kOKCol = 128;
+  static constexpr uint32_t kOUCol = D == 64 ? 192 : 256;
+  static constexpr int kStages = 4;
   static constexpr int kOffQ = 0;
   static constexpr int kOffStage0 = T::kQBytes;
-  static constexpr int kOffShared = kOffStage0 + kStages * T::kStageBytes;
+  static constexpr int kOffPK = kOffStage0 + kStages * T::kStageBytes;  // 128 x 64 bf16, 128-byte swizzle
+  static constexpr int kOffShared = kOffPK + kBM * 128;
   static constexpr size_t kMinSmem = D == 64 ? 0 : 120 * 1024;  // D = 80: keep one CTA per SM
 };
 
 struct alignas(8) CaptureShared {
   uint64_t q_full;
-  uint64_t kv_full[8], kv_empty[8];
+  uint64_t kv_full[4], kv_empty[4];
   uint64_t s_full[2], p_full[2];
-  uint64_t pv_done, o_full, drain;
+  uint64_t pv_done, pk_free, o_full, drain;
   uint32_t tmem_base;
   int abort_flag;
   int ok_any;  // some tile is kept by some row
@@ -782,6 +790,23 @@ template <int D>
 __host__ __device__ constexpr size_t capture_smem_bytes(int n_blocks) {
   const size_t s = 1024 + CaptureLayout<D>::kOffShared + sizeof(CaptureShared) + 2 * sizeof(uint32_t) * attn_words(n_blocks);
   return s > CaptureLayout<D>::kMinSmem ? s : CaptureLayout<D>::kMinSmem;
+}
+
+// acc (+)= P V with P (128 x 64 bf16) in shared memory, K-major with 128-byte swizzle.
+template <int D>
+__device__ __forceinline__ void issue_pv_ss(uint32_t acc_tmem, uint32_t p_base, uint32_t v_base, bool accumulate) {
+  const uint64_t pd = smem_desc(p_base, 16, 1024, kSwizzle128B);
+  const uint64_t vd = smem_desc(v_base, Tiles<D>::kKVMain, 1024, kSwizzle128B);
+  const uint32_t acc0 = accumulate ? 1u : 0u;
+  mma_ss_w(acc_tmem, pd, vd, kIdescPV64, acc0);
+#pragma unroll
+  for (int ks = 1; ks < kBN / 16; ++ks) mma_ss_w(acc_tmem, pd + 2 * ks, vd + 128 * ks, kIdescPV64, 1u);
+  if constexpr (Tiles<D>::kTail) {
+    const uint64_t vt = smem_desc(v_base + Tiles<D>::kKVMain, Tiles<D>::kKVTail, 256, kSwizzle32B);
+    mma_ss_w(acc_tmem + 64, pd, vt, kIdescPV16, acc0);
+#pragma unroll
+    for (int ks = 1; ks < kBN / 16; ++ks) mma_ss_w(acc_tmem + 64, pd + 2 * ks, vt + 32 * ks, kIdescPV16, 1u);
+  }
 }
 
 template <int D, int BS>
@@ -795,7 +820,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   static_assert(BS == 64 || BS == 128, "block size must be 64 or 128");
   constexpr int kQB = kBM / BS;
   constexpr int NS = L::kStages;
-  constexpr int SB = L::kSBufs;
 
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -824,6 +848,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       mbar_init(&sh.p_full[b], 128);
     }
     mbar_init(&sh.pv_done, 1);
+    mbar_init(&sh.pk_free, 1);
     mbar_init(&sh.o_full, 1);
     mbar_init(&sh.drain, 1);
     sh.abort_flag = device_status_set() ? 1 : 0;  // an earlier failure: do nothing
@@ -887,37 +912,45 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     // MMA issuer: the whole warp, one elected lane issues.
     bool ok = warp_wait(&sh.q_full, 0, abort_flag);
     bool ok_started = false, ou_started = false;
-    auto pv = [&](int i) -> bool {
-      if (!warp_wait(&sh.p_full[i % SB], (i / SB) & 1, abort_flag)) return false;
+    auto qk = [&](int j) -> bool {
+      const int st = j % NS;
+      if (!warp_wait(&sh.kv_full[st], (j / NS) & 1, abort_flag)) return false;
+      tc_fence_after();
+      issue_qk<D>(tmem + (j & 1) * 64, sbase + L::kOffQ, sbase + L::kOffStage0 + st * T::kStageBytes);
+      mma_commit_w(&sh.s_full[j & 1]);
+      return true;
+    };
+    auto pv = [&](int j) -> bool {
+      if (!warp_wait(&sh.p_full[j & 1], (j >> 1) & 1, abort_flag)) return false;
       tc_fence_after();
       bool kept_any, masked_any;
-      tile_kind(i, kept_any, masked_any);
-      const uint32_t v_base = sbase + L::kOffStage0 + (i % NS) * T::kStageBytes + T::kKVBytes;
-      if (kept_any) {
-        issue_pv<D>(tmem + L::kOKCol, tmem + L::kPKCol + (i % SB) * 32, v_base, ok_started);
+      tile_kind(j, kept_any, masked_any);
+      const uint32_t v_base = sbase + L::kOffStage0 + (j % NS) * T::kStageBytes + T::kKVBytes;
+      const uint32_t sbuf = tmem + (j & 1) * 64;
+      if (!masked_any) {  // kept by every row: P in the S buffer
+        issue_pv<D>(tmem + L::kOKCol, sbuf, v_base, ok_started);
         ok_started = true;
-      }
-      if (masked_any) {
-        const uint32_t sbuf = tmem + (i % SB) * 64;
+      } else {
         issue_pv<D>(tmem + L::kOUCol, sbuf, v_base, ou_started);   // bf16(p)
         issue_pv<D>(tmem + L::kOUCol, sbuf + 32, v_base, true);    // p - bf16(p)
         ou_started = true;
+        if (kept_any) {  // mixed: the kept rows' P is in shared memory
+          issue_pv_ss<D>(tmem + L::kOKCol, sbase + L::kOffPK, v_base, ok_started);
+          ok_started = true;
+          mma_commit_w(&sh.pk_free);
+        }
       }
-      mma_commit_w(&sh.kv_empty[i % NS]);
+      mma_commit_w(&sh.kv_empty[j % NS]);
       mma_commit_w(&sh.pv_done);
       return true;
     };
+    if (ok) ok = qk(0);
     for (int j = 0; ok && j < Tn; ++j) {
-      const int st = j % NS;
-      if (!warp_wait(&sh.kv_full[st], (j / NS) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      // One S buffer: P(j-1) must be consumed before QK^T(j) overwrites it.
-      if (SB == 1 && j > 0 && !pv(j - 1)) { ok = false; break; }
-      issue_qk<D>(tmem + (j % SB) * 64, sbase + L::kOffQ, sbase + L::kOffStage0 + st * T::kStageBytes);
-      mma_commit_w(&sh.s_full[j % SB]);
-      if (SB == 2 && j > 0 && !pv(j - 1)) { ok = false; break; }
+      // S[(j+1) & 1] held P(j-1), whose PV was issued in the previous iteration.
+      if (j + 1 < Tn && !qk(j + 1)) { ok = false; break; }
+      if (!pv(j)) { ok = false; break; }
     }
-    if (ok && pv(Tn - 1)) mma_commit_w(&sh.o_full);
+    if (ok) mma_commit_w(&sh.o_full);
     mma_commit_w(&sh.drain);
     volatile int no_abort = 0;
     mbar_wait(&sh.drain, 0, &no_abort, kDrainLimitNs);
@@ -934,13 +967,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const uint32_t* my_bm = bitmaps + (grp < nqb_here ? grp : 0) * words;
     float m_run = -INFINITY, m_seen = -INFINITY, zk = 0.f, zm = 0.f;
     bool ok = true;
+    int mixed = 0;  // mixed key tiles so far
     for (int j = 0; j < Tn; ++j) {
-      if (!warp_wait(&sh.s_full[j % SB], (j / SB) & 1, abort_flag)) { ok = false; break; }
+      if (!warp_wait(&sh.s_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       bool kept_any, masked_any;
       tile_kind(j, kept_any, masked_any);
       const bool kept = grp < nqb_here && bitmap_has(my_bm, j * kBN / BS);  // warp-uniform
-      const uint32_t sbuf = tmem + lane_off + (j % SB) * 64;
+      const uint32_t sbuf = tmem + lane_off + (j & 1) * 64;
       float s[64];
       tmem_ld64(sbuf, s);
       mask_tail(s, j * kBN, a.N);
@@ -965,12 +999,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       for (int c = 0; c < 64; c += 2) pk[c / 2] = pack_bf16x2(s[c], s[c + 1]);
       if (kept) zk += zt;
       else zm += zt;
-      const uint32_t pkt = tmem + lane_off + L::kPKCol + (j % SB) * 32;
-      if (kept_any) {
-        if (kept) tmem_st32(pkt, pk);
-        else tmem_st32_zero(pkt);
-      }
-      if (masked_any) {
+      if (!masked_any) {
+        tmem_st32(sbuf, pk);  // kept by every row
+      } else {
         if (!kept) {
           uint32_t lo[32];  // residual p - bf16(p), so U keeps ~16 mantissa bits of p
 #pragma unroll
@@ -982,10 +1013,24 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           tmem_st32_zero(sbuf);
           tmem_st32_zero(sbuf + 32);
         }
+        if (kept_any) {
+          // Mixed tile: the kept rows' P (masked rows zero) into the shared-memory tile, once
+          // the previous mixed tile's product has read it.
+          if (mixed > 0 && !warp_wait(&sh.pk_free, (mixed - 1) & 1, abort_flag)) { ok = false; break; }
+          unsigned char* prow = smem + L::kOffPK + r * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 val = kept ? make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3])
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = val;
+          }
+          fence_proxy_async_smem();
+          ++mixed;
+        }
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&sh.p_full[j % SB]);
+      mbar_arrive(&sh.p_full[j & 1]);
     }
     if (ok) ok = warp_wait(&sh.o_full, 0, abort_flag);
     tc_fence_after();
