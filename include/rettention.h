@@ -105,8 +105,10 @@ typedef struct rt_shape {
  * col_idx       out, int32 [B*H*n_blocks*keep_blocks] device.
  * block_scores  optional out (may be NULL), fp32 [B,H,n_blocks,n_blocks] device:
  *               the scores the selection used.
- * Takes a transient device workspace of 2*B*H*n_blocks*d*4 bytes from the
- * stream-ordered allocator on `stream` and returns it on the same stream.
+ * Takes a transient device workspace of 2*B*H*n_blocks*D*4 bytes (the pooled
+ * block means) on `stream` and returns it on the same stream.  Transient
+ * workspaces come from a stream-ordered memory pool the library creates once
+ * per device; it keeps freed memory cached for later calls.
  */
 rt_status rt_build_block_mask(const rt_shape *shape, const void *q, const void *k, float scale,
                               int32_t keep_blocks, int32_t forced_prefix_tokens,
@@ -159,6 +161,10 @@ rt_status rt_attn_full_capture(const rt_shape *shape, const void *q, const void 
  * row_ptr, col_idx  the CSR used at the capture step.
  * stat_*        fp32 statistics written by rt_attn_full_capture, or all NULL.
  * out           out, bf16 [B,H,N,D] device.
+ * Takes a transient workspace of ceil(N/128)*B*H*c uint16, c = ceil(N/64)+1
+ * rounded up to a multiple of 8 (the union of the kept key tiles of each
+ * 128-row query tile), from the library's
+ * stream-ordered pool (see rt_build_block_mask) and returns it on `stream`.
  */
 rt_status rt_attn_sparse_reshape(const rt_shape *shape, const void *q, const void *k,
                                  const void *v, float scale, const int32_t *row_ptr,

@@ -779,7 +779,7 @@ struct alignas(8) CaptureShared {
   uint64_t q_full;
   uint64_t kv_full[4], kv_empty[4];
   uint64_t s_full[2], p_full[2];
-  uint64_t pv_done, pk_free, o_full, drain;
+  uint64_t pk_free, o_full, drain;
   uint32_t tmem_base;
   int abort_flag;
   int ok_any;  // some tile is kept by some row
@@ -847,7 +847,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       mbar_init(&sh.s_full[b], 1);
       mbar_init(&sh.p_full[b], 128);
     }
-    mbar_init(&sh.pv_done, 1);
     mbar_init(&sh.pk_free, 1);
     mbar_init(&sh.o_full, 1);
     mbar_init(&sh.drain, 1);
@@ -940,8 +939,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           mma_commit_w(&sh.pk_free);
         }
       }
-      mma_commit_w(&sh.kv_empty[j % NS]);
-      mma_commit_w(&sh.pv_done);
+      mma_commit_w(&sh.kv_empty[j % NS]);  // K/V stage free and PV(j) done
       return true;
     };
     if (ok) ok = qk(0);
@@ -984,7 +982,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       if (m_run == -INFINITY) ref = m_seen;
       else if (m_seen > m_run + kRescaleUp) { need = true; ref = m_seen; }
       if (__any_sync(0xffffffffu, need)) {
-        if (j > 0 && !warp_wait(&sh.pv_done, (j - 1) & 1, abort_flag)) { ok = false; break; }
+        // PV(j-1) done: its commit also freed the K/V stage of tile j-1.
+        if (j > 0 && !warp_wait(&sh.kv_empty[(j - 1) % NS], ((j - 1) / NS) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const float f = need ? ex2_approx(m_run - ref) : 1.f;
         tmem_row_scale<D>(tmem + lane_off + L::kOKCol, f);
@@ -993,10 +992,25 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         zm *= f;
       }
       m_run = ref;
-      const float zt = exp_inplace64(s, C, m_run);  // s now holds p
+      // p = 2^(s*C - m'), two lanes of f32x2 arithmetic at a time; s now holds p.
       uint32_t pk[32];
+      float zt;
+      {
+        const uint64_t C2 = f2_pack(C, C), nref = f2_pack(-m_run, -m_run);
+        uint64_t zz = f2_pack(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) pk[c / 2] = pack_bf16x2(s[c], s[c + 1]);
+        for (int c = 0; c < 64; c += 2) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), C2, nref), x0, x1);
+          s[c] = ex2_approx(x0);
+          s[c + 1] = ex2_approx(x1);
+          zz = f2_add(zz, f2_pack(s[c], s[c + 1]));
+          pk[c / 2] = pack_bf16x2(s[c], s[c + 1]);
+        }
+        float z0, z1;
+        f2_unpack(zz, z0, z1);
+        zt = z0 + z1;
+      }
       if (kept) zk += zt;
       else zm += zt;
       if (!masked_any) {
@@ -1004,9 +1018,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       } else {
         if (!kept) {
           uint32_t lo[32];  // residual p - bf16(p), so U keeps ~16 mantissa bits of p
+          const uint64_t m1 = f2_pack(-1.f, -1.f);
 #pragma unroll
-          for (int c = 0; c < 64; c += 2)
-            lo[c / 2] = pack_bf16x2(s[c] - bf16_lo_to_f32(pk[c / 2]), s[c + 1] - bf16_hi_to_f32(pk[c / 2]));
+          for (int c = 0; c < 64; c += 2) {
+            float r0, r1;  // p - bf16(p), exact in fp32
+            f2_unpack(f2_fma(f2_pack(bf16_lo_to_f32(pk[c / 2]), bf16_hi_to_f32(pk[c / 2])), m1, f2_pack(s[c], s[c + 1])),
+                      r0, r1);
+            lo[c / 2] = pack_bf16x2(r0, r1);
+          }
           tmem_st32(sbuf, pk);
           tmem_st32(sbuf + 32, lo);
         } else {

@@ -124,6 +124,37 @@ int sm_count() {
 
 rt_status launch_status() { return cudaGetLastError() == cudaSuccess ? RT_OK : RT_ERR_CUDA; }
 
+// Transient workspaces (pooled block means, per-tile key lists) come from a
+// stream-ordered memory pool owned by the library, one per device, that keeps
+// freed memory cached instead of returning it to the driver at every
+// synchronisation: repeated calls then never wait in the driver's allocator.
+cudaMemPool_t workspace_pool() {
+  static std::mutex mu;
+  static cudaMemPool_t pools[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (pools[dev] == nullptr) {
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+    uint64_t keep = ~0ull;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    pools[dev] = pool;
+  }
+  return pools[dev];
+}
+
+bool workspace_alloc(void** p, size_t bytes, cudaStream_t s) {
+  cudaMemPool_t pool = workspace_pool();
+  if (pool == nullptr) return false;
+  return cudaMallocFromPoolAsync(p, bytes, pool, s) == cudaSuccess;
+}
+
 // ------------------------------------------------------------------ attention launch
 // Shared-memory size and the largest carveout, so two CTAs fit on an SM when their sizes allow.
 template <typename K>
@@ -141,7 +172,7 @@ rt_status launch_sparse(const Dims& d, const Maps& m, const AttnArgs& a, cudaStr
   const int64_t tiles = rt::query_tiles(N) * d.bh;
   const size_t list_bytes = sizeof(uint16_t) * static_cast<size_t>(tiles) * rt::tile_list_cap(N);
   uint16_t* lists = nullptr;
-  if (cudaMallocAsync(reinterpret_cast<void**>(&lists), list_bytes, stream) != cudaSuccess) return RT_ERR_CUDA;
+  if (!workspace_alloc(reinterpret_cast<void**>(&lists), list_bytes, stream)) return RT_ERR_CUDA;
   rt_status st = RT_OK;
   const size_t bm_bytes = 2 * sizeof(uint32_t) * rt::attn_words(static_cast<int>(d.n_blocks));
   rt::tile_lists_kernel<BS><<<static_cast<unsigned>(tiles), 32, bm_bytes, stream>>>(a, lists);
@@ -271,7 +302,7 @@ rt_status rt_build_block_mask(const rt_shape* shape, const void* q, const void* 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* pooled = nullptr;
   const size_t bytes = sizeof(float) * 2 * d.bh * d.n_blocks * d.D;
-  if (cudaMallocAsync(reinterpret_cast<void**>(&pooled), bytes, s) != cudaSuccess) return RT_ERR_CUDA;
+  if (!workspace_alloc(reinterpret_cast<void**>(&pooled), bytes, s)) return RT_ERR_CUDA;
   st = d.D == 64 ? launch_mask<64>(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx,
                                     block_scores, pooled, s)
                  : launch_mask<80>(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx,
