@@ -18,6 +18,7 @@ weak scaling).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import os
@@ -51,9 +52,14 @@ def parse_args():
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default="video5b", choices=sorted(WORKLOADS))
     p.add_argument("--keep", default=None, help="keep ratio as a fraction, e.g. 1/32 (default: the workload's)")
+    p.add_argument("--heads", type=int, default=None,
+                   help="override the workload's head count (small profiling cases of the same kernels)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=4096, help="rows in the oracle's bounded sample")
+    p.add_argument("--no-sweep", action="store_true", help="skip the per-workload sweep (single-GPU runs only)")
+    p.add_argument("--sweep-steps", type=int, default=10)
+    p.add_argument("--sweep-warmup", type=int, default=3)
     return p.parse_args()
 
 
@@ -184,6 +190,8 @@ def run_ours(args, rank, world, local):
     import ultra_sparse_attention_b200 as usa
 
     w = WORKLOADS[args.workload]
+    if args.heads:
+        w = dataclasses.replace(w, heads=args.heads)
     keep_ratio = Fraction(args.keep) if args.keep else w.keep[0]
     keep = w.keep_blocks(keep_ratio)
     device = torch.device("cuda", local)
@@ -288,6 +296,62 @@ def run_ours(args, rank, world, local):
             "host1": host1, "host0": host0}
 
 
+# --------------------------------------------------------------------------- configuration sweep
+def run_sweep(args, device) -> list:
+    """Per-kernel times of one mask + capture + sparse cycle on every workload
+    (the 5B shape at every keep ratio), L2 flushed between cycles."""
+    import ultra_sparse_attention_b200 as usa
+
+    peaks, _ = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # twice the L2
+    stream = torch.cuda.current_stream(device)
+    cases = [("tiny", None), ("image", None), ("video2b", None)]
+    cases += [("video5b", r) for r in WORKLOADS["video5b"].keep] + [("long", None)]
+    out = []
+    for name, ratio in cases:
+        w = WORKLOADS[name]
+        ratio = w.keep[0] if ratio is None else ratio
+        keep = w.keep_blocks(ratio)
+        steps = denoising_inputs(w, 2)
+        q0, k0, v0 = (x.to(device) for x in next(steps)[1:])
+        q1, k1, v1 = (x.to(device) for x in next(steps)[1:])
+        kw = dict(head_dim=w.head_dim, block_size=w.block_size, scale=w.scale)
+        times = {"mask": [], "capture": [], "sparse": []}
+        rp = ci = None
+        for it in range(args.sweep_warmup + args.sweep_steps):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record(stream)
+            rp, ci = usa.rt_build_block_mask(q0, k0, keep_blocks=keep, forced_prefix_tokens=w.forced_prefix_tokens, **kw)
+            ev[1].record(stream)
+            _, st = usa.rt_attn_full_capture(q0, k0, v0, row_ptr=rp, col_idx=ci, **kw)
+            ev[2].record(stream)
+            usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rp, col_idx=ci, stats=st, **kw)
+            ev[3].record(stream)
+            if it >= args.sweep_warmup:
+                times["mask"].append((ev[0], ev[1]))
+                times["capture"].append((ev[1], ev[2]))
+                times["sparse"].append((ev[2], ev[3]))
+        torch.cuda.synchronize()
+        if usa.rt_take_device_error() != 0:
+            raise RuntimeError(f"a kernel reported a device error in the sweep ({name})")
+        ms = {k: statistics.mean(a.elapsed_time(b) for a, b in v) for k, v in times.items()}
+        nums = workload_numbers(w, keep, rp.cpu().numpy(), ci.cpu().numpy())
+        sp_s, cap_s = ms["sparse"] / 1e3, ms["capture"] / 1e3
+        exe = nums["executed_flops"] / sp_s / 1e12
+        cap = nums["dense_flops"] / cap_s / 1e12
+        out.append({"workload": name, "shape": f"B={w.batch} H={w.heads} N={w.seq_len} d={w.head_dim} D={w.head_dim_padded} "
+                                               f"block={w.block_size}",
+                    "keep": f"{keep}/{w.n_blocks} ({ratio})", "sparse_step_ms": ms["sparse"],
+                    "full_step_ms": ms["mask"] + ms["capture"], "mask_ms": ms["mask"], "capture_ms": ms["capture"],
+                    "dense_equiv_tflops": nums["dense_flops"] / sp_s / 1e12, "executed_tflops": exe,
+                    "sparse_tensor_frac_of_bf16_peak": exe / peaks["bf16_tflops"],
+                    "capture_tflops": cap, "capture_frac_of_bf16_peak": cap / peaks["bf16_tflops"],
+                    "steps": args.sweep_steps, "warmup": args.sweep_warmup, "l2": "flushed between cycles"})
+        del q0, k0, v0, q1, k1, v1, st, rp, ci
+    return out
+
+
 # --------------------------------------------------------------------------- oracle timing (CPU)
 class OracleSample:
     """The fp64 oracle's sparse step on a bounded row sample of the workload.
@@ -328,6 +392,8 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     w = WORKLOADS[args.workload]
+    if args.heads:
+        w = dataclasses.replace(w, heads=args.heads)
     keep_ratio = Fraction(args.keep) if args.keep else w.keep[0]
     keep = w.keep_blocks(keep_ratio)
     steps = list(denoising_inputs(w, 2))
@@ -420,6 +486,9 @@ def main():
                    "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"],
                    "what": "sparse step through the public API: pinned host Q1/K1/V1 -> device, "
                            "rt_attn_sparse_reshape, output -> pinned host"}
+        sweep = None
+        if not args.no_sweep and world == 1:
+            sweep = run_sweep(args, torch.device("cuda", local))
         cpu = None
         if not args.no_cpu_baseline and world >= 1:
             cpu = OracleSample(w, r["keep"], r["host0"], r["host1"], args.cpu_rows).baseline()
@@ -434,6 +503,7 @@ def main():
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": r["clocks"],
             "peaks": {**peaks, "source": peak_src},
+            "sweep": sweep,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

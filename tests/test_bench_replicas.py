@@ -27,7 +27,7 @@ def _worker(rank, world, port, out):
         got = bench.max_over_ranks(mine, torch.device("cpu"), world)
         assert bench.dist_env() == (rank, world, rank)
         class A:  # the reference arm's arguments
-            workload, keep, cpu_rows, warmup, steps, gpus = "tiny", None, 64, 0, 1, world
+            workload, keep, heads, cpu_rows, warmup, steps, gpus = "tiny", None, None, 64, 0, 1, world
         ref = bench.run_reference(A, rank, world)
         dist.barrier()
         out[rank] = (got, ref is None)
