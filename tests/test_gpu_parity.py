@@ -93,6 +93,26 @@ def test_mask_exact_scores_and_ties_bit_exact(cuda_device):
         assert np.array_equal(ci.cpu().numpy(), ci_o), (keep, forced)
 
 
+def test_mask_threshold_selection_ties_bit_exact(cuda_device):
+    """More than eight chosen blocks take the threshold path of the selection:
+    64 blocks with exact scores and many duplicated key blocks, so the k-th
+    score is shared by several blocks; the CSR must equal the oracle's."""
+    B, H, N, d, bs = 1, 3, 4096, 64, 64
+    g = torch.Generator().manual_seed(11)
+    q = (torch.randint(-1, 2, (B, H, N, d), generator=g).float() / 4).to(torch.bfloat16)
+    k = (torch.randint(-1, 2, (B, H, N, d), generator=g).float() / 4).to(torch.bfloat16)
+    for dst in range(1, 64, 3):  # blocks 1, 4, 7, ... copy block dst // 2
+        src = dst // 2
+        k[:, :, dst * bs:(dst + 1) * bs] = k[:, :, src * bs:(src + 1) * bs]
+    scale = 0.125
+    for keep, forced in ((9, 0), (20, 0), (33, 130), (50, 0), (63, 64), (64, 0)):
+        rp, ci = usa.rt_build_block_mask(q.to(cuda_device), k.to(cuda_device), head_dim=d, block_size=bs,
+                                         scale=scale, keep_blocks=keep, forced_prefix_tokens=forced)
+        rp_o, ci_o = oracle.build_block_mask(q, k, d, bs, scale, keep, forced)
+        assert np.array_equal(rp.cpu().numpy(), rp_o)
+        assert np.array_equal(ci.cpu().numpy(), ci_o), (keep, forced)
+
+
 # ------------------------------------------------------------------ capture step
 @pytest.mark.parametrize("N,d,D,bs", CASES)
 @pytest.mark.parametrize("keep_frac", [Fraction(1, 4), Fraction(1, 1)])

@@ -11,9 +11,11 @@
 //   pool_blocks_kernel   reads Q and K once (HBM-bound), writes fp32 block
 //                        means [BH, n_blocks, D] (pad columns zero);
 //   score_select_kernel  one warp per query block: scores against every key
-//                        block from shared memory, then k rounds of a warp
-//                        arg-max with a (score desc, index asc) order, then a
-//                        ballot scan that writes the row sorted ascending.
+//                        block from shared memory, then the top k in the
+//                        (score desc, index asc) order -- up to 8 by rounds of
+//                        a warp arg-max, more by a threshold found with a
+//                        binary search over order-preserving score keys --
+//                        then a ballot scan that writes the row ascending.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -77,6 +79,15 @@ __host__ __device__ constexpr size_t score_select_smem_bytes(int n_blocks) {
   return sizeof(float) * (static_cast<size_t>(kSelChunk) * (D + 1) + kSelWarps * D +
                           static_cast<size_t>(kSelWarps) * n_blocks) +
          sizeof(uint32_t) * kSelWarps * select_words(n_blocks);
+}
+
+// Up to this many blocks are chosen by rounds of a warp arg-max; more by a threshold.
+constexpr int kSelRoundsMax = 8;
+
+// Unsigned key with the order of the float scores (-inf lowest; NaN never reaches here).
+__device__ __forceinline__ uint32_t order_key(float s) {
+  const uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 // (score, index) order of the selection: higher score first, lower index on ties.
@@ -143,7 +154,34 @@ __global__ void __launch_bounds__(32 * kSelWarps)
   const int forced = min(n_blocks, forced_tokens > 0 ? (forced_tokens + bs - 1) / bs : 0);
   for (int kb = lane; kb < forced; kb += 32) atomicOr(&my_taken[kb / 32], 1u << (kb % 32));
   __syncwarp();
-  for (int round = forced; round < keep; ++round) {
+  const int need = keep - forced;  // blocks to choose among kb >= forced
+  if (need > kSelRoundsMax) {
+    // Threshold selection: T = the need-th largest order key among the candidates (a binary
+    // search over the 32 key bits, one warp count per bit), then every candidate above T and
+    // the lowest-index candidates equal to T.  Same set as `need` rounds of the arg-max.
+    uint32_t T = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      int c = 0;
+      for (int kb = forced + lane; kb < n_blocks; kb += 32) c += order_key(my_sc[kb]) >= cand ? 1 : 0;
+      if (static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<uint32_t>(c))) >= need) T = cand;
+    }
+    int gt = 0;
+    for (int kb = forced + lane; kb < n_blocks; kb += 32) gt += order_key(my_sc[kb]) > T ? 1 : 0;
+    int ties_left = need - static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<uint32_t>(gt)));
+    for (int base = forced; base < n_blocks; base += 32) {
+      const int kb = base + lane;
+      const bool in = kb < n_blocks;
+      const uint32_t key = in ? order_key(my_sc[kb]) : 0u;
+      const bool tie = in && key == T;
+      const uint32_t tmask = __ballot_sync(0xffffffffu, tie);
+      const int before = __popc(tmask & ((1u << lane) - 1u));
+      if (in && (key > T || (tie && before < ties_left))) atomicOr(&my_taken[kb / 32], 1u << (kb % 32));
+      ties_left -= __popc(tmask);
+    }
+    __syncwarp();
+  }
+  for (int round = need > kSelRoundsMax ? keep : forced; round < keep; ++round) {
     float best_s = -INFINITY;
     int best_k = n_blocks;  // sentinel: loses to every real block
     for (int kb = forced + lane; kb < n_blocks; kb += 32) {
