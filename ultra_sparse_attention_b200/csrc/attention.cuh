@@ -239,33 +239,6 @@ __device__ __forceinline__ float row_max64(const float (&s)[64]) {
   return fmax3(m[0], m[1], fmaxf(m[2], m[3]));
 }
 
-// p = 2^(s*C - ref) for 64 columns, packed as bf16 pairs; returns the fp32 sum of p.
-__device__ __forceinline__ float exp_pack64(const float (&s)[64], float C, float ref, uint32_t (&pk)[32]) {
-  float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-  for (int c = 0; c < 64; c += 2) {
-    const float p0 = ex2_approx(fmaf(s[c], C, -ref));
-    const float p1 = ex2_approx(fmaf(s[c + 1], C, -ref));
-    z0 += p0;
-    z1 += p1;
-    pk[c / 2] = pack_bf16x2(p0, p1);
-  }
-  return z0 + z1;
-}
-
-// p = 2^(s*C - ref) in place for 64 columns; returns the fp32 sum of p.
-__device__ __forceinline__ float exp_inplace64(float (&s)[64], float C, float ref) {
-  float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-  for (int c = 0; c < 64; c += 2) {
-    s[c] = ex2_approx(fmaf(s[c], C, -ref));
-    s[c + 1] = ex2_approx(fmaf(s[c + 1], C, -ref));
-    z0 += s[c];
-    z1 += s[c + 1];
-  }
-  return z0 + z1;
-}
-
 __device__ __forceinline__ bool bitmap_has(const uint32_t* bm, int kb) { return (bm[kb / 32] >> (kb % 32)) & 1u; }
 
 // Set the bits of the kept key blocks of query block `qb` of head `bh` (threads `t0, t0+stride, ...`).
