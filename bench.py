@@ -357,9 +357,18 @@ def run_sweep(args, device) -> list:
                 times["mask"].append((ev[0], ev[1]))
                 times["capture"].append((ev[1], ev[2]))
                 times["sparse"].append((ev[2], ev[3]))
+        # How close the reshaped sparse step comes to full attention of its own inputs (the
+        # capture kernel's output on them), against plain block-sparse attention.
+        full1, _ = usa.rt_attn_full_capture(q1, k1, v1, row_ptr=rp, col_idx=ci, **kw)
+        resh1 = usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rp, col_idx=ci, stats=st, **kw)
+        plain1 = usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rp, col_idx=ci, stats=None, **kw)
         torch.cuda.synchronize()
         if usa.rt_take_device_error() != 0:
             raise RuntimeError(f"a kernel reported a device error in the sweep ({name})")
+        ref_norm = torch.linalg.vector_norm(full1.float()).item()
+        err_r = torch.linalg.vector_norm(resh1.float() - full1.float()).item() / ref_norm
+        err_p = torch.linalg.vector_norm(plain1.float() - full1.float()).item() / ref_norm
+        del full1, resh1, plain1
         ms = {k: statistics.mean(a.elapsed_time(b) for a, b in v) for k, v in times.items()}
         nums = workload_numbers(w, keep, rp.cpu().numpy(), ci.cpu().numpy())
         sp_s, cap_s = ms["sparse"] / 1e3, ms["capture"] / 1e3
@@ -372,6 +381,7 @@ def run_sweep(args, device) -> list:
                     "dense_equiv_tflops": nums["dense_flops"] / sp_s / 1e12, "executed_tflops": exe,
                     "sparse_tensor_frac_of_bf16_peak": exe / peaks["bf16_tflops"],
                     "capture_tflops": cap, "capture_frac_of_bf16_peak": cap / peaks["bf16_tflops"],
+                    "reshape_rel_l2_vs_full": err_r, "plain_sparse_rel_l2_vs_full": err_p,
                     "steps": args.sweep_steps, "warmup": args.sweep_warmup, "l2": "flushed between cycles"})
         del q0, k0, v0, q1, k1, v1, st, rp, ci
     return out
