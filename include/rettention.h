@@ -161,11 +161,7 @@ rt_status rt_attn_full_capture(const rt_shape *shape, const void *q, const void 
  * row_ptr, col_idx  the CSR used at the capture step.
  * stat_*        fp32 statistics written by rt_attn_full_capture, or all NULL.
  * out           out, bf16 [B,H,N,D] device.
- * Takes a transient workspace of ceil(N/128)*B*H*c uint16, c = ceil(N/64)+1
- * rounded up to a multiple of 8 (the union of the kept key tiles of each
- * 128-row query tile), from the library's
- * stream-ordered pool (see rt_build_block_mask) and returns it on `stream`.
- */
+*/
 rt_status rt_attn_sparse_reshape(const rt_shape *shape, const void *q, const void *k,
                                  const void *v, float scale, const int32_t *row_ptr,
                                  const int32_t *col_idx, const float *stat_m,

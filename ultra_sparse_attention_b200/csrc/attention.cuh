@@ -256,40 +256,12 @@ __device__ __forceinline__ void mark_kept_blocks(uint32_t* bm, const AttnArgs& a
 
 // ================================================================== sparse step (persistent)
 //
-// Kept key tiles of every 128-row query tile, precomputed from the CSR by
-// tile_lists_kernel: lists[t * cap] = count, lists[t * cap + 1 + j] =
+// Kept key tiles of a 128-row query tile, built from the CSR in shared memory
+// by the producer warp two tiles ahead: list[0] = count, list[1 + j] =
 // tile << 2 | (kept by query block 0) | (kept by query block 1) << 1, the
 // union of the tile's query blocks' kept lists in ascending order.
 __host__ __device__ constexpr int tile_list_cap(int N) { return (key_tiles(N) + 1 + 7) / 8 * 8; }
 
-template <int BS>
-__global__ void __launch_bounds__(32) tile_lists_kernel(const AttnArgs a, uint16_t* __restrict__ lists) {
-  extern __shared__ uint32_t bm[];  // [2][words]
-  constexpr int kQB = kBM / BS;
-  const int lane = threadIdx.x;
-  if (__shfl_sync(0xffffffffu, device_status_set() ? 1 : 0, 0)) return;  // an earlier kernel failed
-  const int n_qt = query_tiles(a.N), t = blockIdx.x, bh = t / n_qt, qt = t % n_qt;
-  const int words = attn_words(a.n_blocks), n_kt = key_tiles(a.N), cap = tile_list_cap(a.N);
-  for (int w = lane; w < 2 * words; w += 32) bm[w] = 0u;
-  __syncwarp();
-  for (int q = 0; q < kQB; ++q) mark_kept_blocks(bm + q * words, a, bh, qt * kQB + q, lane, 32);
-  __syncwarp();
-  uint16_t* out = lists + static_cast<size_t>(t) * cap;
-  int count = 0;
-  for (int t0 = 0; t0 < n_kt; t0 += 32) {
-    const int tile = t0 + lane;
-    uint32_t flags = 0u;
-    if (tile < n_kt) {
-      const int kb = tile * kBN / BS;
-      flags = bitmap_has(bm, kb) ? 1u : 0u;
-      if (kQB == 2) flags |= bitmap_has(bm + words, kb) ? 2u : 0u;
-    }
-    const uint32_t mask = __ballot_sync(0xffffffffu, flags != 0u);
-    if (flags) out[1 + count + __popc(mask & ((1u << lane) - 1u))] = static_cast<uint16_t>((tile << 2) | flags);
-    count += __popc(mask);
-  }
-  if (lane == 0) out[0] = static_cast<uint16_t>(count);
-}
 
 // The sparse kernel.  Grid: up to two CTAs per SM, each walking query tiles
 // t = blockIdx.x, blockIdx.x + gridDim.x, ... in head-major order
@@ -298,10 +270,11 @@ __global__ void __launch_bounds__(32) tile_lists_kernel(const AttnArgs a, uint16
 // Measured on this part: a tcgen05.mma issued by an elected lane of a
 // converged warp costs ~11 cycles, a commit ~50, a wait on a completed
 // mbarrier ~60 and a hand-off between warps ~110-150.  The pipeline:
-//  * warp 0, lane 0 (producer): bulk-copies the precomputed list of tile i+2,
-//    loads Q(i) into one of two buffers, streams K(g) and V(g) of every key
-//    tile g into two rings under ONE barrier per key tile, and issues the TMA
-//    store of each finished tile (polled, so no warp ever waits on a store);
+//  * warp 0 (producer): builds the key-tile list of tile i+2 from the CSR
+//    (kept-block bitmaps and a ballot scan), and its lane 0 loads Q(i) into
+//    one of two buffers, streams K(g) and V(g) of every key tile g into two
+//    rings under ONE barrier per key tile, and issues the TMA store of each
+//    finished tile (polled, so no warp ever waits on a store);
 //  * warp 1 (MMA, warp-collective issue): at the first key tile of a query
 //    tile it copies Q into TMEM (head dim 64); step g issues PV(g-2), then
 //    QK^T(g), then one commit to step[g % 8] -- which tells the softmax that
@@ -338,6 +311,7 @@ struct alignas(8) SparseShared {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
+  uint32_t list_bits[2 * 64];  // the producer's scratch: kept-block bitmaps of a tile's two query blocks
 };
 
 template <int D>
@@ -351,11 +325,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                           const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tk_tail,
                           const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tv_tail,
                           const __grid_constant__ CUtensorMap to, const __grid_constant__ CUtensorMap to_tail,
-                          const AttnArgs a, const uint16_t* __restrict__ tile_lists) {
+                          const AttnArgs a) {
   using T = Tiles<D>;
   using L = SparseLayout<D>;
   static_assert(BS == 64 || BS == 128, "block size must be 64 or 128");
   constexpr int NK = L::kNK, NV = L::kNV, NL = L::kNL;
+  constexpr int kQB = kBM / BS;
   constexpr uint32_t kTmemCols = 256;
   constexpr uint32_t kOCol = 128;
   constexpr uint32_t kQCol = 192;             // head dim 64: two Q buffers of 32 columns
@@ -371,6 +346,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = query_tiles(a.N);
+  const int n_kt = key_tiles(a.N);
+  const int words = attn_words(a.n_blocks);
   const int total = n_qt * a.n_heads;
   const int n_mine = total > static_cast<int>(blockIdx.x) ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   const bool has_stats = a.stat_m != nullptr;
@@ -387,8 +364,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       mbar_init(&sh.step[s], 1);
     }
     for (int s = 0; s < NL; ++s) {
-      mbar_init(&sh.list_full[s], 1);
-      mbar_init(&sh.list_empty[s], 5);  // the MMA thread + one lane of each softmax warp
+      mbar_init(&sh.list_full[s], 1);   // the producer, once the list is built
+      mbar_init(&sh.list_empty[s], 5);  // the MMA warp + one lane of each softmax warp
     }
     mbar_init(&sh.o_full, 1);
     mbar_init(&sh.o_empty, 128);
@@ -407,55 +384,85 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   if (!run) {
     // an earlier kernel failed: leave the outputs untouched
   } else if (warp == 0) {
-    // ---------------- producer (one thread)
-    if (lane == 0) {
-      int lists_issued = 0, stores_issued = 0, q_loads = 0, g = 0, kslot = 0, vslot = 0;
-      bool ok = true;
-      // Bring the list of tile `lists_issued` into its buffer; `block` waits for the buffer.
-      auto issue_list = [&](bool block) -> bool {
-        const int i = lists_issued, lb = i % NL;
-        if (i >= n_mine) return true;
-        if (i >= NL) {
-          const uint32_t par = ((i / NL) - 1) & 1;
-          if (block ? !mbar_wait(&sh.list_empty[lb], par, abort_flag) : !mbar_test(&sh.list_empty[lb], par))
-            return !block;
+    // ---------------- producer (the whole warp; lane 0 issues the copies)
+    int lists_built = 0, stores_issued = 0, q_loads = 0, g = 0, kslot = 0, vslot = 0;
+    bool ok = true;
+    uint32_t* bm = sh.list_bits;  // [2][words] scratch: the tile's query blocks' kept blocks
+    // Build the key-tile list of tile `lists_built` in its buffer from the CSR; `block` waits
+    // for the buffer, otherwise the call returns without building when it is still in use.
+    auto build_list = [&](bool block) -> bool {
+      const int i = lists_built, lb = i % NL;
+      if (i >= n_mine) return true;
+      if (i >= NL) {
+        const uint32_t par = ((i / NL) - 1) & 1;
+        if (block) {
+          if (!warp_wait(&sh.list_empty[lb], par, abort_flag)) return false;
+        } else if (!__all_sync(0xffffffffu, mbar_test(&sh.list_empty[lb], par))) {
+          return true;
         }
-        mbar_arrive_expect_tx(&sh.list_full[lb], 2 * cap);
-        bulk_load(lists + lb * cap, tile_lists + static_cast<size_t>(tile_of(i)) * cap, 2 * cap, &sh.list_full[lb]);
-        ++lists_issued;
+      }
+      const int t = tile_of(i), bh = t / n_qt, qt = t % n_qt;
+      for (int w = lane; w < 2 * words; w += 32) bm[w] = 0u;
+      __syncwarp();
+      for (int q = 0; q < kQB; ++q) mark_kept_blocks(bm + q * words, a, bh, qt * kQB + q, lane, 32);
+      __syncwarp();
+      uint16_t* out = lists + lb * cap;
+      int count = 0;
+      for (int t0 = 0; t0 < n_kt; t0 += 32) {
+        const int tile = t0 + lane;
+        uint32_t flags = 0u;
+        if (tile < n_kt) {
+          const int kb = tile * kBN / BS;
+          flags = bitmap_has(bm, kb) ? 1u : 0u;
+          if (kQB == 2) flags |= bitmap_has(bm + words, kb) ? 2u : 0u;
+        }
+        const uint32_t mask = __ballot_sync(0xffffffffu, flags != 0u);
+        if (flags) out[1 + count + __popc(mask & ((1u << lane) - 1u))] = static_cast<uint16_t>((tile << 2) | flags);
+        count += __popc(mask);
+      }
+      if (lane == 0) out[0] = static_cast<uint16_t>(count);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.list_full[lb]);
+      ++lists_built;
+      return true;
+    };
+    // Store the output of tile `stores_issued` once its epilogue has staged it.
+    auto issue_store = [&](bool block) -> bool {
+      const int i = stores_issued;
+      const uint32_t par = (i >> 1) & 1;
+      if (block) {
+        if (!warp_wait(&sh.staged[i & 1], par, abort_flag)) return false;
+      } else if (!__all_sync(0xffffffffu, mbar_test(&sh.staged[i & 1], par))) {
         return true;
-      };
-      // Store the output of tile `stores_issued` once its epilogue has staged it.
-      auto issue_store = [&](bool block) -> bool {
-        const int i = stores_issued;
-        const uint32_t par = (i >> 1) & 1;
-        if (block ? !mbar_wait(&sh.staged[i & 1], par, abort_flag) : !mbar_test(&sh.staged[i & 1], par))
-          return !block;
-        const int t = tile_of(i), bh = t / n_qt, qt = t % n_qt;
+      }
+      const int t = tile_of(i), bh = t / n_qt, qt = t % n_qt;
+      if (lane == 0) {
         const unsigned char* stg = smem + L::kOffQ + (i & 1) * T::kQBytes;
         tma_store_3d(&to, stg, 0, qt * kBM, bh);
         if constexpr (T::kTail) tma_store_3d(&to_tail, stg + T::kQMain, 64, qt * kBM, bh);
         bulk_commit_group();
-        ++stores_issued;
-        return true;
-      };
-      for (int i = 0; ok && i < n_mine; ++i) {
-        const int t = tile_of(i), bh = t / n_qt, qt = t % n_qt;
-        while (ok && lists_issued < i + 2 && lists_issued < n_mine) ok = issue_list(true);
+      }
+      ++stores_issued;
+      return true;
+    };
+    for (int i = 0; ok && i < n_mine; ++i) {
+      const int t = tile_of(i), bh = t / n_qt, qt = t % n_qt;
+      while (ok && lists_built < i + 2 && lists_built < n_mine) ok = build_list(true);
+      if (!ok) break;
+      const int count = lists[(i % NL) * cap];  // built by this warp
+      const uint16_t* lst = lists + (i % NL) * cap + 1;
+      // Q(i) reuses the buffer of tile i-2 once its output store has read it.
+      if (i >= 2) {
+        while (ok && stores_issued <= i - 2) ok = issue_store(true);
         if (!ok) break;
-        if (!mbar_wait(&sh.list_full[i % NL], (i / NL) & 1, abort_flag)) break;
-        const int count = lists[(i % NL) * cap];
-        const uint16_t* lst = lists + (i % NL) * cap + 1;
-        // Q(i) reuses the buffer of tile i-2 once its output store has read it.
-        if (i >= 2) {
-          while (ok && stores_issued <= i - 2) ok = issue_store(true);
-          if (!ok) break;
-          bulk_wait_group_read0();
-        }
-        load_q<D>(smem + L::kOffQ + (i & 1) * T::kQBytes, &tq, &tq_tail, &sh.q_full[i & 1], qt * kBM, bh);
-        ++q_loads;
-        for (int j = 0; j < count; ++j, ++g) {
-          if (g >= NK && !mbar_wait(&sh.step[(g - NK) & 7], ((g - NK) >> 3) & 1, abort_flag)) { ok = false; break; }
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+      }
+      if (lane == 0) load_q<D>(smem + L::kOffQ + (i & 1) * T::kQBytes, &tq, &tq_tail, &sh.q_full[i & 1], qt * kBM, bh);
+      ++q_loads;
+      for (int j = 0; j < count; ++j, ++g) {
+        if (g >= NK && !warp_wait(&sh.step[(g - NK) & 7], ((g - NK) >> 3) & 1, abort_flag)) { ok = false; break; }
+        if (lane == 0) {
           const int row0 = (lst[j] >> 2) * kBN;
           uint64_t* bar = &sh.kv_full[g & 7];
           mbar_arrive_expect_tx(bar, 2 * T::kKVBytes);
@@ -465,14 +472,17 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           if constexpr (T::kTail) tma_load_3d(kd + T::kKVMain, &tk_tail, bar, 64, row0, bh);
           tma_load_3d(vd, &tv, bar, 0, row0, bh);
           if constexpr (T::kTail) tma_load_3d(vd + T::kKVMain, &tv_tail, bar, 64, row0, bh);
-          if (++kslot == NK) kslot = 0;
-          if (++vslot == NV) vslot = 0;
-          // Opportunistic work that must not wait: the next list, a finished tile's store.
-          if (lists_issued < n_mine) issue_list(false);
-          if (stores_issued < i) issue_store(false);
         }
+        __syncwarp();
+        if (++kslot == NK) kslot = 0;
+        if (++vslot == NV) vslot = 0;
+        // Opportunistic work that must not wait: the next list, a finished tile's store.
+        if (lists_built < n_mine) build_list(false);
+        if (stores_issued < i) issue_store(false);
       }
-      while (ok && stores_issued < n_mine) ok = issue_store(true);
+    }
+    while (ok && stores_issued < n_mine) ok = issue_store(true);
+    if (lane == 0) {
       bulk_wait_group0();
       if (*abort_flag) {
         // Let every copy this block started land before the block exits.
@@ -480,10 +490,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         for (int i = q_loads > 2 ? q_loads - 2 : 0; i < q_loads; ++i)
           mbar_wait(&sh.q_full[i & 1], (i >> 1) & 1, &no_abort, kDrainLimitNs);
         for (int h = g > 8 ? g - 8 : 0; h < g; ++h) mbar_wait(&sh.kv_full[h & 7], (h >> 3) & 1, &no_abort, kDrainLimitNs);
-        for (int i = lists_issued > NL ? lists_issued - NL : 0; i < lists_issued; ++i)
-          mbar_wait(&sh.list_full[i % NL], (i / NL) & 1, &no_abort, kDrainLimitNs);
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ---------------- MMA issuer (the whole warp; one elected lane issues)
     struct Item { int j, T, e; bool valid; };

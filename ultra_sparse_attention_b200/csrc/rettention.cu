@@ -23,6 +23,8 @@ namespace {
 using rt::AttnArgs;
 
 constexpr int kMaxBlocks = 2048;
+// The sparse kernel's producer keeps two query blocks' kept-block bitmaps in shared memory.
+static_assert(2 * rt::attn_words(kMaxBlocks) <= 2 * 64, "sparse list scratch too small");
 
 // ------------------------------------------------------------------ validation
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -167,30 +169,15 @@ bool set_smem(K kernel, size_t smem) {
 
 template <int D, int BS>
 rt_status launch_sparse(const Dims& d, const Maps& m, const AttnArgs& a, cudaStream_t stream) {
-  // Per-query-tile kept lists (transient, stream-ordered), then the persistent kernel.
+  // One persistent kernel; it builds each query tile's key-tile list from the CSR itself.
   const int N = static_cast<int>(d.N);
   const int64_t tiles = rt::query_tiles(N) * d.bh;
-  const size_t list_bytes = sizeof(uint16_t) * static_cast<size_t>(tiles) * rt::tile_list_cap(N);
-  uint16_t* lists = nullptr;
-  if (!workspace_alloc(reinterpret_cast<void**>(&lists), list_bytes, stream)) return RT_ERR_CUDA;
-  rt_status st = RT_OK;
-  const size_t bm_bytes = 2 * sizeof(uint32_t) * rt::attn_words(static_cast<int>(d.n_blocks));
-  rt::tile_lists_kernel<BS><<<static_cast<unsigned>(tiles), 32, bm_bytes, stream>>>(a, lists);
-  st = launch_status();
-  if (st == RT_OK) {
-    const size_t smem = rt::sparse_smem_bytes<D>(N);
-    auto kernel = rt::sparse_reshape_kernel<D, BS>;
-    if (!set_smem(kernel, smem)) {
-      st = RT_ERR_CUDA;
-    } else {
-      const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, 2 * sm_count()));
-      kernel<<<grid, rt::kAttnThreads, smem, stream>>>(m.q, m.q_tail, m.k, m.k_tail, m.v, m.v_tail, m.o, m.o_tail, a,
-                                                       lists);
-      st = launch_status();
-    }
-  }
-  if (cudaFreeAsync(lists, stream) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
-  return st;
+  const size_t smem = rt::sparse_smem_bytes<D>(N);
+  auto kernel = rt::sparse_reshape_kernel<D, BS>;
+  if (!set_smem(kernel, smem)) return RT_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, 2 * sm_count()));
+  kernel<<<grid, rt::kAttnThreads, smem, stream>>>(m.q, m.q_tail, m.k, m.k_tail, m.v, m.v_tail, m.o, m.o_tail, a);
+  return launch_status();
 }
 
 template <int D, int BS>
