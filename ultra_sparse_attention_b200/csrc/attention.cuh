@@ -47,6 +47,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleUp = 8.f;    // log2 units
 constexpr float kRescaleDown = 64.f; // log2 units
+constexpr float kSumUp = 0x1p8f;      // 2^kRescaleUp
+constexpr float kSumDown = 0x1p-64f;  // 2^-kRescaleDown
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 
 // Tile byte sizes for head dim D (bf16 Q/K/V tiles).  A K or V tile is the
@@ -237,6 +239,23 @@ __device__ __forceinline__ float row_max64(const float (&s)[64]) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) m[k] = fmaxf(m[k], s[60 + k]);
   return fmax3(m[0], m[1], fmaxf(m[2], m[3]));
+}
+
+// One row's 64 scores to p = 2^(s*C - m): bf16 pairs into pk, returns their fp32 sum.
+__device__ __forceinline__ float exp_row64(const float (&s)[64], float m, uint64_t C2, uint32_t (&pk)[32]) {
+  const uint64_t nref = f2_pack(-m, -m);
+  uint64_t zz = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    float x0, x1;
+    f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), C2, nref), x0, x1);
+    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+    zz = f2_add(zz, f2_pack(p0, p1));
+    pk[c / 2] = pack_bf16x2(p0, p1);
+  }
+  float z0, z1;
+  f2_unpack(zz, z0, z1);
+  return z0 + z1;
 }
 
 __device__ __forceinline__ bool bitmap_has(const uint32_t* bm, int kb) { return (bm[kb / 32] >> (kb % 32)) & 1u; }
@@ -602,41 +621,43 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           float s[64];
           tmem_ld64(pt, s);
           mask_tail(s, static_cast<int>(ent >> 2) * kBN, a.N);
-          m_seen = fmaxf(m_seen, row_max64(s) * C);
-          float ref = m_run;
-          bool need = false;
-          if (m_run == -INFINITY) {
-            ref = m_seen;
-          } else if (m_seen > m_run + kRescaleUp || m_seen < m_run - kRescaleDown) {
-            need = true;
-            ref = m_seen;
+          // With a finite reference m' (the capture step's row max, or an earlier key tile's)
+          // the exponentials need no row max: only a tile sum above 2^kRescaleUp (some p may be
+          // that large) or a row total below 2^-kRescaleDown (all of it negligible) sends the
+          // warp to the max-based path, which recomputes the tile.
+          bool slow = true;
+          if (__all_sync(0xffffffffu, m_run != -INFINITY)) {
+            const float zt = exp_row64(s, m_run, C2, pk);
+            slow = __any_sync(0xffffffffu, !(zt <= kSumUp) || z + zt < kSumDown);
+            if (!slow) z += zt;
           }
-          if (__any_sync(0xffffffffu, need)) {
-            // Rescaling O needs PV(g-1) done: step g+1 (the previous tile's O is already read when j == 0).
-            if (j > 0 && !warp_wait(&sh.step[(g + 1) & 7], ((g + 1) >> 3) & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            const float f = need ? ex2_approx(m_run - ref) : 1.f;
-            tmem_row_scale<D>(tmem + lane_off + kOCol, f);
-            z *= f;
-          }
-          m_run = ref;
-          if (m_run == -INFINITY) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) pk[c] = 0u;
-          } else {
-            const uint64_t nref = f2_pack(-m_run, -m_run);
-            uint64_t zz = f2_pack(0.f, 0.f);
-#pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-              float x0, x1;
-              f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), C2, nref), x0, x1);
-              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-              zz = f2_add(zz, f2_pack(p0, p1));
-              pk[c / 2] = pack_bf16x2(p0, p1);
+          if (slow) {
+            // The earlier tiles' scores are at most m' + log2(z): none of their p exceeds z.
+            if (z > 0.f) m_seen = fmaxf(m_seen, m_run + __log2f(z));
+            m_seen = fmaxf(m_seen, row_max64(s) * C);
+            float ref = m_run;
+            bool need = false;
+            if (m_run == -INFINITY) {
+              ref = m_seen;
+            } else if (m_seen > m_run + kRescaleUp || m_seen < m_run - kRescaleDown) {
+              need = true;
+              ref = m_seen;
             }
-            float z0, z1;
-            f2_unpack(zz, z0, z1);
-            z += z0 + z1;
+            if (__any_sync(0xffffffffu, need)) {
+              // Rescaling O needs PV(g-1) done: step g+1 (the previous tile's O is already read when j == 0).
+              if (j > 0 && !warp_wait(&sh.step[(g + 1) & 7], ((g + 1) >> 3) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              const float f = need ? ex2_approx(m_run - ref) : 1.f;
+              tmem_row_scale<D>(tmem + lane_off + kOCol, f);
+              z *= f;
+            }
+            m_run = ref;
+            if (m_run == -INFINITY) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) pk[c] = 0u;
+            } else {
+              z += exp_row64(s, m_run, C2, pk);
+            }
           }
         } else {
 #pragma unroll
