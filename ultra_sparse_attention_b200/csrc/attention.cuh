@@ -571,8 +571,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const int grp = r / BS;
     const float C = a.scale_log2;
     const uint64_t C2 = f2_pack(C, C);
-    // Prefetch into L2 what the epilogue of tile i reads: this row's U and statistics.
-    auto prefetch_row = [&](int i) {
+    // Prefetch into L2 the row of U that the epilogue of tile i reads.
+    auto prefetch_u = [&](int i) {
       if (!has_stats || i >= n_mine) return;
       const int t = tile_of(i), bh = t / n_qt, row = (t % n_qt) * kBM + r;
       if (row >= a.N) return;
@@ -581,29 +581,34 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
       for (int off = 0; off < D * 4; off += 128) prefetch_l2(u + off);
       prefetch_l2(u + D * 4 - 4);
-      if ((r & 31) == 0) {
-        prefetch_l2(a.stat_m + rg);
-        prefetch_l2(a.stat_zfull + rg);
-        prefetch_l2(a.stat_zkept + rg);
-      }
     };
-    prefetch_row(0);
+    // This row's cached m, Z_full and Z_kept for tile i, read a tile ahead into registers
+    // (the neutral 0, 1, 1 for rows past N or without statistics).
+    auto load_stats = [&](int i, float& m, float& zf, float& zk) {
+      m = 0.f;
+      zf = 1.f;
+      zk = 1.f;
+      if (!has_stats || i >= n_mine) return;
+      const int t = tile_of(i), bh = t / n_qt, row = (t % n_qt) * kBM + r;
+      if (row >= a.N) return;
+      const size_t rg = static_cast<size_t>(bh) * a.N + row;
+      m = __ldg(a.stat_m + rg);
+      zf = __ldg(a.stat_zfull + rg);
+      zk = __ldg(a.stat_zkept + rg);
+    };
+    prefetch_u(0);
+    float next_m, next_zf, next_zk;
+    load_stats(0, next_m, next_zf, next_zk);
     int g = 0, e = 0;
     for (int i = 0; i < n_mine; ++i) {
-      prefetch_row(i + 1);
+      prefetch_u(i + 1);
       const int t = tile_of(i), bh = t / n_qt, qt = t % n_qt;
       const int row = qt * kBM + r;
       const bool valid = row < a.N;
       const size_t row_g = static_cast<size_t>(bh) * a.N + (valid ? row : 0);
-      float m_run = -INFINITY, mc2 = 0.f, zf_c = 1.f, zk_c = 1.f;
-      if (has_stats) {
-        if (valid) {
-          mc2 = __ldg(a.stat_m + row_g) * kLog2e;
-          zf_c = __ldg(a.stat_zfull + row_g);
-          zk_c = __ldg(a.stat_zkept + row_g);
-        }
-        m_run = mc2;
-      }
+      const float mc2 = next_m * kLog2e, zf_c = next_zf, zk_c = next_zk;
+      load_stats(i + 1, next_m, next_zf, next_zk);
+      float m_run = has_stats ? mc2 : -INFINITY;
       const int lb = i % NL;
       if (!warp_wait(&sh.list_full[lb], (i / NL) & 1, abort_flag)) break;
       const int Tn = lists[lb * cap];
