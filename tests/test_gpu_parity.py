@@ -182,6 +182,34 @@ def test_sparse_reshape_with_rescales(cuda_device, N, d, D, bs, gain):
     compare_out(out.reshape(-1, D), want, d, f"sparse O (Q x {gain})")
 
 
+@pytest.mark.parametrize("N,d,D,bs", [(1000, 64, 64, 64), (1000, 72, 80, 64)])
+@pytest.mark.parametrize("shift", [50.0, -10.0, 3.0])
+def test_sparse_reshape_cached_reference_shift(cuda_device, N, d, D, bs, shift):
+    """The reshape formula does not depend on which reference the statistics are cached
+    against: m_c + delta with Z_full, Z_kept and U scaled by e^-delta give the same output.
+
+    delta = 50 puts every kept p below 2^-64 of the shifted reference, so the kernel's
+    no-max fast path must hand the tile to the max-based path and rescale down; delta = -10
+    makes the tile sums exceed 2^8, the rescale-up hand-off; delta = 3 stays on the fast
+    path.  The expected output is the oracle's on the unshifted statistics."""
+    w = _wl(N, d, D, bs, std=1.0, seed=11 * N + d, drift=0.05)
+    (h0, h1), (d0, d1) = _inputs(w, cuda_device)
+    bh, nb = w.batch * w.heads, w.n_blocks
+    keep = w.keep_blocks(Fraction(1, 4))
+    rp, ci = random_csr(bh, nb, keep, seed=N + 3)
+    st_o = oracle.full_capture(*h0, d, bs, w.scale, rp, ci)
+    f = np.exp(-shift)
+    shifted = {"m": st_o["m"] + shift, "zfull": st_o["zfull"] * f, "zkept": st_o["zkept"] * f,
+               "u": st_o["u"] * f}
+    st_d = _stats_to_dev(shifted, d0[0].shape, cuda_device)
+    out = usa.rt_attn_sparse_reshape(*d1, head_dim=d, block_size=bs, scale=w.scale, row_ptr=to_dev(rp, cuda_device),
+                                     col_idx=to_dev(ci, cuda_device), stats=st_d)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp, ci, st_o)
+    compare_out(out.reshape(-1, D), want, d, f"sparse O (cached reference shifted by {shift})")
+
+
 # ------------------------------------------------------------------ invariants the pages fix
 @pytest.mark.parametrize("N,d,D,bs", [(1000, 72, 80, 64), (1000, 64, 64, 128)])
 def test_reshape_keep_all_equals_full_attention(cuda_device, N, d, D, bs):
