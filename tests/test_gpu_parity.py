@@ -182,6 +182,26 @@ def test_sparse_reshape_with_rescales(cuda_device, N, d, D, bs, gain):
     compare_out(out.reshape(-1, D), want, d, f"sparse O (Q x {gain})")
 
 
+@pytest.mark.parametrize("N,d,D,bs,keep", [(896, 64, 64, 128, 1), (2048, 72, 80, 128, 1), (1000, 64, 64, 64, 1),
+                                             (1000, 72, 80, 64, 1), (2048, 64, 64, 128, 2)])
+def test_sparse_reshape_short_query_tiles(cuda_device, N, d, D, bs, keep):
+    """Query tiles with one or two kept key tiles: fewer than the key tiles the MMA issuer
+    keeps in flight, so a tile's PVs are still pending when the query tile two ahead needs
+    its Q buffer back (the issuer must drain them first)."""
+    w = _wl(N, d, D, bs, std=1.0, seed=7 * N + keep, drift=0.05)
+    (h0, h1), (d0, d1) = _inputs(w, cuda_device)
+    bh, nb = w.batch * w.heads, w.n_blocks
+    rp, ci = random_csr(bh, nb, keep, seed=N + keep)
+    st_o = oracle.full_capture(*h0, d, bs, w.scale, rp, ci)
+    st_d = _stats_to_dev(st_o, d0[0].shape, cuda_device)
+    out = usa.rt_attn_sparse_reshape(*d1, head_dim=d, block_size=bs, scale=w.scale, row_ptr=to_dev(rp, cuda_device),
+                                     col_idx=to_dev(ci, cuda_device), stats=st_d)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp, ci, st_o)
+    compare_out(out.reshape(-1, D), want, d, f"sparse O (keep {keep} of {nb})")
+
+
 @pytest.mark.parametrize("N,d,D,bs", [(1000, 64, 64, 64), (1000, 72, 80, 64)])
 @pytest.mark.parametrize("shift", [50.0, -10.0, 3.0])
 def test_sparse_reshape_cached_reference_shift(cuda_device, N, d, D, bs, shift):

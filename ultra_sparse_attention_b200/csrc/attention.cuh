@@ -514,8 +514,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     __syncwarp();
   } else if (warp == 1) {
     // ---------------- MMA issuer (the whole warp; one elected lane issues)
-    struct Item { int j, T, e; bool valid; };
-    Item q0{0, 0, 0, false}, q1{0, 0, 0, false};  // key tiles g-2 and g-1
+    struct Item { int i, j, T, e; bool valid; };  // query tile, key tile in it, its count, non-empty ordinal
+    Item q0{-1, 0, 0, 0, false}, q1{-1, 0, 0, 0, false};  // key tiles g-2 and g-1, while their PV is pending
     int g = 0, e = 0, kslot = 0, vslot = 0;
     bool ok = true;
     // PV of key tile h = g - 2 (or later in the drain).
@@ -534,6 +534,18 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.list_empty[i % NL]);
       if (Tn == 0) continue;
+      // Q(i) reuses the buffer that tile i-2's output is stored from, which needs every PV of
+      // i-2; after a query tile with a single key tile one may still be pending: issue it now
+      // (the later step commits still cover it).
+      if (ok && q0.valid && q0.i <= i - 2) {
+        ok = pv(q0, g - 2);
+        q0.valid = false;
+      }
+      if (ok && q1.valid && q1.i <= i - 2) {
+        ok = pv(q1, g - 1);
+        q1.valid = false;
+      }
+      if (!ok) break;
       if (!warp_wait(&sh.q_full[i & 1], (i >> 1) & 1, abort_flag)) { ok = false; break; }
       const uint32_t q_base = sbase + L::kOffQ + (i & 1) * T::kQBytes;
       const uint32_t q_tm = tmem + kQCol + (e & 1) * 32;  // head dim 64: Q of the e-th non-empty tile
@@ -550,7 +562,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         mma_commit_w(&sh.step[g & 7]);
         if (++kslot == NK) kslot = 0;
         q0 = q1;
-        q1 = Item{j, Tn, e, true};
+        q1 = Item{i, j, Tn, e, true};
       }
       ++e;
     }
