@@ -34,7 +34,7 @@
  *    aligned, owned by the caller and never freed or retained by the library.
  *    Calls are asynchronous on `stream` (NULL = the legacy default stream);
  *    nothing is synchronised.
- *  - Supported: head_dim_padded in {64, 80}, 1 <= head_dim <= head_dim_padded,
+ *  - Supported: head_dim_padded in {64, 80, 128}, 1 <= head_dim <= head_dim_padded,
  *    block_size in {64, 128}, n_blocks <= 2048.
  *
  * Errors

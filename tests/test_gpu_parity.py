@@ -51,6 +51,8 @@ CASES = [
     (1000, 72, 80, 128),    # 8 blocks, last one 104 tokens
     (896, 64, 64, 128),     # exact multiple of the block size
     (200, 64, 64, 64),      # one ragged query tile, odd number of blocks (4: 64,64,64,8)
+    (1000, 128, 128, 64),   # head dim 128: a second 64-column tile part
+    (1000, 112, 128, 128),  # head dim 112 stored as 128 (zero pad)
 ]
 
 
@@ -154,7 +156,8 @@ def test_sparse_matches_oracle(cuda_device, N, d, D, bs, keep_frac, with_stats):
     compare_out(out.reshape(-1, D), want, d, "sparse O")
 
 
-@pytest.mark.parametrize("N,d,D,bs", [(1000, 64, 64, 64), (1000, 72, 80, 64), (200, 64, 64, 64), (896, 64, 64, 128)])
+@pytest.mark.parametrize("N,d,D,bs", [(1000, 64, 64, 64), (1000, 72, 80, 64), (200, 64, 64, 64), (896, 64, 64, 128),
+                                      (1000, 128, 128, 64)])
 @pytest.mark.parametrize("gain", [3.0, 0.25])
 def test_sparse_reshape_with_rescales(cuda_device, N, d, D, bs, gain):
     """Sparse step on Q scaled by `gain` against statistics of the unscaled step.
@@ -183,7 +186,7 @@ def test_sparse_reshape_with_rescales(cuda_device, N, d, D, bs, gain):
 
 
 @pytest.mark.parametrize("N,d,D,bs,keep", [(896, 64, 64, 128, 1), (2048, 72, 80, 128, 1), (1000, 64, 64, 64, 1),
-                                             (1000, 72, 80, 64, 1), (2048, 64, 64, 128, 2)])
+                                             (1000, 72, 80, 64, 1), (2048, 64, 64, 128, 2), (1000, 128, 128, 64, 1)])
 def test_sparse_reshape_short_query_tiles(cuda_device, N, d, D, bs, keep):
     """Query tiles with one or two kept key tiles: fewer than the key tiles the MMA issuer
     keeps in flight, so a tile's PVs are still pending when the query tile two ahead needs

@@ -51,21 +51,30 @@ constexpr float kSumUp = 0x1p8f;      // 2^kRescaleUp
 constexpr float kSumDown = 0x1p-64f;  // 2^-kRescaleDown
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 
-// Tile byte sizes for head dim D (bf16 Q/K/V tiles).  A K or V tile is the
-// 64-column part (128-byte swizzle) followed, for D = 80, by the 16-column
-// tail (32-byte swizzle).
+// Tile byte sizes for head dim D (bf16 Q/K/V tiles).  A tile is its 64-column
+// main part (128-byte rows, 128-byte swizzle) followed, for D > 64, by a tail
+// part: 16 columns (32-byte rows, 32-byte swizzle) for D = 80, another 64
+// columns laid out like the main part for D = 128.
 template <int D>
 struct Tiles {
-  static_assert(D == 64 || D == 80, "head_dim_padded must be 64 or 80");
-  static constexpr bool kTail = D == 80;
+  static_assert(D == 64 || D == 80 || D == 128, "head_dim_padded must be 64, 80 or 128");
+  static constexpr int kTailCols = D - 64;
+  static constexpr bool kTail = kTailCols > 0;
+  static constexpr bool kTailWide = kTailCols == 64;
+  static constexpr int kTailRow = kTailCols * 2;                          // bytes per tail row
+  static constexpr uint32_t kTailSwizzle = kTailWide ? kSwizzle128B : kSwizzle32B;
+  static constexpr int kTailSBO = 8 * kTailRow;                           // 8-row group stride
+  static constexpr int kTailKSteps = kTailCols / 16;
   static constexpr int kQMain = kBM * 128;
-  static constexpr int kQTail = kTail ? kBM * 32 : 0;
+  static constexpr int kQTail = kBM * kTailRow;
   static constexpr int kQBytes = kQMain + kQTail;
   static constexpr int kKVMain = kBN * 128;
-  static constexpr int kKVTail = kTail ? kBN * 32 : 0;
+  static constexpr int kKVTail = kBN * kTailRow;
   static constexpr int kKVBytes = kKVMain + kKVTail;   // one K or one V tile
   static constexpr int kStageBytes = 2 * kKVBytes;     // K tile then V tile
   static constexpr int kKSteps = D / 16;
+  // PV into the tail columns of the accumulator: N = the tail's width.
+  static constexpr uint32_t kIdescPVTail = idesc_bf16(kBM, kTail ? kTailCols : 16, false, true);
 };
 
 struct AttnArgs {
@@ -96,7 +105,6 @@ __host__ __device__ constexpr int query_tiles(int N) { return (N + kBM - 1) / kB
 // ------------------------------------------------------------------ MMA issue
 constexpr uint32_t kIdescQK = idesc_bf16(kBM, kBN, false, false);
 constexpr uint32_t kIdescPV64 = idesc_bf16(kBM, 64, false, true);
-constexpr uint32_t kIdescPV16 = idesc_bf16(kBM, 16, false, true);
 
 // S = Q K^T for one key tile into TMEM at `s_tmem`, Q and K in shared memory.
 // The issue helpers below are warp-collective (one elected lane issues).  The
@@ -109,9 +117,13 @@ __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_base, uint3
   mma_ss_w(s_tmem, qd, kd, kIdescQK, 0u);
 #pragma unroll
   for (int ks = 1; ks < 4; ++ks) mma_ss_w(s_tmem, qd + 2 * ks, kd + 2 * ks, kIdescQK, 1u);
-  if constexpr (Tiles<D>::kTail)
-    mma_ss_w(s_tmem, smem_desc(q_base + Tiles<D>::kQMain, 16, 256, kSwizzle32B),
-             smem_desc(k_base + Tiles<D>::kKVMain, 16, 256, kSwizzle32B), kIdescQK, 1u);
+  if constexpr (Tiles<D>::kTail) {
+    using T = Tiles<D>;
+    const uint64_t qt = smem_desc(q_base + T::kQMain, 16, T::kTailSBO, T::kTailSwizzle);
+    const uint64_t kt = smem_desc(k_base + T::kKVMain, 16, T::kTailSBO, T::kTailSwizzle);
+#pragma unroll
+    for (int ks = 0; ks < T::kTailKSteps; ++ks) mma_ss_w(s_tmem, qt + 2 * ks, kt + 2 * ks, kIdescQK, 1u);
+  }
 }
 
 // The same with Q resident in TMEM (D/2 columns of bf16 pairs): only K is
@@ -124,8 +136,7 @@ __device__ __forceinline__ void issue_qk_tq(uint32_t s_tmem, uint32_t q_tmem, ui
   mma_ts_w(s_tmem, q_tmem, kd, kIdescQK, 0u);
 #pragma unroll
   for (int ks = 1; ks < 4; ++ks) mma_ts_w(s_tmem, q_tmem + ks * 8, kd + 2 * ks, kIdescQK, 1u);
-  if constexpr (Tiles<D>::kTail)
-    mma_ts_w(s_tmem, q_tmem + 32, smem_desc(k_base + Tiles<D>::kKVMain, 16, 256, kSwizzle32B), kIdescQK, 1u);
+  static_assert(!Tiles<D>::kTail, "Q in TMEM is used for head dim 64 only");
 }
 
 // Copy a 128-row bf16 Q tile (K-major: 128-byte swizzled main part, 32-byte
@@ -135,8 +146,7 @@ __device__ __forceinline__ void copy_q_to_tmem(uint32_t q_tmem, uint32_t q_base)
   const uint64_t qd = smem_desc(q_base, 16, 1024, kSwizzle128B);
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks) tmem_cp_128x256b_w(q_tmem + ks * 8, qd + 2 * ks);
-  if constexpr (Tiles<D>::kTail)
-    tmem_cp_128x256b_w(q_tmem + 32, smem_desc(q_base + Tiles<D>::kQMain, 16, 256, kSwizzle32B));
+  static_assert(!Tiles<D>::kTail, "Q in TMEM is used for head dim 64 only");
 }
 
 // acc (+)= P V for one key tile; P is bf16 in TMEM at `p_tmem` (32 columns).
@@ -148,10 +158,12 @@ __device__ __forceinline__ void issue_pv(uint32_t acc_tmem, uint32_t p_tmem, uin
 #pragma unroll
   for (int ks = 1; ks < kBN / 16; ++ks) mma_ts_w(acc_tmem, p_tmem + ks * 8, vd + 128 * ks, kIdescPV64, 1u);
   if constexpr (Tiles<D>::kTail) {
-    const uint64_t vt = smem_desc(v_base + Tiles<D>::kKVMain, Tiles<D>::kKVTail, 256, kSwizzle32B);
-    mma_ts_w(acc_tmem + 64, p_tmem, vt, kIdescPV16, acc0);
+    using T = Tiles<D>;
+    const uint64_t vt = smem_desc(v_base + T::kKVMain, T::kKVTail, T::kTailSBO, T::kTailSwizzle);
+    mma_ts_w(acc_tmem + 64, p_tmem, vt, T::kIdescPVTail, acc0);
 #pragma unroll
-    for (int ks = 1; ks < kBN / 16; ++ks) mma_ts_w(acc_tmem + 64, p_tmem + ks * 8, vt + 32 * ks, kIdescPV16, 1u);
+    for (int ks = 1; ks < kBN / 16; ++ks)
+      mma_ts_w(acc_tmem + 64, p_tmem + ks * 8, vt + T::kTailRow * ks, T::kIdescPVTail, 1u);
   }
 }
 
@@ -553,7 +565,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         if (q0.valid && !pv(q0, g - 2)) { ok = false; break; }
         // P(g-2) consumed means every QK^T up to g-2 is done, in particular those of the
         // non-empty tile e-2, the last reader of this Q buffer.
-        if (kQTmem && j == 0) copy_q_to_tmem<D>(q_tm, q_base);
+        if constexpr (kQTmem) {
+          if (j == 0) copy_q_to_tmem<D>(q_tm, q_base);
+        }
         if (!warp_wait(&sh.kv_full[g & 7], (g >> 3) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t k_base = sbase + L::kOffK + kslot * T::kKVBytes;
@@ -690,15 +704,18 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       if (lane == 0) mbar_arrive(&sh.list_empty[lb]);
 
       // ---- epilogue
-      float u[D];
+      // U is read before waiting for O so its latency overlaps the last PV (its first 64
+      // columns for head dim 128, the rest as each 16-column chunk is combined).
+      constexpr int kUPre = D <= 80 ? D : 64;
+      const bool has_u = has_stats && valid;
+      const float4* up = reinterpret_cast<const float4*>(a.stat_u + row_g * D);
+      float u[kUPre];
 #pragma unroll
-      for (int c = 0; c < D; ++c) u[c] = 0.f;
+      for (int c = 0; c < kUPre; ++c) u[c] = 0.f;
       float fu = 0.f;
-      if (has_stats && valid) {
-        // U is read before waiting for O so its latency overlaps the last PV.
-        const float4* up = reinterpret_cast<const float4*>(a.stat_u + row_g * D);
+      if (has_u) {
 #pragma unroll
-        for (int q4 = 0; q4 < D / 4; ++q4) {
+        for (int q4 = 0; q4 < kUPre / 4; ++q4) {
           const float4 x = __ldg(up + q4);
           u[4 * q4 + 0] = x.x;
           u[4 * q4 + 1] = x.y;
@@ -728,11 +745,25 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
           for (int c = 0; c < 16; ++c) v[c] = 0.f;
         }
+        float uc[16];
+        if (c0 < kUPre) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) uc[c] = u[(c0 < kUPre ? c0 : 0) + c];
+        } else {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 x = has_u ? __ldg(up + c0 / 4 + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            uc[4 * q4 + 0] = x.x;
+            uc[4 * q4 + 1] = x.y;
+            uc[4 * q4 + 2] = x.z;
+            uc[4 * q4 + 3] = x.w;
+          }
+        }
         uint32_t w[8];
 #pragma unroll
         for (int c = 0; c < 16; c += 2) {
-          const float v0 = (c0 + c < a.d) ? fmaf(fu, u[c0 + c], v[c]) * inv : 0.f;
-          const float v1 = (c0 + c + 1 < a.d) ? fmaf(fu, u[c0 + c + 1], v[c + 1]) * inv : 0.f;
+          const float v0 = (c0 + c < a.d) ? fmaf(fu, uc[c], v[c]) * inv : 0.f;
+          const float v1 = (c0 + c + 1 < a.d) ? fmaf(fu, uc[c + 1], v[c + 1]) * inv : 0.f;
           w[c / 2] = pack_bf16x2(v0, v1);
         }
 #pragma unroll
@@ -740,6 +771,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           const int c8 = c0 + 8 * h;
           unsigned char* dst;
           if (c8 < 64) dst = stg + r * 128 + (((c8 >> 3) ^ (r & 7)) << 4);
+          else if (T::kTailWide) dst = stg + T::kQMain + r * 128 + ((((c8 - 64) >> 3) ^ (r & 7)) << 4);
           else dst = stg + T::kQMain + r * 32 + ((((c8 - 64) >> 3) ^ ((r >> 2) & 1)) << 4);
           *reinterpret_cast<uint4*>(dst) = make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]);
         }
@@ -792,7 +824,7 @@ struct CaptureLayout {
   static constexpr int kOffStage0 = T::kQBytes;
   static constexpr int kOffPK = kOffStage0 + kStages * T::kStageBytes;  // 128 x 64 bf16, 128-byte swizzle
   static constexpr int kOffShared = kOffPK + kBM * 128;
-  static constexpr size_t kMinSmem = D == 64 ? 0 : 120 * 1024;  // D = 80: keep one CTA per SM
+  static constexpr size_t kMinSmem = D == 64 ? 0 : 120 * 1024;  // D > 64: keep one CTA per SM
 };
 
 struct alignas(8) CaptureShared {
@@ -822,10 +854,12 @@ __device__ __forceinline__ void issue_pv_ss(uint32_t acc_tmem, uint32_t p_base, 
 #pragma unroll
   for (int ks = 1; ks < kBN / 16; ++ks) mma_ss_w(acc_tmem, pd + 2 * ks, vd + 128 * ks, kIdescPV64, 1u);
   if constexpr (Tiles<D>::kTail) {
-    const uint64_t vt = smem_desc(v_base + Tiles<D>::kKVMain, Tiles<D>::kKVTail, 256, kSwizzle32B);
-    mma_ss_w(acc_tmem + 64, pd, vt, kIdescPV16, acc0);
+    using T = Tiles<D>;
+    const uint64_t vt = smem_desc(v_base + T::kKVMain, T::kKVTail, T::kTailSBO, T::kTailSwizzle);
+    mma_ss_w(acc_tmem + 64, pd, vt, T::kIdescPVTail, acc0);
 #pragma unroll
-    for (int ks = 1; ks < kBN / 16; ++ks) mma_ss_w(acc_tmem + 64, pd + 2 * ks, vt + 32 * ks, kIdescPV16, 1u);
+    for (int ks = 1; ks < kBN / 16; ++ks)
+      mma_ss_w(acc_tmem + 64, pd + 2 * ks, vt + T::kTailRow * ks, T::kIdescPVTail, 1u);
   }
 }
 

@@ -39,7 +39,7 @@ rt_status check_shape(const rt_shape* s, Dims* out) {
       s->block_size <= 0)
     return RT_ERR_INVALID_ARGUMENT;
   if (s->head_dim > s->head_dim_padded) return RT_ERR_INVALID_ARGUMENT;
-  if (s->head_dim_padded != 64 && s->head_dim_padded != 80) return RT_ERR_UNSUPPORTED;
+  if (s->head_dim_padded != 64 && s->head_dim_padded != 80 && s->head_dim_padded != 128) return RT_ERR_UNSUPPORTED;
   if (s->block_size != 64 && s->block_size != 128) return RT_ERR_UNSUPPORTED;
   Dims d;
   d.B = s->batch;
@@ -100,10 +100,13 @@ bool make_maps(Maps* m, const Dims& d, const void* q, const void* k, const void*
   std::memset(m, 0, sizeof(*m));
   bool ok = make_map(&m->q, q, d, 64, rt::kBM, true) && make_map(&m->k, k, d, 64, rt::kBN, true) &&
             make_map(&m->v, v, d, 64, rt::kBN, true) && make_map(&m->o, out, d, 64, rt::kBM, true);
-  if (d.D == 80)
-    ok = ok && make_map(&m->q_tail, q, d, 16, rt::kBM, false) && make_map(&m->k_tail, k, d, 16, rt::kBN, false) &&
-         make_map(&m->v_tail, v, d, 16, rt::kBN, false) && make_map(&m->o_tail, out, d, 16, rt::kBM, false);
-  else {
+  if (d.D > 64) {
+    // Columns 64..D-1: 16 of them (32-byte swizzle) for D = 80, 64 (128-byte swizzle) for D = 128.
+    const int tc = static_cast<int>(d.D) - 64;
+    const bool wide = tc == 64;
+    ok = ok && make_map(&m->q_tail, q, d, tc, rt::kBM, wide) && make_map(&m->k_tail, k, d, tc, rt::kBN, wide) &&
+         make_map(&m->v_tail, v, d, tc, rt::kBN, wide) && make_map(&m->o_tail, out, d, tc, rt::kBM, wide);
+  } else {
     m->q_tail = m->q;
     m->k_tail = m->k;
     m->v_tail = m->v;
@@ -197,11 +200,15 @@ rt_status dispatch_attention(const Dims& d, const Maps& m, const AttnArgs& a, cu
     if (d.D == 64 && d.bs == 128) return launch_capture<64, 128>(d, m, a, s);
     if (d.D == 80 && d.bs == 64) return launch_capture<80, 64>(d, m, a, s);
     if (d.D == 80 && d.bs == 128) return launch_capture<80, 128>(d, m, a, s);
+    if (d.D == 128 && d.bs == 64) return launch_capture<128, 64>(d, m, a, s);
+    if (d.D == 128 && d.bs == 128) return launch_capture<128, 128>(d, m, a, s);
   } else {
     if (d.D == 64 && d.bs == 64) return launch_sparse<64, 64>(d, m, a, s);
     if (d.D == 64 && d.bs == 128) return launch_sparse<64, 128>(d, m, a, s);
     if (d.D == 80 && d.bs == 64) return launch_sparse<80, 64>(d, m, a, s);
     if (d.D == 80 && d.bs == 128) return launch_sparse<80, 128>(d, m, a, s);
+    if (d.D == 128 && d.bs == 64) return launch_sparse<128, 64>(d, m, a, s);
+    if (d.D == 128 && d.bs == 128) return launch_sparse<128, 128>(d, m, a, s);
   }
   return RT_ERR_UNSUPPORTED;
 }
@@ -233,6 +240,13 @@ rt_status launch_mask(const Dims& d, const void* q, const void* k, float scale, 
 // uses it never allocates.
 constexpr size_t kStaticPoolFloats = size_t(2) * 1024 * 1024;  // 8 MiB
 static __device__ __align__(256) float g_static_pool[kStaticPoolFloats];
+
+rt_status mask_for_dim(const Dims& d, const void* q, const void* k, float scale, int keep, int forced,
+                       int32_t* row_ptr, int32_t* col_idx, float* block_scores, float* pooled, cudaStream_t s) {
+  if (d.D == 64) return launch_mask<64>(d, q, k, scale, keep, forced, row_ptr, col_idx, block_scores, pooled, s);
+  if (d.D == 80) return launch_mask<80>(d, q, k, scale, keep, forced, row_ptr, col_idx, block_scores, pooled, s);
+  return launch_mask<128>(d, q, k, scale, keep, forced, row_ptr, col_idx, block_scores, pooled, s);
+}
 
 constexpr int kMaxDevices = 64;
 std::mutex g_static_pool_mutex;
@@ -290,10 +304,7 @@ rt_status rt_build_block_mask(const rt_shape* shape, const void* q, const void* 
   float* pooled = nullptr;
   const size_t bytes = sizeof(float) * 2 * d.bh * d.n_blocks * d.D;
   if (!workspace_alloc(reinterpret_cast<void**>(&pooled), bytes, s)) return RT_ERR_CUDA;
-  st = d.D == 64 ? launch_mask<64>(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx,
-                                    block_scores, pooled, s)
-                 : launch_mask<80>(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx,
-                                    block_scores, pooled, s);
+  st = mask_for_dim(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx, block_scores, pooled, s);
   if (cudaFreeAsync(pooled, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
   return st;
 }
@@ -382,10 +393,7 @@ rt_status rt_build_block_mask_static(const rt_shape* shape, const void* q, const
   st = static_pool_address(&pooled);
   if (st != RT_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return d.D == 64 ? launch_mask<64>(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx,
-                                      block_scores, pooled, s)
-                   : launch_mask<80>(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx,
-                                      block_scores, pooled, s);
+  return mask_for_dim(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx, block_scores, pooled, s);
 }
 
 rt_status rt_take_device_error(int32_t* code) {
