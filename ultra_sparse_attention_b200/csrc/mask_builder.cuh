@@ -74,9 +74,14 @@ constexpr int kSelChunk = 64;     // key blocks staged in shared memory at a tim
 
 __host__ __device__ constexpr int select_words(int n_blocks) { return (n_blocks + 31) / 32; }
 
+// Pooled rows in shared memory are D + 4 floats apart: 16-byte aligned for 128-bit loads, and
+// eight consecutive rows (one phase of a warp's 128-bit access) fall on distinct banks.
+template <int D>
+__host__ __device__ constexpr int sel_stride() { return D + 4; }
+
 template <int D>
 __host__ __device__ constexpr size_t score_select_smem_bytes(int n_blocks) {
-  return sizeof(float) * (static_cast<size_t>(kSelChunk) * (D + 1) + kSelWarps * D +
+  return sizeof(float) * (static_cast<size_t>(kSelChunk) * sel_stride<D>() + kSelWarps * D +
                           static_cast<size_t>(kSelWarps) * n_blocks) +
          sizeof(uint32_t) * kSelWarps * select_words(n_blocks);
 }
@@ -102,8 +107,10 @@ __global__ void __launch_bounds__(32 * kSelWarps)
                         int bs, float scale, int keep, int forced_tokens, int32_t* __restrict__ row_ptr,
                         int32_t* __restrict__ col_idx, float* __restrict__ block_scores) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* pk = reinterpret_cast<float*>(smem_raw);                 // [kSelChunk][D+1]
-  float* pq = pk + kSelChunk * (D + 1);                           // [kSelWarps][D]
+  constexpr int kS = sel_stride<D>();
+  static_assert(D % 4 == 0, "pooled rows are read as float4");
+  float* pk = reinterpret_cast<float*>(smem_raw);                 // [kSelChunk][D+4]
+  float* pq = pk + kSelChunk * kS;                                // [kSelWarps][D]
   float* sc = pq + kSelWarps * D;                                 // [kSelWarps][n_blocks]
   uint32_t* taken = reinterpret_cast<uint32_t*>(sc + kSelWarps * n_blocks);  // [kSelWarps][words]
   __shared__ int skip;
@@ -118,10 +125,11 @@ __global__ void __launch_bounds__(32 * kSelWarps)
   const int words = select_words(n_blocks);
   const size_t head = static_cast<size_t>(bh) * n_blocks;
 
-  for (int i = threadIdx.x; i < kSelWarps * D; i += blockDim.x) {
-    const int w = i / D, c = i % D;
+  for (int i = threadIdx.x; i < kSelWarps * (D / 4); i += blockDim.x) {
+    const int w = i / (D / 4), c4 = i % (D / 4);
     const int qq = blockIdx.x * kSelWarps + w;
-    pq[i] = qq < n_blocks ? pooled_q[(head + qq) * D + c] : 0.f;
+    reinterpret_cast<float4*>(pq + w * D)[c4] =
+        qq < n_blocks ? reinterpret_cast<const float4*>(pooled_q + (head + qq) * D)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   for (int i = threadIdx.x; i < kSelWarps * words; i += blockDim.x) taken[i] = 0u;
 
@@ -129,19 +137,26 @@ __global__ void __launch_bounds__(32 * kSelWarps)
   for (int kb0 = 0; kb0 < n_blocks; kb0 += kSelChunk) {
     __syncthreads();
     const int nch = min(kSelChunk, n_blocks - kb0);
-    for (int i = threadIdx.x; i < nch * D; i += blockDim.x) {
-      const int r = i / D, c = i % D;
-      pk[r * (D + 1) + c] = pooled_k[(head + kb0 + r) * D + c];
+    for (int i = threadIdx.x; i < nch * (D / 4); i += blockDim.x) {
+      const int r = i / (D / 4), c4 = i % (D / 4);
+      reinterpret_cast<float4*>(pk + r * kS)[c4] = reinterpret_cast<const float4*>(pooled_k + (head + kb0 + r) * D)[c4];
     }
     __syncthreads();
     if (have_row) {
-      const float* a = pq + warp * D;
+      const float4* a = reinterpret_cast<const float4*>(pq + warp * D);
       for (int r = lane; r < nch; r += 32) {
-        const float* b = pk + r * (D + 1);
-        float acc = 0.f;
-#pragma unroll 16
-        for (int c = 0; c < D; ++c) acc = fmaf(a[c], b[c], acc);
-        float s = scale * acc;
+        const float4* b = reinterpret_cast<const float4*>(pk + r * kS);
+        // Four partial sums (one per float4 lane) keep four FMA chains in flight.
+        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll
+        for (int c4 = 0; c4 < D / 4; ++c4) {
+          const float4 x = a[c4], y = b[c4];
+          acc0 = fmaf(x.x, y.x, acc0);
+          acc1 = fmaf(x.y, y.y, acc1);
+          acc2 = fmaf(x.z, y.z, acc2);
+          acc3 = fmaf(x.w, y.w, acc3);
+        }
+        float s = scale * ((acc0 + acc1) + (acc2 + acc3));
         if (s != s) s = -INFINITY;  // a NaN never wins
         my_sc[kb0 + r] = s;
       }
