@@ -129,7 +129,7 @@ int sm_count() {
 
 rt_status launch_status() { return cudaGetLastError() == cudaSuccess ? RT_OK : RT_ERR_CUDA; }
 
-// Transient workspaces (pooled block means, per-tile key lists) come from a
+// The mask builder's transient workspace (pooled block means) comes from a
 // stream-ordered memory pool owned by the library, one per device, that keeps
 // freed memory cached instead of returning it to the driver at every
 // synchronisation: repeated calls then never wait in the driver's allocator.
