@@ -327,3 +327,40 @@ def test_timeout_self_test_reports_and_recovers(cuda_device):
     assert usa.rt_take_device_error() == 0
     x = torch.ones(4, device=cuda_device)
     assert float(x.sum()) == 4.0
+
+
+# ------------------------------------------------------------------ maximum size
+def test_cycle_at_the_block_limit(cuda_device):
+    """One mask + capture + sparse cycle at the largest supported block count (2048 blocks
+    of 64 tokens, one head): the key-tile lists are at their longest and the sparse kernel's
+    list buffers push it to one CTA per SM.  Mask rows, then sampled rows of the capture and
+    the sparse step, against the oracle."""
+    N, d, bs = 2048 * 64, 64, 64
+    w = _wl(N, d, d, bs, B=1, H=1, std=1.0, seed=17, drift=0.05)
+    (h0, h1), (d0, d1) = _inputs(w, cuda_device)
+    keep = 16
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale)
+    rp, ci, sc = usa.rt_build_block_mask(d0[0], d0[1], keep_blocks=keep, block_scores=True, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    pq = oracle.pool_blocks(h0[0], d, bs)
+    pk = oracle.pool_blocks(h0[1], d, bs)
+    s64 = oracle.block_scores(pq, pk, w.scale)
+    tol = score_tol(s64)
+    assert np.max(np.abs(sc.double().cpu().numpy().reshape(s64.shape) - s64)) <= tol
+    rp_h, ci_h = rp.cpu().numpy(), ci.cpu().numpy()
+    assert check_mask(rp_h, ci_h, s64, keep, bs, 0, tol) <= 20
+
+    out0, st = usa.rt_attn_full_capture(*d0, row_ptr=rp, col_idx=ci, **kw)
+    out1 = usa.rt_attn_sparse_reshape(*d1, row_ptr=rp, col_idx=ci, stats=st, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    rng = np.random.default_rng(3)
+    rows = np.unique(np.concatenate([[0, 63, 64, 127, N - 129, N - 1], rng.choice(N, 90, replace=False)]))
+    idx = torch.as_tensor(rows, device=cuda_device)
+    orc = oracle.full_capture(*h0, d, bs, w.scale, rp_h, ci_h, rows=rows)
+    orc_abs = oracle.full_capture(h0[0], h0[1], h0[2].abs(), d, bs, w.scale, rp_h, ci_h, rows=rows)["u"]
+    compare_out(out0.reshape(-1, d)[idx], orc["o"], d, "capture O at the block limit")
+    compare_stats(st, rows, orc, orc_abs, d, "capture stats at the block limit")
+    want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp_h, ci_h, orc, rows=rows)
+    compare_out(out1.reshape(-1, d)[idx], want, d, "sparse O at the block limit")
