@@ -364,3 +364,28 @@ def test_cycle_at_the_block_limit(cuda_device):
     compare_stats(st, rows, orc, orc_abs, d, "capture stats at the block limit")
     want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp_h, ci_h, orc, rows=rows)
     compare_out(out1.reshape(-1, d)[idx], want, d, "sparse O at the block limit")
+
+
+# ------------------------------------------------------------------ degenerate lengths
+@pytest.mark.parametrize("N,d,D,bs", [(1, 64, 64, 64), (17, 72, 80, 64), (63, 64, 64, 64), (65, 64, 64, 64),
+                                      (129, 64, 64, 128), (1, 128, 128, 128)])
+def test_cycle_short_sequences(cuda_device, N, d, D, bs):
+    """Sequences shorter than one query tile, or one token past a block: the TMA boxes reach
+    past the tensor and every tile is ragged.  Mask, capture and sparse step on every row."""
+    w = _wl(N, d, D, bs, B=2, H=2, std=1.0, seed=100 + N, drift=0.05)
+    (h0, h1), (d0, d1) = _inputs(w, cuda_device)
+    nb = w.n_blocks
+    keep = max(1, nb // 2)
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale)
+    rp, ci = usa.rt_build_block_mask(d0[0], d0[1], keep_blocks=keep, **kw)
+    out0, st = usa.rt_attn_full_capture(*d0, row_ptr=rp, col_idx=ci, **kw)
+    out1 = usa.rt_attn_sparse_reshape(*d1, row_ptr=rp, col_idx=ci, stats=st, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    s64 = oracle.block_scores(oracle.pool_blocks(h0[0], d, bs), oracle.pool_blocks(h0[1], d, bs), w.scale)
+    rpo, cio = rp.cpu().numpy(), ci.cpu().numpy()  # checked against the oracle's selection
+    check_mask(rpo, cio, s64, keep, bs, 0, score_tol(s64))
+    orc = oracle.full_capture(*h0, d, bs, w.scale, rpo, cio)
+    compare_out(out0.reshape(-1, D), orc["o"], d, "capture O (short)")
+    want = oracle.sparse_reshape(*h1, d, bs, w.scale, rpo, cio, orc)
+    compare_out(out1.reshape(-1, D), want, d, "sparse O (short)")
