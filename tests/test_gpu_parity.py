@@ -389,3 +389,27 @@ def test_cycle_short_sequences(cuda_device, N, d, D, bs):
     compare_out(out0.reshape(-1, D), orc["o"], d, "capture O (short)")
     want = oracle.sparse_reshape(*h1, d, bs, w.scale, rpo, cio, orc)
     compare_out(out1.reshape(-1, D), want, d, "sparse O (short)")
+
+
+# ------------------------------------------------------------------ binding checks
+def test_binding_rejects_mismatched_buffers(cuda_device):
+    """Caller-supplied buffers of the wrong dtype, shape or device raise before any launch
+    (the C ABI cannot see buffer sizes)."""
+    B, H, N, d = 1, 2, 256, 64
+    q = torch.zeros(B, H, N, d, dtype=torch.bfloat16, device=cuda_device)
+    kw = dict(head_dim=d, block_size=64, scale=0.125)
+    rp, ci = usa.rt_build_block_mask(q, q, keep_blocks=2, **kw)
+    with pytest.raises(ValueError):
+        usa.rt_build_block_mask(q, q, keep_blocks=2, row_ptr=rp[:-1], **kw)              # too short
+    with pytest.raises(ValueError):
+        usa.rt_build_block_mask(q, q, keep_blocks=2, col_idx=ci.to(torch.int64), **kw)     # dtype
+    _, st = usa.rt_attn_full_capture(q, q, q, row_ptr=rp, col_idx=ci, **kw)
+    with pytest.raises(ValueError):
+        usa.rt_attn_full_capture(q, q, q, row_ptr=rp, col_idx=ci, out=q[:, :1], **kw)      # shape
+    bad = usa.Stats(st.m, st.zfull, st.zkept, st.u[..., :32].contiguous())
+    with pytest.raises(ValueError):
+        usa.rt_attn_sparse_reshape(q, q, q, row_ptr=rp, col_idx=ci, stats=bad, **kw)       # U width
+    with pytest.raises(ValueError):
+        usa.rt_attn_sparse_reshape(q, q, q, row_ptr=rp.cpu(), col_idx=ci, stats=st, **kw)  # device
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0

@@ -136,7 +136,27 @@ def _check_qkv(name: str, *xs: torch.Tensor) -> tuple[int, int, int, int]:
             shape = tuple(x.shape)
         elif tuple(x.shape) != shape:
             raise ValueError(f"{name}: Q/K/V shapes differ")
+        if x.device != xs[0].device:
+            raise ValueError(f"{name}: Q/K/V are on different devices")
     return shape
+
+
+def _check_buf(name: str, what: str, t: torch.Tensor, dtype: torch.dtype, device: torch.device,
+               shape: tuple | None = None, min_numel: int | None = None):
+    """A caller-supplied buffer the library reads or writes: the C side cannot see its size."""
+    if not isinstance(t, torch.Tensor) or t.device != device or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: {what} must be a contiguous {dtype} tensor on {device}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: {what} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name}: {what} holds {t.numel()} elements, needs at least {min_numel}")
+
+
+def _check_stats(name: str, st: "Stats", dims, device: torch.device):
+    B, H, N, D = dims
+    for what, t in (("stats.m", st.m), ("stats.zfull", st.zfull), ("stats.zkept", st.zkept)):
+        _check_buf(name, what, t, torch.float32, device, shape=(B, H, N))
+    _check_buf(name, "stats.u", st.u, torch.float32, device, shape=(B, H, N, D))
 
 
 def _shape(dims, head_dim: int, block_size: int) -> RtShape:
@@ -154,24 +174,30 @@ def rt_build_block_mask(q: torch.Tensor, k: torch.Tensor, *, head_dim: int, bloc
                         col_idx: torch.Tensor | None = None, block_scores: torch.Tensor | bool | None = None,
                         stream=None):
     """Kept key blocks per query block (CSR).  Returns (row_ptr, col_idx[, block_scores])."""
-    dims = _check_qkv("rt_build_block_mask", q, k)
+    name = "rt_build_block_mask"
+    dims = _check_qkv(name, q, k)
     B, H, N, D = dims
-    nb = -(-N // block_size)
+    nb = -(-N // block_size) if block_size > 0 else 0
     dev = q.device
     if row_ptr is None:
         row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=dev)
     if col_idx is None:
         col_idx = torch.empty(B * H * nb * max(keep_blocks, 0), dtype=torch.int32, device=dev)
+    _check_buf(name, "row_ptr", row_ptr, torch.int32, dev, min_numel=B * H * nb + 1)
+    _check_buf(name, "col_idx", col_idx, torch.int32, dev, min_numel=B * H * nb * max(keep_blocks, 0))
     want_scores = block_scores is True
     if want_scores:
         block_scores = torch.empty(B, H, nb, nb, dtype=torch.float32, device=dev)
     elif block_scores is False:
         block_scores = None
+    if block_scores is not None:
+        _check_buf(name, "block_scores", block_scores, torch.float32, dev, min_numel=B * H * nb * nb)
     shape = _shape(dims, head_dim, block_size)
-    _call(load_library().rt_build_block_mask(ctypes.byref(shape), _ptr(q), _ptr(k), float(scale), int(keep_blocks),
-                                             int(forced_prefix_tokens), _ptr(row_ptr), _ptr(col_idx),
-                                             _ptr(block_scores), _stream_handle(dev, stream)),
-          "rt_build_block_mask")
+    with torch.cuda.device(dev):
+        _call(load_library().rt_build_block_mask(ctypes.byref(shape), _ptr(q), _ptr(k), float(scale),
+                                                 int(keep_blocks), int(forced_prefix_tokens), _ptr(row_ptr),
+                                                 _ptr(col_idx), _ptr(block_scores), _stream_handle(dev, stream)),
+              name)
     return (row_ptr, col_idx, block_scores) if want_scores else (row_ptr, col_idx)
 
 
@@ -179,7 +205,8 @@ def rt_attn_full_capture(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, h
                          scale: float, row_ptr: torch.Tensor, col_idx: torch.Tensor,
                          out: torch.Tensor | None = None, stats: Stats | None = None, stream=None):
     """Full attention at a capture step plus the statistics cache.  Returns (out, stats)."""
-    dims = _check_qkv("rt_attn_full_capture", q, k, v)
+    name = "rt_attn_full_capture"
+    dims = _check_qkv(name, q, k, v)
     B, H, N, D = dims
     dev = q.device
     if out is None:
@@ -189,12 +216,17 @@ def rt_attn_full_capture(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, h
                       torch.empty(B, H, N, dtype=torch.float32, device=dev),
                       torch.empty(B, H, N, dtype=torch.float32, device=dev),
                       torch.empty(B, H, N, D, dtype=torch.float32, device=dev))
+    _check_buf(name, "out", out, torch.bfloat16, dev, shape=dims)
+    _check_stats(name, stats, dims, dev)
+    _check_buf(name, "row_ptr", row_ptr, torch.int32, dev)
+    _check_buf(name, "col_idx", col_idx, torch.int32, dev)
     shape = _shape(dims, head_dim, block_size)
-    _call(load_library().rt_attn_full_capture(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale),
-                                              _ptr(row_ptr), _ptr(col_idx), _ptr(out), _ptr(stats.m),
-                                              _ptr(stats.zfull), _ptr(stats.zkept), _ptr(stats.u),
-                                              _stream_handle(dev, stream)),
-          "rt_attn_full_capture")
+    with torch.cuda.device(dev):
+        _call(load_library().rt_attn_full_capture(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale),
+                                                  _ptr(row_ptr), _ptr(col_idx), _ptr(out), _ptr(stats.m),
+                                                  _ptr(stats.zfull), _ptr(stats.zkept), _ptr(stats.u),
+                                                  _stream_handle(dev, stream)),
+              name)
     return out, stats
 
 
@@ -202,17 +234,24 @@ def rt_attn_sparse_reshape(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
                            scale: float, row_ptr: torch.Tensor, col_idx: torch.Tensor, stats: Stats | None,
                            out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Sparse step over the kept blocks, reshaped with ``stats`` (plain block-sparse if None)."""
-    dims = _check_qkv("rt_attn_sparse_reshape", q, k, v)
+    name = "rt_attn_sparse_reshape"
+    dims = _check_qkv(name, q, k, v)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
+    _check_buf(name, "out", out, torch.bfloat16, dev, shape=dims)
+    if stats is not None:
+        _check_stats(name, stats, dims, dev)
+    _check_buf(name, "row_ptr", row_ptr, torch.int32, dev)
+    _check_buf(name, "col_idx", col_idx, torch.int32, dev)
     shape = _shape(dims, head_dim, block_size)
     s = stats
-    _call(load_library().rt_attn_sparse_reshape(
-        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale), _ptr(row_ptr), _ptr(col_idx),
-        _ptr(s.m if s else None), _ptr(s.zfull if s else None), _ptr(s.zkept if s else None),
-        _ptr(s.u if s else None), _ptr(out), _stream_handle(dev, stream)),
-        "rt_attn_sparse_reshape")
+    with torch.cuda.device(dev):
+        _call(load_library().rt_attn_sparse_reshape(
+            ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale), _ptr(row_ptr), _ptr(col_idx),
+            _ptr(s.m if s else None), _ptr(s.zfull if s else None), _ptr(s.zkept if s else None),
+            _ptr(s.u if s else None), _ptr(out), _stream_handle(dev, stream)),
+            name)
     return out
 
 
@@ -243,20 +282,27 @@ def rt_build_block_mask_static(q: torch.Tensor, k: torch.Tensor, *, head_dim: in
     preallocated ``row_ptr`` / ``col_idx`` to avoid allocations on the Python
     side as well.  Shapes with 2*B*H*n_blocks*D > STATIC_POOL_FLOATS raise.
     """
-    dims = _check_qkv("rt_build_block_mask_static", q, k)
+    name = "rt_build_block_mask_static"
+    dims = _check_qkv(name, q, k)
     B, H, N, D = dims
-    nb = -(-N // block_size)
+    nb = -(-N // block_size) if block_size > 0 else 0
     if 2 * B * H * nb * D > STATIC_POOL_FLOATS:
-        raise ValueError(f"rt_build_block_mask_static: workspace needs {2 * B * H * nb * D} fp32 values, "
+        raise ValueError(f"{name}: workspace needs {2 * B * H * nb * D} fp32 values, "
                          f"the fixed array holds {STATIC_POOL_FLOATS}")
     dev = q.device
     if row_ptr is None:
         row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=dev)
     if col_idx is None:
         col_idx = torch.empty(B * H * nb * max(keep_blocks, 0), dtype=torch.int32, device=dev)
+    _check_buf(name, "row_ptr", row_ptr, torch.int32, dev, min_numel=B * H * nb + 1)
+    _check_buf(name, "col_idx", col_idx, torch.int32, dev, min_numel=B * H * nb * max(keep_blocks, 0))
+    if block_scores is not None:
+        _check_buf(name, "block_scores", block_scores, torch.float32, dev, min_numel=B * H * nb * nb)
     shape = _shape(dims, head_dim, block_size)
-    _call(load_library().rt_build_block_mask_static(ctypes.byref(shape), _ptr(q), _ptr(k), float(scale),
-                                                    int(keep_blocks), int(forced_prefix_tokens), _ptr(row_ptr),
-                                                    _ptr(col_idx), _ptr(block_scores), _stream_handle(dev, stream)),
-          "rt_build_block_mask_static")
+    with torch.cuda.device(dev):
+        _call(load_library().rt_build_block_mask_static(ctypes.byref(shape), _ptr(q), _ptr(k), float(scale),
+                                                        int(keep_blocks), int(forced_prefix_tokens), _ptr(row_ptr),
+                                                        _ptr(col_idx), _ptr(block_scores),
+                                                        _stream_handle(dev, stream)),
+              name)
     return row_ptr, col_idx
