@@ -46,8 +46,12 @@
  * RT_ERR_CUDA.  Kernels never trap: every wait inside a kernel is bounded;
  * when one runs out the kernel records RT_ERR_TIMEOUT in a device status word
  * (read it with rt_take_device_error), leaves its outputs unspecified and
- * returns.  A malformed CSR (indices out of range, unsorted rows) never makes
- * a kernel read or write out of bounds; its results are unspecified.
+ * returns.  The CSR must be readable where row_ptr points: row_ptr holds
+ * B*H*n_blocks + 1 entries and 0 <= row_ptr[r] <= row_ptr[r+1] <= the length
+ * of col_idx (the library cannot see that length).  Beyond that, malformed
+ * contents (block indices out of range, unsorted or repeated entries, rows
+ * longer than n_blocks) never make a kernel read or write out of bounds;
+ * their results are unspecified.
  */
 #ifndef RETTENTION_H
 #define RETTENTION_H
