@@ -467,84 +467,86 @@ def main():
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
                                              device_id=torch.device("cuda", local))
-    try:
-        r = run_ours(args, rank, world, local)
-    finally:
-        pass
+    r = run_ours(args, rank, world, local)
     if rank == 0:
         peaks, peak_src = load_peaks()
-        w, nums = r["w"], r["nums"]
-        sp_s = r["sparse_ms"] / 1e3
-        value = job_throughput(nums["dense_flops"], world, r["sparse_ms"])
-        exec_tflops = nums["executed_flops"] / sp_s / 1e12
-        cap_tflops = nums["dense_flops"] / (r["capture_ms"] / 1e3) / 1e12
-        kernels = {
-            "rt_build_block_mask": {"ms": r["mask_ms"], "bound": "hbm",
-                                    "achieved_gbs": nums["mask_bytes"] / (r["mask_ms"] / 1e3) / 1e9},
-            "rt_attn_full_capture": {"ms": r["capture_ms"], "bound": "tensor", "achieved_tflops": cap_tflops,
-                                     "algorithmic_tflop": nums["dense_flops"] / 1e12,
-                                     "achieved_gbs": nums["capture_bytes"] / (r["capture_ms"] / 1e3) / 1e9},
-            "rt_attn_sparse_reshape": {"ms": r["sparse_ms"], "bound": "tensor+hbm",
-                                       "executed_tflops": exec_tflops,
-                                       "executed_tflop": nums["executed_flops"] / 1e12,
-                                       "dense_equiv_tflops": nums["dense_flops"] / sp_s / 1e12,
-                                       "tensor_frac_of_bf16_peak": exec_tflops / peaks["bf16_tflops"],
-                                       "achieved_gbs": nums["sparse_bytes"] / sp_s / 1e9,
-                                       "hbm_frac": nums["sparse_bytes"] / sp_s / 1e9 / peaks["hbm_gbs"],
-                                       "algorithmic_bytes": nums["sparse_bytes"]},
-        }
-        # dominant kernel of the step (by device time)
-        dom = max(("rt_attn_full_capture", r["capture_ms"]), ("rt_attn_sparse_reshape", r["sparse_ms"]),
-                  ("rt_build_block_mask", r["mask_ms"]), key=lambda t: t[1])[0]
-        wl_tag = f"{w.name}@{r['keep']}"
-        if dom == "rt_attn_full_capture":
-            ach = cap_tflops
-            roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
-                    "traffic": stored_traffic("full_capture_kernel", wl_tag),
-                    "peak_source": f"bf16_tflops ({peak_src}, burst)",
-                    "per_launch": f"{nums['dense_flops'] / 1e12:.3f} TFLOP algorithmic (4*B*H*N^2*d)"}
-        elif dom == "rt_attn_sparse_reshape":
-            ach = exec_tflops
-            roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
-                    "traffic": stored_traffic("sparse_reshape_kernel", wl_tag),
-                    "peak_source": f"bf16_tflops ({peak_src}, burst)"}
-        else:
-            ach = kernels["rt_build_block_mask"]["achieved_gbs"]
-            roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": f"hbm_gbs ({peak_src})"}
-        e2e = None
-        if r["e2e"]:
-            e2e = {"value": job_throughput(nums["dense_flops"], world, r["e2e_ms"]), "unit": UNIT,
-                   "ms_per_step": r["e2e_ms"], "h2d_bytes_per_step": r["e2e"]["h2d_bytes_per_step"],
-                   "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"],
-                   "what": "sparse step through the public API: pinned host Q1/K1/V1 -> device, "
-                           "rt_attn_sparse_reshape, output -> pinned host; steps pipelined on three "
-                           "streams (next step's upload overlaps this step's kernel and read-back)"}
         sweep = None
         if not args.no_sweep and world == 1:
             sweep = run_sweep(args, torch.device("cuda", local))
         cpu = None
-        if not args.no_cpu_baseline and world >= 1:
-            cpu = OracleSample(w, r["keep"], r["host0"], r["host1"], args.cpu_rows).baseline()
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": r["total_ms"] / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": _config(w, r["keep"], r["keep_ratio"], world),
-            "sparse_step_ms": r["sparse_ms"], "full_step_ms": r["mask_ms"] + r["capture_ms"],
-            "dense_equiv_tflops": nums["dense_flops"] / sp_s / 1e12, "executed_tflops": exec_tflops,
-            "tensor_pct_of_bf16_peak": 100.0 * exec_tflops / peaks["bf16_tflops"],
-            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": r["clocks"],
-            "peaks": {**peaks, "source": peak_src},
-            "sweep": sweep,
-        }
-        print(json.dumps(line), flush=True)
+        if not args.no_cpu_baseline and world == 1:
+            cpu = OracleSample(r["w"], r["keep"], r["host0"], r["host1"], args.cpu_rows).baseline()
+        print(json.dumps(build_line(args, r, world, peaks, peak_src, sweep, cpu)), flush=True)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def build_line(args, r: dict, world: int, peaks: dict, peak_src: str, sweep, cpu) -> dict:
+    """The JSON line of our arm from one measurement `r` of run_ours (rank 0)."""
+    w, nums = r["w"], r["nums"]
+    sp_s = r["sparse_ms"] / 1e3
+    value = job_throughput(nums["dense_flops"], world, r["sparse_ms"])
+    exec_tflops = nums["executed_flops"] / sp_s / 1e12
+    cap_tflops = nums["dense_flops"] / (r["capture_ms"] / 1e3) / 1e12
+    kernels = {
+        "rt_build_block_mask": {"ms": r["mask_ms"], "bound": "hbm",
+                                "achieved_gbs": nums["mask_bytes"] / (r["mask_ms"] / 1e3) / 1e9},
+        "rt_attn_full_capture": {"ms": r["capture_ms"], "bound": "tensor", "achieved_tflops": cap_tflops,
+                                 "algorithmic_tflop": nums["dense_flops"] / 1e12,
+                                 "achieved_gbs": nums["capture_bytes"] / (r["capture_ms"] / 1e3) / 1e9},
+        "rt_attn_sparse_reshape": {"ms": r["sparse_ms"], "bound": "tensor+hbm",
+                                   "executed_tflops": exec_tflops,
+                                   "executed_tflop": nums["executed_flops"] / 1e12,
+                                   "dense_equiv_tflops": nums["dense_flops"] / sp_s / 1e12,
+                                   "tensor_frac_of_bf16_peak": exec_tflops / peaks["bf16_tflops"],
+                                   "achieved_gbs": nums["sparse_bytes"] / sp_s / 1e9,
+                                   "hbm_frac": nums["sparse_bytes"] / sp_s / 1e9 / peaks["hbm_gbs"],
+                                   "algorithmic_bytes": nums["sparse_bytes"]},
+    }
+    # dominant kernel of the step (by device time)
+    dom = max(("rt_attn_full_capture", r["capture_ms"]), ("rt_attn_sparse_reshape", r["sparse_ms"]),
+              ("rt_build_block_mask", r["mask_ms"]), key=lambda t: t[1])[0]
+    wl_tag = f"{w.name}@{r['keep']}"
+    if dom == "rt_attn_full_capture":
+        ach = cap_tflops
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                "traffic": stored_traffic("full_capture_kernel", wl_tag),
+                "peak_source": f"bf16_tflops ({peak_src}, burst)",
+                "per_launch": f"{nums['dense_flops'] / 1e12:.3f} TFLOP algorithmic (4*B*H*N^2*d)"}
+    elif dom == "rt_attn_sparse_reshape":
+        ach = exec_tflops
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                "traffic": stored_traffic("sparse_reshape_kernel", wl_tag),
+                "peak_source": f"bf16_tflops ({peak_src}, burst)"}
+    else:
+        ach = kernels["rt_build_block_mask"]["achieved_gbs"]
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": f"hbm_gbs ({peak_src})"}
+    e2e = None
+    if r["e2e"]:
+        e2e = {"value": job_throughput(nums["dense_flops"], world, r["e2e_ms"]), "unit": UNIT,
+               "ms_per_step": r["e2e_ms"], "h2d_bytes_per_step": r["e2e"]["h2d_bytes_per_step"],
+               "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"],
+               "what": "sparse step through the public API: pinned host Q1/K1/V1 -> device, "
+                       "rt_attn_sparse_reshape, output -> pinned host; steps pipelined on three "
+                       "streams (next step's upload overlaps this step's kernel and read-back)"}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["total_ms"] / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config(w, r["keep"], r["keep_ratio"], world),
+        "sparse_step_ms": r["sparse_ms"], "full_step_ms": r["mask_ms"] + r["capture_ms"],
+        "dense_equiv_tflops": nums["dense_flops"] / sp_s / 1e12, "executed_tflops": exec_tflops,
+        "tensor_pct_of_bf16_peak": 100.0 * exec_tflops / peaks["bf16_tflops"],
+        "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": r["clocks"],
+        "peaks": {**peaks, "source": peak_src},
+        "sweep": sweep,
+    }
+    return line
 
 
 if __name__ == "__main__":
