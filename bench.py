@@ -39,8 +39,8 @@ from ultra_sparse_attention_b200.workloads import WORKLOADS, denoising_inputs  #
 METRIC = "sparse-step ms & dense-equiv TFLOP/s; tensor-pipe % of BF16 peak (1xB200)"
 UNIT = "TFLOP/s (dense-equivalent, sparse step)"
 # Kernels the library launches per step: block pooling + score/select (mask),
-# the capture kernel, the sparse kernel.
-LAUNCHES_PER_STEP = 4
+# the tile pairing, the capture kernel, the sparse kernel.
+LAUNCHES_PER_STEP = 5
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -173,6 +173,29 @@ def kept_work(row_ptr: np.ndarray, col_idx: np.ndarray, N: int, bs: int, bh: int
     return total
 
 
+def key_tiles_per_query_tile(row_ptr: np.ndarray, col_idx: np.ndarray, tiles: np.ndarray | None, nb: int, bs: int,
+                             bh: int, N: int) -> float:
+    """Mean key-tile steps of the sparse kernel per 128-row query tile: the union of the
+    kept blocks of the tile's query blocks (neighbouring blocks when `tiles` is None)."""
+    n_tiles = -(-N // 128)
+    if tiles is None:
+        per = 128 // bs
+        tiles = np.full((bh, n_tiles, 2), -1, np.int64)
+        for t in range(n_tiles):
+            for h in range(per):
+                if t * per + h < nb:
+                    tiles[:, t, h] = t * per + h
+    total = 0
+    for b in range(bh):
+        for t in range(n_tiles):
+            u = set()
+            for qb in tiles[b, t]:
+                if 0 <= qb < nb:
+                    u.update(col_idx[row_ptr[b * nb + qb]:row_ptr[b * nb + qb + 1]].tolist())
+            total += len(u) * (bs // 64)
+    return total / (bh * n_tiles)
+
+
 def workload_numbers(w, keep: int, row_ptr, col_idx):
     B, H, N, d, D = w.batch, w.heads, w.seq_len, w.head_dim, w.head_dim_padded
     bh = B * H
@@ -209,8 +232,9 @@ def run_ours(args, rank, world, local):
     out0, out1 = torch.empty_like(q0), torch.empty_like(q1)
     stats = usa.Stats(torch.empty(B, H, N, device=device), torch.empty(B, H, N, device=device),
                       torch.empty(B, H, N, device=device), torch.empty(B, H, N, D, device=device))
+    tiles = torch.empty(B * H, -(-N // 128), 2, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream(device)
-    ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(2)] for k in ("mask", "capture", "sparse")}
+    ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(2)] for k in ("mask", "pair", "capture", "sparse")}
     times = {k: [] for k in ev}
 
     def step(record: bool):
@@ -221,11 +245,15 @@ def run_ours(args, rank, world, local):
         usa.rt_build_block_mask(q0, k0, keep_blocks=keep, forced_prefix_tokens=w.forced_prefix_tokens,
                                 row_ptr=row_ptr, col_idx=col_idx, **kw)
         mark("mask", 1)
+        mark("pair", 0)
+        usa.rt_pair_query_blocks(q0, row_ptr, col_idx, head_dim=w.head_dim, block_size=w.block_size, tile_blocks=tiles)
+        mark("pair", 1)
         mark("capture", 0)
         usa.rt_attn_full_capture(q0, k0, v0, row_ptr=row_ptr, col_idx=col_idx, out=out0, stats=stats, **kw)
         mark("capture", 1)
         mark("sparse", 0)
-        usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=row_ptr, col_idx=col_idx, stats=stats, out=out1, **kw)
+        usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=row_ptr, col_idx=col_idx, stats=stats, tile_blocks=tiles,
+                                   out=out1, **kw)
         mark("sparse", 1)
 
     def barrier():
@@ -262,6 +290,8 @@ def run_ours(args, rank, world, local):
 
     rp, ci = row_ptr.cpu().numpy(), col_idx.cpu().numpy()
     nums = workload_numbers(w, keep, rp, ci)
+    nums["key_tiles_per_query_tile"] = key_tiles_per_query_tile(rp, ci, tiles.cpu().numpy(), nb, w.block_size, B * H, N)
+    nums["key_tiles_per_query_tile_neighbours"] = key_tiles_per_query_tile(rp, ci, None, nb, w.block_size, B * H, N)
 
     # e2e: the sparse step through the public API with host buffers (pinned), copies inside the
     # timed region.  Steps are pipelined as a server would run them: step k+1's host-to-device
@@ -296,7 +326,8 @@ def run_ours(args, rank, world, local):
             stream.wait_event(ev_in[b])
             if it >= 2:
                 stream.wait_event(ev_out[b])
-            usa.rt_attn_sparse_reshape(*d_in[b], row_ptr=row_ptr, col_idx=col_idx, stats=stats, out=d_out[b], **kw)
+            usa.rt_attn_sparse_reshape(*d_in[b], row_ptr=row_ptr, col_idx=col_idx, stats=stats, tile_blocks=tiles,
+                                       out=d_out[b], **kw)
             ev_used[b].record(stream)
             with torch.cuda.stream(s_d2h):
                 s_d2h.wait_event(ev_used[b])
@@ -313,11 +344,11 @@ def run_ours(args, rank, world, local):
                "d2h_bytes_per_step": int(h_out[0].numel() * h_out[0].element_size())}
         del d_in, d_out
 
-    total_ms, mask_ms, cap_ms, sp_ms, e2e_ms = max_over_ranks(
-        [total_ms, per_kernel["mask"], per_kernel["capture"], per_kernel["sparse"],
+    total_ms, mask_ms, pair_ms, cap_ms, sp_ms, e2e_ms = max_over_ranks(
+        [total_ms, per_kernel["mask"], per_kernel["pair"], per_kernel["capture"], per_kernel["sparse"],
          e2e["ms_per_step"] if e2e else 0.0], device, world)
     return {"w": w, "keep": keep, "keep_ratio": keep_ratio, "total_ms": total_ms, "mask_ms": mask_ms,
-            "capture_ms": cap_ms, "sparse_ms": sp_ms, "e2e": e2e, "e2e_ms": e2e_ms, "clocks": clk, "nums": nums,
+            "pair_ms": pair_ms, "capture_ms": cap_ms, "sparse_ms": sp_ms, "e2e": e2e, "e2e_ms": e2e_ms, "clocks": clk, "nums": nums,
             "host1": host1, "host0": host0}
 
 
@@ -341,26 +372,27 @@ def run_sweep(args, device) -> list:
         q0, k0, v0 = (x.to(device) for x in next(steps)[1:])
         q1, k1, v1 = (x.to(device) for x in next(steps)[1:])
         kw = dict(head_dim=w.head_dim, block_size=w.block_size, scale=w.scale)
-        times = {"mask": [], "capture": [], "sparse": []}
-        rp = ci = None
+        times = {"mask": [], "pair": [], "capture": [], "sparse": []}
+        rp = ci = tb = None
         for it in range(args.sweep_warmup + args.sweep_steps):
             flush.zero_()
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
             ev[0].record(stream)
             rp, ci = usa.rt_build_block_mask(q0, k0, keep_blocks=keep, forced_prefix_tokens=w.forced_prefix_tokens, **kw)
             ev[1].record(stream)
-            _, st = usa.rt_attn_full_capture(q0, k0, v0, row_ptr=rp, col_idx=ci, **kw)
+            tb = usa.rt_pair_query_blocks(q0, rp, ci, head_dim=w.head_dim, block_size=w.block_size)
             ev[2].record(stream)
-            usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rp, col_idx=ci, stats=st, **kw)
+            _, st = usa.rt_attn_full_capture(q0, k0, v0, row_ptr=rp, col_idx=ci, **kw)
             ev[3].record(stream)
+            usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rp, col_idx=ci, stats=st, tile_blocks=tb, **kw)
+            ev[4].record(stream)
             if it >= args.sweep_warmup:
-                times["mask"].append((ev[0], ev[1]))
-                times["capture"].append((ev[1], ev[2]))
-                times["sparse"].append((ev[2], ev[3]))
+                for i, k in enumerate(("mask", "pair", "capture", "sparse")):
+                    times[k].append((ev[i], ev[i + 1]))
         # How close the reshaped sparse step comes to full attention of its own inputs (the
         # capture kernel's output on them), against plain block-sparse attention.
         full1, _ = usa.rt_attn_full_capture(q1, k1, v1, row_ptr=rp, col_idx=ci, **kw)
-        resh1 = usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rp, col_idx=ci, stats=st, **kw)
+        resh1 = usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rp, col_idx=ci, stats=st, tile_blocks=tb, **kw)
         plain1 = usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rp, col_idx=ci, stats=None, **kw)
         torch.cuda.synchronize()
         if usa.rt_take_device_error() != 0:
@@ -377,13 +409,14 @@ def run_sweep(args, device) -> list:
         out.append({"workload": name, "shape": f"B={w.batch} H={w.heads} N={w.seq_len} d={w.head_dim} D={w.head_dim_padded} "
                                                f"block={w.block_size}",
                     "keep": f"{keep}/{w.n_blocks} ({ratio})", "sparse_step_ms": ms["sparse"],
-                    "full_step_ms": ms["mask"] + ms["capture"], "mask_ms": ms["mask"], "capture_ms": ms["capture"],
+                    "full_step_ms": ms["mask"] + ms["pair"] + ms["capture"], "mask_ms": ms["mask"],
+                    "pair_ms": ms["pair"], "capture_ms": ms["capture"],
                     "dense_equiv_tflops": nums["dense_flops"] / sp_s / 1e12, "executed_tflops": exe,
                     "sparse_tensor_frac_of_bf16_peak": exe / peaks["bf16_tflops"],
                     "capture_tflops": cap, "capture_frac_of_bf16_peak": cap / peaks["bf16_tflops"],
                     "reshape_rel_l2_vs_full": err_r, "plain_sparse_rel_l2_vs_full": err_p,
                     "steps": args.sweep_steps, "warmup": args.sweep_warmup, "l2": "flushed between cycles"})
-        del q0, k0, v0, q1, k1, v1, st, rp, ci
+        del q0, k0, v0, q1, k1, v1, st, rp, ci, tb
     return out
 
 
@@ -449,7 +482,7 @@ def run_reference(args, rank, world):
 def _config(w, keep, keep_ratio, gpus):
     return {"workload": (f"{w.name}: B={w.batch} H={w.heads} N={w.seq_len} d={w.head_dim} D={w.head_dim_padded} "
                          f"block={w.block_size} keep={keep}/{w.n_blocks} ({keep_ratio})"),
-            "step": "mask + full capture at t0, sparse reshape at t1 (drifted inputs)",
+            "step": "mask + tile pairing + full capture at t0, sparse reshape at t1 (drifted inputs)",
             "forced_prefix_tokens": w.forced_prefix_tokens,
             "l2": "inputs larger than L2 (about 1.1 GB touched per step; no flush)",
             "parallelism": f"replicas x{gpus}"}
@@ -492,6 +525,7 @@ def build_line(args, r: dict, world: int, peaks: dict, peak_src: str, sweep, cpu
     kernels = {
         "rt_build_block_mask": {"ms": r["mask_ms"], "bound": "hbm",
                                 "achieved_gbs": nums["mask_bytes"] / (r["mask_ms"] / 1e3) / 1e9},
+        "rt_pair_query_blocks": {"ms": r["pair_ms"], "bound": "latency (one CTA per head, once per mask)"},
         "rt_attn_full_capture": {"ms": r["capture_ms"], "bound": "tensor", "achieved_tflops": cap_tflops,
                                  "algorithmic_tflop": nums["dense_flops"] / 1e12,
                                  "achieved_gbs": nums["capture_bytes"] / (r["capture_ms"] / 1e3) / 1e9},
@@ -502,7 +536,9 @@ def build_line(args, r: dict, world: int, peaks: dict, peak_src: str, sweep, cpu
                                    "tensor_frac_of_bf16_peak": exec_tflops / peaks["bf16_tflops"],
                                    "achieved_gbs": nums["sparse_bytes"] / sp_s / 1e9,
                                    "hbm_frac": nums["sparse_bytes"] / sp_s / 1e9 / peaks["hbm_gbs"],
-                                   "algorithmic_bytes": nums["sparse_bytes"]},
+                                   "algorithmic_bytes": nums["sparse_bytes"],
+                                   "key_tiles_per_query_tile": nums.get("key_tiles_per_query_tile"),
+                                   "key_tiles_per_query_tile_neighbours": nums.get("key_tiles_per_query_tile_neighbours")},
     }
     # dominant kernel of the step (by device time)
     dom = max(("rt_attn_full_capture", r["capture_ms"]), ("rt_attn_sparse_reshape", r["sparse_ms"]),
@@ -538,7 +574,7 @@ def build_line(args, r: dict, world: int, peaks: dict, peak_src: str, sweep, cpu
         "warmup": args.warmup, "ms_per_step": r["total_ms"] / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": _config(w, r["keep"], r["keep_ratio"], world),
-        "sparse_step_ms": r["sparse_ms"], "full_step_ms": r["mask_ms"] + r["capture_ms"],
+        "sparse_step_ms": r["sparse_ms"], "full_step_ms": r["mask_ms"] + r["pair_ms"] + r["capture_ms"],
         "dense_equiv_tflops": nums["dense_flops"] / sp_s / 1e12, "executed_tflops": exec_tflops,
         "tensor_pct_of_bf16_peak": 100.0 * exec_tflops / peaks["bf16_tflops"],
         "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,

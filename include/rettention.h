@@ -12,6 +12,10 @@
  *   rt_build_block_mask     which key blocks each query block keeps;
  *   rt_attn_full_capture    full attention at a capture step, plus the cache;
  *   rt_attn_sparse_reshape  block-sparse attention reshaped with the cache.
+ * A fourth, rt_pair_query_blocks, only schedules: it groups query blocks
+ * into the sparse kernel's 128-row tiles so that a tile's blocks keep mostly
+ * the same key blocks, which makes the sparse step faster without changing
+ * its result.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -62,7 +66,7 @@
 extern "C" {
 #endif
 
-#define RT_ABI_VERSION 1
+#define RT_ABI_VERSION 2
 
 typedef enum rt_status {
     RT_OK = 0,
@@ -163,14 +167,58 @@ rt_status rt_attn_full_capture(const rt_shape *shape, const void *q, const void 
  *
  * q, k, v       bf16 [B,H,N,D] device (the current step's inputs).
  * row_ptr, col_idx  the CSR used at the capture step.
+ * tile_blocks   optional (may be NULL), int32 [B*H][n_tiles][2] device,
+ *               n_tiles = ceil(N / 128): which query blocks the kernel computes
+ *               together in each 128-row tile, as written by
+ *               rt_pair_query_blocks (block size 64: two blocks per tile;
+ *               block size 128: one, the second entry unused).  NULL means
+ *               the neighbouring blocks (tile t = blocks 2t, 2t+1 at block
+ *               size 64).  Every row's result is the same for any table in
+ *               which each query block of a head appears exactly once (-1 or
+ *               an out-of-range entry is an empty half); a block that appears
+ *               in no tile leaves its output rows unwritten, one that appears
+ *               twice is computed twice.
  * stat_*        fp32 statistics written by rt_attn_full_capture, or all NULL.
  * out           out, bf16 [B,H,N,D] device.
 */
 rt_status rt_attn_sparse_reshape(const rt_shape *shape, const void *q, const void *k,
                                  const void *v, float scale, const int32_t *row_ptr,
-                                 const int32_t *col_idx, const float *stat_m,
-                                 const float *stat_zfull, const float *stat_zkept,
-                                 const float *stat_u, void *out, rt_stream_t stream);
+                                 const int32_t *col_idx, const int32_t *tile_blocks,
+                                 const float *stat_m, const float *stat_zfull,
+                                 const float *stat_zkept, const float *stat_u, void *out,
+                                 rt_stream_t stream);
+
+/*
+ * rt_pair_query_blocks -- group the query blocks of each head into the
+ * sparse kernel's 128-row tiles.
+ *
+ * Not part of the method (the pages describe no kernel): a schedule for
+ * rt_attn_sparse_reshape.  A 128-row tile is computed against the union of
+ * its query blocks' kept key blocks, so at block size 64 a key block kept by
+ * only one of the two costs the other a wasted step.  This call pairs blocks
+ * that keep many of the same key blocks, deterministically:
+ *   1. for each query block i, its 8 best partners j with |i - j| <= 224 in
+ *      the order (overlap desc, |i - j| asc, j asc), where overlap is the
+ *      number of key blocks both rows keep (entries outside [0, n_blocks)
+ *      ignored, a row cut to its first n_blocks entries);
+ *   2. 8 rounds in which every unpaired block picks its first unpaired
+ *      candidate and two blocks that pick each other become a pair;
+ *   3. tiles: the pairs in order of their lower block, then the unpaired
+ *      blocks two by two in ascending order (-1 for an odd last half).
+ * At block size 128 a tile is one block: tile t = (t, -1).  Compute it once
+ * per mask (at the capture step) and pass it to every sparse step that uses
+ * that mask.
+ *
+ * row_ptr, col_idx  the CSR (as for rt_attn_sparse_reshape).
+ * tile_blocks   out, int32 [B*H][ceil(N / 128)][2] device.
+ * Malformed CSR contents give a valid table of unspecified quality.  At block
+ * size 64 takes a transient device workspace of B*H*n_blocks*16 bytes (the
+ * candidates of step 1) from the library's stream-ordered pool, as
+ * rt_build_block_mask does.
+ */
+rt_status rt_pair_query_blocks(const rt_shape *shape, const int32_t *row_ptr,
+                               const int32_t *col_idx, int32_t *tile_blocks,
+                               rt_stream_t stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *rt_status_string(rt_status status);

@@ -18,9 +18,10 @@ def _declared_functions():
     return sorted(set(re.findall(r"\b(rt_[a-z_]+)\s*\(", text)))
 
 
-def test_header_declares_the_three_calls():
+def test_header_declares_the_path_calls():
     names = _declared_functions()
-    for n in ("rt_build_block_mask", "rt_attn_full_capture", "rt_attn_sparse_reshape", "rt_status_string"):
+    for n in ("rt_build_block_mask", "rt_attn_full_capture", "rt_attn_sparse_reshape", "rt_pair_query_blocks",
+              "rt_status_string"):
         assert n in names
 
 
@@ -31,7 +32,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    assert usa.rt_abi_version() == 1
+    assert usa.rt_abi_version() == 2
     for code in range(5):
         s = usa.rt_status_string(code)
         assert s.startswith("RT_")
@@ -49,8 +50,12 @@ def _mask(lib, shape, q=A16, k=A16, scale=0.125, keep=2, forced=0, rp=A16, ci=A1
                                    rp, ci, sc, None)
 
 
-def _sparse(lib, shape, stats=(None, None, None, None), out=A16, scale=0.125):
-    return lib.rt_attn_sparse_reshape(ctypes.byref(shape), A16, A16, A16, scale, A16, A16, *stats, out, None)
+def _sparse(lib, shape, stats=(None, None, None, None), out=A16, scale=0.125, tiles=None):
+    return lib.rt_attn_sparse_reshape(ctypes.byref(shape), A16, A16, A16, scale, A16, A16, tiles, *stats, out, None)
+
+
+def _pair(lib, shape, rp=A16, ci=A16, tiles=A16):
+    return lib.rt_pair_query_blocks(ctypes.byref(shape) if shape is not None else None, rp, ci, tiles, None)
 
 
 def _capture(lib, shape, u=A16, m=A16):
@@ -86,10 +91,23 @@ def test_attention_argument_validation():
     assert _sparse(lib, ok, out=None) == usa.RT_ERR_INVALID_ARGUMENT
     assert _sparse(lib, ok, scale=-1.0) == usa.RT_ERR_INVALID_ARGUMENT
     assert _sparse(lib, RtShape(2, 3, 1000, 72, 72, 64)) == usa.RT_ERR_UNSUPPORTED
+    assert _sparse(lib, ok, tiles=MIS) == usa.RT_ERR_INVALID_ARGUMENT                     # table misaligned
     assert _capture(lib, ok, u=None) == usa.RT_ERR_INVALID_ARGUMENT
     assert _capture(lib, ok, u=A4) == usa.RT_ERR_INVALID_ARGUMENT
     assert _capture(lib, ok, m=MIS) == usa.RT_ERR_INVALID_ARGUMENT
     assert _capture(lib, RtShape(2, 3, 1000, 72, 80, 256)) == usa.RT_ERR_UNSUPPORTED
+
+
+def test_pairing_argument_validation():
+    lib = usa.load_library()
+    ok = RtShape(1, 2, 512, 64, 64, 64)
+    assert _pair(lib, None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _pair(lib, ok, rp=None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _pair(lib, ok, ci=None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _pair(lib, ok, tiles=None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _pair(lib, ok, tiles=MIS) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _pair(lib, RtShape(1, 2, 512, 64, 64, 32)) == usa.RT_ERR_UNSUPPORTED
+    assert _pair(lib, RtShape(1, 1, 64 * 4097, 64, 64, 64)) == usa.RT_ERR_UNSUPPORTED
 
 
 def test_python_binding_rejects_cpu_tensors():

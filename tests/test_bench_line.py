@@ -29,7 +29,7 @@ def _measurement(world, with_e2e=True):
     nums = bench.workload_numbers(w, keep, row_ptr, col_idx)
     e2e = {"h2d_bytes_per_step": 3 * bh * w.seq_len * w.head_dim_padded * 2,
            "d2h_bytes_per_step": bh * w.seq_len * w.head_dim_padded * 2} if with_e2e else None
-    return {"w": w, "keep": keep, "keep_ratio": w.keep[0], "total_ms": 10.0, "mask_ms": 0.05,
+    return {"w": w, "keep": keep, "keep_ratio": w.keep[0], "total_ms": 10.0, "mask_ms": 0.05, "pair_ms": 0.01,
             "capture_ms": 1.5, "sparse_ms": 0.25, "e2e": e2e, "e2e_ms": 0.4,
             "clocks": {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 12},
             "nums": nums}
@@ -76,9 +76,26 @@ def test_our_line_has_the_contract_keys(world):
         assert line["cpu_baseline"] is None
 
 
+def line_full_step(r):
+    return bench.build_line(_Args, r, 1, dict(bench.FALLBACK_PEAKS), "fallback", None, None)["full_step_ms"]
+
+
+def test_key_tiles_per_query_tile_counts_the_union():
+    # 2 heads x 4 query blocks (block 64, N = 256): head 0 rows {0,1},{0,2},{0,1},{0,2}; head 1 all {3}
+    rp = np.arange(9, dtype=np.int64) * 2
+    ci = np.array([0, 1, 0, 2, 0, 1, 0, 2] + [3, 3] * 4)
+    ci[9::2] = 3
+    # neighbours: head 0 tiles {0,1,2} {0,1,2} -> 3, 3; head 1 {3} -> 1, 1
+    assert bench.key_tiles_per_query_tile(rp, ci, None, 4, 64, 2, 256) == pytest.approx((3 + 3 + 1 + 1) / 4)
+    tiles = np.array([[[0, 2], [1, 3]], [[0, 1], [2, 3]]])
+    # paired: head 0 {0,1} {0,2} -> 2, 2
+    assert bench.key_tiles_per_query_tile(rp, ci, tiles, 4, 64, 2, 256) == pytest.approx((2 + 2 + 1 + 1) / 4)
+
+
 def test_roofline_follows_the_dominant_kernel():
     r = _measurement(1)
     r["capture_ms"], r["sparse_ms"] = 0.1, 0.5
+    assert line_full_step(r) == pytest.approx(0.05 + 0.01 + 0.1)
     line = bench.build_line(_Args, r, 1, dict(bench.FALLBACK_PEAKS), "fallback", None, None)
     roof = line["roofline"]
     assert roof["kernel"] == "rt_attn_sparse_reshape"

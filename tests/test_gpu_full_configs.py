@@ -22,6 +22,7 @@ import oracle
 import ultra_sparse_attention_b200 as usa
 from ultra_sparse_attention_b200.workloads import WORKLOADS, denoising_inputs
 
+from pairing_ref import check_table, pair_query_blocks
 from parity import check_mask, compare_out, compare_stats, sample_rows, score_tol
 
 pytestmark = pytest.mark.gpu
@@ -94,6 +95,19 @@ def test_full_size_cycle_matches_oracle(cuda_device, name, keep):
     got = out1.reshape(-1, D)[torch.as_tensor(rows, device=cuda_device)]
     want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp_h, ci_h, orc, rows=rows)
     compare_out(got, want, d, f"{name} sparse O")
+
+    # the same step with the query blocks paired by kept-set overlap (as the benchmark runs
+    # it): a valid table, equal to the tests' restatement on the first heads, same bits
+    tiles = usa.rt_pair_query_blocks(d1[0], rp, ci, head_dim=d, block_size=bs)
+    out1p = usa.rt_attn_sparse_reshape(*d1, row_ptr=rp, col_idx=ci, stats=st, tile_blocks=tiles, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    tiles_h = tiles.cpu().numpy()
+    check_table(tiles_h, nb, bs)
+    if nb <= 600:
+        nh = min(2, bh)
+        np.testing.assert_array_equal(tiles_h[:nh], pair_query_blocks(rp_h, ci_h, nh, nb, bs, tiles_h.shape[1]))
+    assert torch.equal(out1p.view(torch.int16), out1.view(torch.int16))
     full = oracle.full_capture(*h1, d, bs, w.scale, rp_h, ci_h, rows=rows)["o"]
     if keep == nb:
         compare_out(got, full, d, f"{name} keep-all sparse step vs full attention")

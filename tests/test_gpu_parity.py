@@ -13,6 +13,7 @@ import oracle
 import ultra_sparse_attention_b200 as usa
 from ultra_sparse_attention_b200.workloads import Workload, denoising_inputs
 
+from pairing_ref import check_table, pair_query_blocks
 from parity import (check_mask, compare_out, compare_stats, random_csr, score_tol, to_dev)
 
 pytestmark = pytest.mark.gpu
@@ -154,6 +155,85 @@ def test_sparse_matches_oracle(cuda_device, N, d, D, bs, keep_frac, with_stats):
     assert usa.rt_take_device_error() == 0
     want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp, ci, st_o)
     compare_out(out.reshape(-1, D), want, d, "sparse O")
+
+
+# ------------------------------------------------------------------ tile pairing
+def _random_table(bh, nb, bs, N, seed):
+    """Each head's blocks in random tiles and halves (an odd count leaves a random empty half)."""
+    rng = np.random.default_rng(seed)
+    n_tiles = -(-N // 128)
+    per = 2 if bs == 64 else 1
+    t = np.full((bh, n_tiles, 2), -1, np.int32)
+    for h in range(bh):
+        slots = np.full(n_tiles * per, -1, np.int64)
+        slots[:nb] = rng.permutation(nb)
+        slots = rng.permutation(slots) if per == 2 else slots
+        t[h, :, :per] = slots.reshape(n_tiles, per)
+    return t
+
+
+@pytest.mark.parametrize("N,bs,keep", [(1000, 64, 4), (200, 64, 2), (64 * 301, 64, 9), (1000, 128, 3), (64, 64, 1),
+                                        (1000, 64, 16), (64 * 2048, 64, 20), (64 * 900 - 5, 64, 30)])
+def test_pairing_matches_reference(cuda_device, N, bs, keep):
+    bh, nb = 3, -(-N // bs)
+    rp, ci = random_csr(bh, nb, keep, seed=N + keep, forced=1)
+    q = torch.zeros(1, bh, N, 64, dtype=torch.bfloat16, device=cuda_device)
+    got = usa.rt_pair_query_blocks(q, to_dev(rp, cuda_device), to_dev(ci, cuda_device), head_dim=64, block_size=bs)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    got = got.cpu().numpy()
+    check_table(got, nb, bs)
+    np.testing.assert_array_equal(got, pair_query_blocks(rp, ci, bh, nb, bs, -(-N // 128)))
+
+
+def test_pairing_of_a_malformed_csr_is_valid_and_matches(cuda_device):
+    """Out-of-range entries, repeats, empty rows and rows longer than n_blocks: the
+    table is still a valid one and the same as the reference's."""
+    N, bs, bh = 1000, 64, 2
+    nb = -(-N // bs)
+    rng = np.random.default_rng(3)
+    rows = []
+    for r in range(bh * nb):
+        n = int(rng.choice([0, 1, 3, nb + 5]))
+        rows.append(rng.integers(-3, nb + 3, size=n))
+    rp = np.array([0] + list(np.cumsum([len(x) for x in rows])), np.int32)
+    ci = np.concatenate(rows).astype(np.int32)
+    q = torch.zeros(1, bh, N, 64, dtype=torch.bfloat16, device=cuda_device)
+    got = usa.rt_pair_query_blocks(q, to_dev(rp, cuda_device), to_dev(ci, cuda_device), head_dim=64, block_size=bs)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    got = got.cpu().numpy()
+    check_table(got, nb, bs)
+    np.testing.assert_array_equal(got, pair_query_blocks(rp, ci, bh, nb, bs, -(-N // 128)))
+
+
+@pytest.mark.parametrize("N,d,D,bs", CASES + [(1064, 64, 64, 64), (1064, 72, 80, 64)])  # 17 blocks: an empty half
+def test_sparse_with_any_tile_table_is_bit_identical(cuda_device, N, d, D, bs):
+    """The pairing only regroups rows: the sparse step with the computed pairing, with a
+    random table (blocks in any tile and half, empty halves anywhere) and with the
+    neighbouring blocks gives the same bits, with and without statistics, and matches
+    the oracle."""
+    w = _wl(N, d, D, bs, std=1.2, seed=13 * N + d, drift=0.05)
+    (h0, h1), (d0, d1) = _inputs(w, cuda_device)
+    bh, nb = w.batch * w.heads, w.n_blocks
+    keep = w.keep_blocks(Fraction(1, 4))
+    rp, ci = random_csr(bh, nb, keep, seed=N + 3, forced=1)
+    rp_d, ci_d = to_dev(rp, cuda_device), to_dev(ci, cuda_device)
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale, row_ptr=rp_d, col_idx=ci_d)
+    _, st = usa.rt_attn_full_capture(*d0, **kw)
+    paired = usa.rt_pair_query_blocks(d1[0], rp_d, ci_d, head_dim=d, block_size=bs)
+    rand = to_dev(_random_table(bh, nb, bs, N, seed=N), cuda_device)
+    for stats in (st, None):
+        base = usa.rt_attn_sparse_reshape(*d1, stats=stats, **kw)
+        for table in (paired, rand):
+            out = torch.full_like(base, float("nan"))
+            usa.rt_attn_sparse_reshape(*d1, stats=stats, tile_blocks=table, out=out, **kw)
+            torch.cuda.synchronize()
+            assert usa.rt_take_device_error() == 0
+            assert torch.equal(out.view(torch.int16), base.view(torch.int16))
+    check_table(paired.cpu().numpy(), nb, bs)
+    want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp, ci, None)
+    compare_out(out.reshape(-1, D), want, d, "sparse O (random tile table, no statistics)")
 
 
 @pytest.mark.parametrize("N,d,D,bs", [(1000, 64, 64, 64), (1000, 72, 80, 64), (200, 64, 64, 64), (896, 64, 64, 128),

@@ -11,6 +11,7 @@ The functions carry the C ABI's names (see include/rettention.h):
     rt_build_block_mask(q, k, ...)      -> (row_ptr, col_idx)
     rt_attn_full_capture(q, k, v, ...)  -> (out, stats)
     rt_attn_sparse_reshape(q, k, v, ...) -> out
+    rt_pair_query_blocks(q, row_ptr, col_idx, ...) -> tile_blocks  (schedule for the sparse step)
 """
 from __future__ import annotations
 
@@ -30,6 +31,7 @@ __all__ = [
     "rt_build_block_mask",
     "rt_attn_full_capture",
     "rt_attn_sparse_reshape",
+    "rt_pair_query_blocks",
     "rt_status_string",
     "rt_abi_version",
     "rt_take_device_error",
@@ -81,7 +83,8 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
             shp = ctypes.POINTER(RtShape)
             lib.rt_build_block_mask.argtypes = [shp, vp, vp, f32, i32, i32, vp, vp, vp, vp]
             lib.rt_attn_full_capture.argtypes = [shp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp]
-            lib.rt_attn_sparse_reshape.argtypes = [shp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp]
+            lib.rt_attn_sparse_reshape.argtypes = [shp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            lib.rt_pair_query_blocks.argtypes = [shp, vp, vp, vp, vp]
             lib.rt_status_string.argtypes = [ctypes.c_int]
             lib.rt_status_string.restype = ctypes.c_char_p
             lib.rt_abi_version.argtypes = []
@@ -91,7 +94,7 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.rt_build_block_mask_static.argtypes = [shp, vp, vp, f32, i32, i32, vp, vp, vp, vp]
             lib.rt_build_block_mask_static.restype = ctypes.c_int
             for fn in ("rt_build_block_mask", "rt_attn_full_capture", "rt_attn_sparse_reshape",
-                       "rt_take_device_error", "rt_selftest_wait_timeout"):
+                       "rt_pair_query_blocks", "rt_take_device_error", "rt_selftest_wait_timeout"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -232,11 +235,17 @@ def rt_attn_full_capture(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, h
 
 def rt_attn_sparse_reshape(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, head_dim: int, block_size: int,
                            scale: float, row_ptr: torch.Tensor, col_idx: torch.Tensor, stats: Stats | None,
-                           out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Sparse step over the kept blocks, reshaped with ``stats`` (plain block-sparse if None)."""
+                           tile_blocks: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                           stream=None) -> torch.Tensor:
+    """Sparse step over the kept blocks, reshaped with ``stats`` (plain block-sparse if None).
+
+    ``tile_blocks`` (from rt_pair_query_blocks) groups the query blocks into the
+    kernel's 128-row tiles; None takes neighbouring blocks.  The result is the same."""
     name = "rt_attn_sparse_reshape"
     dims = _check_qkv(name, q, k, v)
     dev = q.device
+    if tile_blocks is not None:
+        _check_buf(name, "tile_blocks", tile_blocks, torch.int32, dev, shape=_tile_table_shape(dims))
     if out is None:
         out = torch.empty_like(q)
     _check_buf(name, "out", out, torch.bfloat16, dev, shape=dims)
@@ -249,10 +258,36 @@ def rt_attn_sparse_reshape(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
     with torch.cuda.device(dev):
         _call(load_library().rt_attn_sparse_reshape(
             ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale), _ptr(row_ptr), _ptr(col_idx),
-            _ptr(s.m if s else None), _ptr(s.zfull if s else None), _ptr(s.zkept if s else None),
+            _ptr(tile_blocks), _ptr(s.m if s else None), _ptr(s.zfull if s else None), _ptr(s.zkept if s else None),
             _ptr(s.u if s else None), _ptr(out), _stream_handle(dev, stream)),
             name)
     return out
+
+
+def _tile_table_shape(dims) -> tuple[int, int, int]:
+    B, H, N, _ = dims
+    return (B * H, -(-N // 128), 2)
+
+
+def rt_pair_query_blocks(q: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor, *, head_dim: int,
+                         block_size: int, tile_blocks: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Group each head's query blocks into the sparse kernel's 128-row tiles (``q`` gives the shape).
+
+    Returns int32 [B*H, ceil(N/128), 2]: the query blocks of each tile, -1 for an empty half."""
+    name = "rt_pair_query_blocks"
+    dims = _check_qkv(name, q)
+    dev = q.device
+    if tile_blocks is None:
+        tile_blocks = torch.empty(_tile_table_shape(dims), dtype=torch.int32, device=dev)
+    _check_buf(name, "tile_blocks", tile_blocks, torch.int32, dev, shape=_tile_table_shape(dims))
+    _check_buf(name, "row_ptr", row_ptr, torch.int32, dev)
+    _check_buf(name, "col_idx", col_idx, torch.int32, dev)
+    shape = _shape(dims, head_dim, block_size)
+    with torch.cuda.device(dev):
+        _call(load_library().rt_pair_query_blocks(ctypes.byref(shape), _ptr(row_ptr), _ptr(col_idx),
+                                                  _ptr(tile_blocks), _stream_handle(dev, stream)),
+              name)
+    return tile_blocks
 
 
 def rt_take_device_error() -> int:

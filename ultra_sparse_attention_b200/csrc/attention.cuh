@@ -91,6 +91,9 @@ struct AttnArgs {
   float* out_zkept;
   float* out_u;
   __nv_bfloat16* out;
+  // sparse step: the query blocks of each 128-row tile, int32 [B*H][n_tiles][2]
+  // (-1: empty half); null = the neighbouring blocks
+  const int32_t* tile_blocks;
   int N;
   int d;
   int n_blocks;
@@ -275,7 +278,7 @@ __device__ __forceinline__ bool bitmap_has(const uint32_t* bm, int kb) { return 
 // Set the bits of the kept key blocks of query block `qb` of head `bh` (threads `t0, t0+stride, ...`).
 __device__ __forceinline__ void mark_kept_blocks(uint32_t* bm, const AttnArgs& a, int bh, int qb, int t0,
                                                  int stride) {
-  if (qb >= a.n_blocks) return;
+  if (qb < 0 || qb >= a.n_blocks) return;
   const size_t r = static_cast<size_t>(bh) * a.n_blocks + qb;
   const int s = a.row_ptr[r], e = a.row_ptr[r + 1];
   const int len = max(0, min(e - s, a.n_blocks));
@@ -292,6 +295,17 @@ __device__ __forceinline__ void mark_kept_blocks(uint32_t* bm, const AttnArgs& a
 // tile << 2 | (kept by query block 0) | (kept by query block 1) << 1, the
 // union of the tile's query blocks' kept lists in ascending order.
 __host__ __device__ constexpr int tile_list_cap(int N) { return (key_tiles(N) + 1 + 7) / 8 * 8; }
+
+// Query block in half h of 128-row tile qt of head bh, or -1 for none: the
+// pairing table's entry when there is one (out-of-range entries read as -1),
+// else the neighbouring blocks qt * (128 / BS) + h.
+template <int BS>
+__device__ __forceinline__ int tile_query_block(const AttnArgs& a, int n_qt, int bh, int qt, int h) {
+  if (h >= kBM / BS) return -1;
+  const int qb = a.tile_blocks != nullptr ? __ldg(a.tile_blocks + (static_cast<size_t>(bh) * n_qt + qt) * 2 + h)
+                                          : qt * (kBM / BS) + h;
+  return qb >= 0 && qb < a.n_blocks ? qb : -1;
+}
 
 
 // The sparse kernel.  Grid: up to two CTAs per SM, each walking query tiles
@@ -435,7 +449,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       const int t = tile_of(i), bh = t / n_qt, qt = t % n_qt;
       for (int w = lane; w < 2 * words; w += 32) bm[w] = 0u;
       __syncwarp();
-      for (int q = 0; q < kQB; ++q) mark_kept_blocks(bm + q * words, a, bh, qt * kQB + q, lane, 32);
+      for (int q = 0; q < kQB; ++q)
+        mark_kept_blocks(bm + q * words, a, bh, tile_query_block<BS>(a, n_qt, bh, qt, q), lane, 32);
       __syncwarp();
       uint16_t* out = lists + lb * cap;
       int count = 0;
@@ -469,8 +484,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       const int t = tile_of(i), bh = t / n_qt, qt = t % n_qt;
       if (lane == 0) {
         const unsigned char* stg = smem + L::kOffQ + (i & 1) * T::kQBytes;
-        tma_store_3d(&to, stg, 0, qt * kBM, bh);
-        if constexpr (T::kTail) tma_store_3d(&to_tail, stg + T::kQMain, 64, qt * kBM, bh);
+        // One BS-row box per query block of the tile.
+#pragma unroll
+        for (int h = 0; h < kQB; ++h) {
+          const int qb = tile_query_block<BS>(a, n_qt, bh, qt, h);
+          if (qb < 0) continue;
+          tma_store_3d(&to, stg + h * BS * 128, 0, qb * BS, bh);
+          if constexpr (T::kTail) tma_store_3d(&to_tail, stg + T::kQMain + h * BS * T::kTailRow, 64, qb * BS, bh);
+        }
         bulk_commit_group();
       }
       ++stores_issued;
@@ -489,7 +510,22 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         if (lane == 0) bulk_wait_group_read0();
         __syncwarp();
       }
-      if (lane == 0) load_q<D>(smem + L::kOffQ + (i & 1) * T::kQBytes, &tq, &tq_tail, &sh.q_full[i & 1], qt * kBM, bh);
+      if (lane == 0) {
+        // One BS-row box per query block of the tile; an empty half is not loaded (its
+        // rows keep no key tile, so their scores are never read).
+        unsigned char* dst = smem + L::kOffQ + (i & 1) * T::kQBytes;
+        int qb[kQB], n = 0;
+#pragma unroll
+        for (int h = 0; h < kQB; ++h) n += (qb[h] = tile_query_block<BS>(a, n_qt, bh, qt, h)) >= 0;
+        mbar_arrive_expect_tx(&sh.q_full[i & 1], n * (T::kQBytes / kQB));
+#pragma unroll
+        for (int h = 0; h < kQB; ++h) {
+          if (qb[h] < 0) continue;
+          tma_load_3d(dst + h * BS * 128, &tq, &sh.q_full[i & 1], 0, qb[h] * BS, bh);
+          if constexpr (T::kTail)
+            tma_load_3d(dst + T::kQMain + h * BS * T::kTailRow, &tq_tail, &sh.q_full[i & 1], 64, qb[h] * BS, bh);
+        }
+      }
       ++q_loads;
       for (int j = 0; j < count; ++j, ++g) {
         if (g >= NK && !warp_wait(&sh.step[(g - NK) & 7], ((g - NK) >> 3) & 1, abort_flag)) { ok = false; break; }
@@ -600,8 +636,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     // Prefetch into L2 the row of U that the epilogue of tile i reads.
     auto prefetch_u = [&](int i) {
       if (!has_stats || i >= n_mine) return;
-      const int t = tile_of(i), bh = t / n_qt, row = (t % n_qt) * kBM + r;
-      if (row >= a.N) return;
+      const int t = tile_of(i), bh = t / n_qt, qb = tile_query_block<BS>(a, n_qt, bh, t % n_qt, r / BS);
+      const int row = qb * BS + r % BS;
+      if (qb < 0 || row >= a.N) return;
       const size_t rg = static_cast<size_t>(bh) * a.N + row;
       const unsigned char* u = reinterpret_cast<const unsigned char*>(a.stat_u + rg * D);
 #pragma unroll
@@ -615,8 +652,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       zf = 1.f;
       zk = 1.f;
       if (!has_stats || i >= n_mine) return;
-      const int t = tile_of(i), bh = t / n_qt, row = (t % n_qt) * kBM + r;
-      if (row >= a.N) return;
+      const int t = tile_of(i), bh = t / n_qt, qb = tile_query_block<BS>(a, n_qt, bh, t % n_qt, r / BS);
+      const int row = qb * BS + r % BS;
+      if (qb < 0 || row >= a.N) return;
       const size_t rg = static_cast<size_t>(bh) * a.N + row;
       m = __ldg(a.stat_m + rg);
       zf = __ldg(a.stat_zfull + rg);
@@ -629,8 +667,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     for (int i = 0; i < n_mine; ++i) {
       prefetch_u(i + 1);
       const int t = tile_of(i), bh = t / n_qt, qt = t % n_qt;
-      const int row = qt * kBM + r;
-      const bool valid = row < a.N;
+      const int qb = tile_query_block<BS>(a, n_qt, bh, qt, r / BS);
+      const int row = qb * BS + r % BS;
+      const bool valid = qb >= 0 && row < a.N;
       const size_t row_g = static_cast<size_t>(bh) * a.N + (valid ? row : 0);
       const float mc2 = next_m * kLog2e, zf_c = next_zf, zk_c = next_zk;
       load_stats(i + 1, next_m, next_zf, next_zk);

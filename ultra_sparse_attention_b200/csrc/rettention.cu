@@ -17,6 +17,7 @@
 #include "ptx.cuh"
 #include "mask_builder.cuh"
 #include "attention.cuh"
+#include "pairing.cuh"
 
 namespace {
 
@@ -96,16 +97,18 @@ struct Maps {
   CUtensorMap q, q_tail, k, k_tail, v, v_tail, o, o_tail;
 };
 
-bool make_maps(Maps* m, const Dims& d, const void* q, const void* k, const void* v, const void* out) {
+// Q and O boxes are `q_rows` high: a whole 128-row tile for the capture kernel, one
+// query block for the sparse kernel (whose tiles may pair any two blocks of a head).
+bool make_maps(Maps* m, const Dims& d, const void* q, const void* k, const void* v, const void* out, int q_rows) {
   std::memset(m, 0, sizeof(*m));
-  bool ok = make_map(&m->q, q, d, 64, rt::kBM, true) && make_map(&m->k, k, d, 64, rt::kBN, true) &&
-            make_map(&m->v, v, d, 64, rt::kBN, true) && make_map(&m->o, out, d, 64, rt::kBM, true);
+  bool ok = make_map(&m->q, q, d, 64, q_rows, true) && make_map(&m->k, k, d, 64, rt::kBN, true) &&
+            make_map(&m->v, v, d, 64, rt::kBN, true) && make_map(&m->o, out, d, 64, q_rows, true);
   if (d.D > 64) {
     // Columns 64..D-1: 16 of them (32-byte swizzle) for D = 80, 64 (128-byte swizzle) for D = 128.
     const int tc = static_cast<int>(d.D) - 64;
     const bool wide = tc == 64;
-    ok = ok && make_map(&m->q_tail, q, d, tc, rt::kBM, wide) && make_map(&m->k_tail, k, d, tc, rt::kBN, wide) &&
-         make_map(&m->v_tail, v, d, tc, rt::kBN, wide) && make_map(&m->o_tail, out, d, tc, rt::kBM, wide);
+    ok = ok && make_map(&m->q_tail, q, d, tc, q_rows, wide) && make_map(&m->k_tail, k, d, tc, rt::kBN, wide) &&
+         make_map(&m->v_tail, v, d, tc, rt::kBN, wide) && make_map(&m->o_tail, out, d, tc, q_rows, wide);
   } else {
     m->q_tail = m->q;
     m->k_tail = m->k;
@@ -323,7 +326,7 @@ rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void*
     return RT_ERR_INVALID_ARGUMENT;
   if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
   Maps m;
-  if (!make_maps(&m, d, q, k, v, out)) return RT_ERR_CUDA;
+  if (!make_maps(&m, d, q, k, v, out, rt::kBM)) return RT_ERR_CUDA;
   AttnArgs a{};
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
@@ -341,9 +344,9 @@ rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void*
 }
 
 rt_status rt_attn_sparse_reshape(const rt_shape* shape, const void* q, const void* k, const void* v, float scale,
-                                 const int32_t* row_ptr, const int32_t* col_idx, const float* stat_m,
-                                 const float* stat_zfull, const float* stat_zkept, const float* stat_u, void* out,
-                                 rt_stream_t stream) {
+                                 const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_blocks,
+                                 const float* stat_m, const float* stat_zfull, const float* stat_zkept,
+                                 const float* stat_u, void* out, rt_stream_t stream) {
   Dims d;
   rt_status st = check_shape(shape, &d);
   if (st != RT_OK) return st;
@@ -351,15 +354,16 @@ rt_status rt_attn_sparse_reshape(const rt_shape* shape, const void* q, const voi
   const int nstats = (stat_m != nullptr) + (stat_zfull != nullptr) + (stat_zkept != nullptr) + (stat_u != nullptr);
   if (nstats != 0 && nstats != 4) return RT_ERR_INVALID_ARGUMENT;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(stat_u, 16) ||
-      !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(stat_m, 4) || !aligned(stat_zfull, 4) ||
-      !aligned(stat_zkept, 4))
+      !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(tile_blocks, 4) || !aligned(stat_m, 4) ||
+      !aligned(stat_zfull, 4) || !aligned(stat_zkept, 4))
     return RT_ERR_INVALID_ARGUMENT;
   if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
   Maps m;
-  if (!make_maps(&m, d, q, k, v, out)) return RT_ERR_CUDA;
+  if (!make_maps(&m, d, q, k, v, out, static_cast<int>(d.bs))) return RT_ERR_CUDA;
   AttnArgs a{};
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
+  a.tile_blocks = tile_blocks;
   a.stat_m = stat_m;
   a.stat_zfull = stat_zfull;
   a.stat_zkept = stat_zkept;
@@ -371,6 +375,51 @@ rt_status rt_attn_sparse_reshape(const rt_shape* shape, const void* q, const voi
   a.n_heads = static_cast<int>(d.bh);
   a.scale_log2 = scale * rt::kLog2e;
   return dispatch_attention<false>(d, m, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+rt_status rt_pair_query_blocks(const rt_shape* shape, const int32_t* row_ptr, const int32_t* col_idx,
+                               int32_t* tile_blocks, rt_stream_t stream) {
+  Dims d;
+  rt_status st = check_shape(shape, &d);
+  if (st != RT_OK) return st;
+  if (!row_ptr || !col_idx || !tile_blocks) return RT_ERR_INVALID_ARGUMENT;
+  if (!aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(tile_blocks, 4)) return RT_ERR_INVALID_ARGUMENT;
+  const int nb = static_cast<int>(d.n_blocks);
+  const int n_tiles = rt::query_tiles(static_cast<int>(d.N));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d.bs != 64) {  // one query block per tile: the identity table
+    rt::pair_match_kernel<<<static_cast<unsigned>(d.bh), rt::kPairThreads, 0, s>>>(nullptr, nb, n_tiles,
+                                                                                 static_cast<int>(d.bs), tile_blocks);
+    return launch_status();
+  }
+  // Candidates of every query block go through a transient workspace (int16 [B*H][n_blocks][8]).
+  const size_t cand_smem = rt::pair_candidates_smem_bytes(nb), match_smem = rt::pair_match_smem_bytes(nb);
+  // Block i's kept-set bitmap lives in registers, in the smallest of these word counts that holds it.
+  const int words = (nb + 31) / 32;
+  auto cand_kernel = words <= 8    ? rt::pair_candidates_kernel<8>
+                     : words <= 12 ? rt::pair_candidates_kernel<12>
+                     : words <= 16 ? rt::pair_candidates_kernel<16>
+                     : words <= 32 ? rt::pair_candidates_kernel<32>
+                                   : rt::pair_candidates_kernel<64>;
+  static_assert(kMaxBlocks <= 64 * 32, "pairing bitmap words");
+  if (cudaFuncSetAttribute(cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(cand_smem)) != cudaSuccess ||
+      cudaFuncSetAttribute(rt::pair_match_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(match_smem)) != cudaSuccess)
+    return RT_ERR_CUDA;
+  int16_t* cand = nullptr;
+  if (!workspace_alloc(reinterpret_cast<void**>(&cand), static_cast<size_t>(d.bh) * nb * rt::kPairCands * 2, s))
+    return RT_ERR_CUDA;
+  dim3 grid(static_cast<unsigned>((nb + rt::kCandBlocks - 1) / rt::kCandBlocks), static_cast<unsigned>(d.bh));
+  cand_kernel<<<grid, rt::kPairThreads, cand_smem, s>>>(row_ptr, col_idx, nb, cand);
+  st = launch_status();
+  if (st == RT_OK) {
+    rt::pair_match_kernel<<<static_cast<unsigned>(d.bh), rt::kPairThreads, match_smem, s>>>(cand, nb, n_tiles, 64,
+                                                                                          tile_blocks);
+    st = launch_status();
+  }
+  if (cudaFreeAsync(cand, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
+  return st;
 }
 
 rt_status rt_build_block_mask_static(const rt_shape* shape, const void* q, const void* k, float scale,
