@@ -67,8 +67,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         sys.stderr.write(res.stdout + res.stderr)
-    with open(LIB + ".ptxas.txt", "w") as f:
-        f.write(res.stderr)
+    with open(LIB + ".ptxas.txt", "w") as f:  # registers, spills, stack per kernel (compile times dropped)
+        f.write("".join(ln for ln in res.stderr.splitlines(keepends=True) if "Compile time" not in ln))
     os.replace(tmp, LIB)
     with open(STAMP, "w") as f:
         f.write(source_hash())
