@@ -22,7 +22,10 @@
 //    its own kept list; the sparse kernel walks the union of both lists and a
 //    row whose block does not keep a tile writes P = 0 for it.  (An M = 64 MMA
 //    per query block would halve the tensor rate; the union costs only the
-//    blocks the two lists do not share.)
+//    blocks the two lists do not share, and the sparse step takes its pairs
+//    of query blocks from a table that pairs blocks with similar lists, see
+//    pairing.cuh.)
+//  * Head dim 128 is two 64-column tiles with 128-byte swizzle.
 //  * Online softmax in base 2 (x = s * scale * log2 e) with a lazy reference:
 //    O is rescaled only when the row max moves up by more than 8 (or down by
 //    more than 64 in the sparse step, whose reference starts at the cached
