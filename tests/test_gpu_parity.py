@@ -236,6 +236,33 @@ def test_sparse_with_any_tile_table_is_bit_identical(cuda_device, N, d, D, bs):
     compare_out(out.reshape(-1, D), want, d, "sparse O (random tile table, no statistics)")
 
 
+@pytest.mark.parametrize("D,d", [(64, 64), (80, 72)])
+def test_sparse_tile_table_with_missing_and_repeated_blocks(cuda_device, D, d):
+    """A table entry out of range is an empty half, a block in no tile leaves its rows
+    unwritten, and a block in two halves is computed twice with the same result."""
+    N, bs = 1000, 64
+    w = _wl(N, d, D, bs, std=1.0, seed=29, drift=0.05)
+    (h0, h1), (d0, d1) = _inputs(w, cuda_device)
+    bh, nb = w.batch * w.heads, w.n_blocks
+    rp, ci = random_csr(bh, nb, w.keep_blocks(Fraction(1, 4)), seed=31, forced=1)
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale, row_ptr=to_dev(rp, cuda_device), col_idx=to_dev(ci, cuda_device))
+    _, st = usa.rt_attn_full_capture(*d0, **kw)
+    base = usa.rt_attn_sparse_reshape(*d1, stats=st, **kw)
+    n_tiles = -(-N // 128)
+    table = np.arange(2 * n_tiles, dtype=np.int32).reshape(1, n_tiles, 2).repeat(bh, 0)
+    table[:, 2, 1] = nb + 7       # block 5: out of range -> empty half, rows unwritten
+    table[:, 3, 0] = 7            # block 6 missing, block 7 in both halves of tile 3
+    table[:, n_tiles - 1, 1] = -1  # block 15 missing
+    out = torch.full_like(base, float("nan"))
+    usa.rt_attn_sparse_reshape(*d1, stats=st, tile_blocks=to_dev(table, cuda_device), out=out, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    rows = torch.arange(N, device=cuda_device) // bs
+    missing = (rows == 5) | (rows == 6) | (rows == 15)
+    assert torch.isnan(out[:, :, missing].float()).all()
+    assert torch.equal(out[:, :, ~missing].view(torch.int16), base[:, :, ~missing].view(torch.int16))
+
+
 @pytest.mark.parametrize("N,d,D,bs", [(1000, 64, 64, 64), (1000, 72, 80, 64), (200, 64, 64, 64), (896, 64, 64, 128),
                                       (1000, 128, 128, 64)])
 @pytest.mark.parametrize("gain", [3.0, 0.25])
