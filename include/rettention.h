@@ -66,14 +66,15 @@
 extern "C" {
 #endif
 
-#define RT_ABI_VERSION 2
+#define RT_ABI_VERSION 3
 
 typedef enum rt_status {
     RT_OK = 0,
     RT_ERR_INVALID_ARGUMENT = 1,
     RT_ERR_UNSUPPORTED = 2,
     RT_ERR_CUDA = 3,
-    RT_ERR_TIMEOUT = 4
+    RT_ERR_TIMEOUT = 4,
+    RT_ERR_RANGE = 5
 } rt_status;
 
 /* Same type as cudaStream_t, spelled without the CUDA headers. */
@@ -137,6 +138,14 @@ rt_status rt_build_block_mask(const rt_shape *shape, const void *q, const void *
  *   Z_kept_i = sum_{j in K(i)} exp(s_ij - m_i)
  *   U_i      = sum_{j not in K(i)} exp(s_ij - m_i) * v_j
  *   out_i    = sum_j exp(s_ij - m_i) * v_j / Z_full_i       (full attention, bf16)
+ *
+ * The P V products take the probabilities in f16 with an f16 copy of V, made
+ * by the call in a transient device workspace of B*H*N*D*2 bytes from the
+ * library's stream-ordered pool: every term of U and out is rounded to 11
+ * mantissa bits of p (a relative error below 2^-12).  V must therefore lie in
+ * the f16 range: a finite |v| above 65504 records RT_ERR_RANGE in the device
+ * status word (read it with rt_take_device_error) and the outputs are left
+ * unspecified.
  *
  * q, k, v       bf16 [B,H,N,D] device.
  * row_ptr, col_idx  CSR of kept blocks (for example from rt_build_block_mask).
@@ -229,7 +238,8 @@ int32_t rt_abi_version(void);
 /*
  * rt_take_device_error -- read and clear the device status word of the
  * current CUDA device.  Waits for all work on the device to finish first.
- * *code receives RT_OK or the first error a kernel recorded (RT_ERR_TIMEOUT).
+ * *code receives RT_OK or the first error a kernel recorded (RT_ERR_TIMEOUT, or
+ * RT_ERR_RANGE from rt_attn_full_capture).
  * While the word holds an error, this library's kernels return at once
  * without touching their outputs, so clear it before going on.
  */

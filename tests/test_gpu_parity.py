@@ -436,6 +436,32 @@ def test_timeout_self_test_reports_and_recovers(cuda_device):
     assert float(x.sum()) == 4.0
 
 
+def test_capture_reports_values_outside_the_f16_range(cuda_device):
+    """The capture's PV products run on an f16 copy of V: a finite |v| above 65504 records
+    RT_ERR_RANGE, the next kernels of the library skip, and after the status is read a
+    capture of in-range values matches the oracle; infinities are not a range error."""
+    N, d, D, bs = 1000, 64, 64, 64
+    w = _wl(N, d, D, bs, std=1.0, seed=41, drift=0.05)
+    (h0, _), (d0, _) = _inputs(w, cuda_device)
+    rp, ci = random_csr(w.batch * w.heads, w.n_blocks, 4, seed=43, forced=1)
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale, row_ptr=to_dev(rp, cuda_device), col_idx=to_dev(ci, cuda_device))
+    assert usa.rt_take_device_error() == 0
+    v_big = d0[2].clone()
+    v_big[1, 2, 777, 5] = 1.0e5
+    usa.rt_attn_full_capture(d0[0], d0[1], v_big, **kw)
+    assert usa.rt_take_device_error() == usa.RT_ERR_RANGE
+    assert usa.rt_take_device_error() == 0
+    v_inf = d0[2].clone()
+    v_inf[0, 0, 3, 0] = float("inf")
+    usa.rt_attn_full_capture(d0[0], d0[1], v_inf, **kw)
+    assert usa.rt_take_device_error() == 0
+    out, st = usa.rt_attn_full_capture(*d0, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    orc = oracle.full_capture(*h0, d, bs, w.scale, rp, ci)
+    compare_out(out.reshape(-1, D), orc["o"], d, "capture O after a range error")
+
+
 # ------------------------------------------------------------------ maximum size
 def test_cycle_at_the_block_limit(cuda_device):
     """One mask + capture + sparse cycle at the largest supported block count (2048 blocks

@@ -78,6 +78,7 @@ struct Tiles {
   static constexpr int kKSteps = D / 16;
   // PV into the tail columns of the accumulator: N = the tail's width.
   static constexpr uint32_t kIdescPVTail = idesc_bf16(kBM, kTail ? kTailCols : 16, false, true);
+  static constexpr uint32_t kIdescPVTailF16 = idesc_f16(kBM, kTail ? kTailCols : 16, false, true);
 };
 
 struct AttnArgs {
@@ -111,6 +112,7 @@ __host__ __device__ constexpr int query_tiles(int N) { return (N + kBM - 1) / kB
 // ------------------------------------------------------------------ MMA issue
 constexpr uint32_t kIdescQK = idesc_bf16(kBM, kBN, false, false);
 constexpr uint32_t kIdescPV64 = idesc_bf16(kBM, 64, false, true);
+constexpr uint32_t kIdescPV64F16 = idesc_f16(kBM, 64, false, true);  // capture: f16 P and f16 V
 
 // S = Q K^T for one key tile into TMEM at `s_tmem`, Q and K in shared memory.
 // The issue helpers below are warp-collective (one elected lane issues).  The
@@ -155,21 +157,23 @@ __device__ __forceinline__ void copy_q_to_tmem(uint32_t q_tmem, uint32_t q_base)
   static_assert(!Tiles<D>::kTail, "Q in TMEM is used for head dim 64 only");
 }
 
-// acc (+)= P V for one key tile; P is bf16 in TMEM at `p_tmem` (32 columns).
-template <int D>
+// acc (+)= P V for one key tile; P is in TMEM at `p_tmem` (32 columns), bf16 with bf16 V,
+// or f16 with f16 V when kF16 (the capture kernel).
+template <int D, bool kF16 = false>
 __device__ __forceinline__ void issue_pv(uint32_t acc_tmem, uint32_t p_tmem, uint32_t v_base, bool accumulate) {
+  constexpr uint32_t kId = kF16 ? kIdescPV64F16 : kIdescPV64;
+  constexpr uint32_t kIdTail = kF16 ? Tiles<D>::kIdescPVTailF16 : Tiles<D>::kIdescPVTail;
   const uint64_t vd = smem_desc(v_base, Tiles<D>::kKVMain, 1024, kSwizzle128B);
   const uint32_t acc0 = accumulate ? 1u : 0u;
-  mma_ts_w(acc_tmem, p_tmem, vd, kIdescPV64, acc0);
+  mma_ts_w(acc_tmem, p_tmem, vd, kId, acc0);
 #pragma unroll
-  for (int ks = 1; ks < kBN / 16; ++ks) mma_ts_w(acc_tmem, p_tmem + ks * 8, vd + 128 * ks, kIdescPV64, 1u);
+  for (int ks = 1; ks < kBN / 16; ++ks) mma_ts_w(acc_tmem, p_tmem + ks * 8, vd + 128 * ks, kId, 1u);
   if constexpr (Tiles<D>::kTail) {
     using T = Tiles<D>;
     const uint64_t vt = smem_desc(v_base + T::kKVMain, T::kKVTail, T::kTailSBO, T::kTailSwizzle);
-    mma_ts_w(acc_tmem + 64, p_tmem, vt, T::kIdescPVTail, acc0);
+    mma_ts_w(acc_tmem + 64, p_tmem, vt, kIdTail, acc0);
 #pragma unroll
-    for (int ks = 1; ks < kBN / 16; ++ks)
-      mma_ts_w(acc_tmem + 64, p_tmem + ks * 8, vt + T::kTailRow * ks, T::kIdescPVTail, 1u);
+    for (int ks = 1; ks < kBN / 16; ++ks) mma_ts_w(acc_tmem + 64, p_tmem + ks * 8, vt + T::kTailRow * ks, kIdTail, 1u);
   }
 }
 
@@ -841,17 +845,18 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 //
 // One CTA per 128-row query tile, every key tile in order.  Each key tile's
 // P V goes to O_kept (rows whose query block keeps the tile's block) and/or
-// to U (the other rows), where U takes P as a bf16 high part plus a bf16
-// residual so the cached numerator keeps about 16 bits of P.
+// to U (the other rows).  The PV products take P in f16 with V in f16 (an f16
+// copy of V made by convert_v_f16_kernel before the launch): P keeps 11
+// mantissa bits, a rounding error below 2^-12 of each term of U, in one
+// product per key tile.
 //
 // S is double-buffered in TMEM, so QK^T(j+1) runs while the softmax works on
 // tile j: the MMA warp issues QK^T(j+1) as soon as PV(j-1) -- the last reader
 // of that buffer -- is issued, then waits for P(j) and issues PV(j).
 // A tile that is kept by some rows and masked for others ("mixed"; a few per
-// cent of the tiles) needs P twice: the masked rows' high/low parts stay in
-// the S buffer (kept rows zero) for the U products, and the kept rows' P goes
-// to a shared-memory tile (masked rows zero) read by one SS product into
-// O_kept.
+// cent of the tiles) needs P twice: the masked rows' P stays in the S buffer
+// (kept rows zero) for the U product, and the kept rows' P goes to a
+// shared-memory tile (masked rows zero) read by one SS product into O_kept.
 // TMEM: S0 [0,64) S1 [64,128) O_kept [128,128+D) U at kOUCol.  Head dim 64
 // fits in 256 columns, so two CTAs share an SM (two softmax warps per SM
 // sub-partition); head dim 80 takes 512 columns and one CTA per SM.
@@ -864,7 +869,7 @@ struct CaptureLayout {
   static constexpr int kStages = 4;
   static constexpr int kOffQ = 0;
   static constexpr int kOffStage0 = T::kQBytes;
-  static constexpr int kOffPK = kOffStage0 + kStages * T::kStageBytes;  // 128 x 64 bf16, 128-byte swizzle
+  static constexpr int kOffPK = kOffStage0 + kStages * T::kStageBytes;  // 128 x 64 f16, 128-byte swizzle
   static constexpr int kOffShared = kOffPK + kBM * 128;
   static constexpr size_t kMinSmem = D == 64 ? 0 : 120 * 1024;  // D > 64: keep one CTA per SM
 };
@@ -886,22 +891,22 @@ __host__ __device__ constexpr size_t capture_smem_bytes(int n_blocks) {
   return s > CaptureLayout<D>::kMinSmem ? s : CaptureLayout<D>::kMinSmem;
 }
 
-// acc (+)= P V with P (128 x 64 bf16) in shared memory, K-major with 128-byte swizzle.
+// acc (+)= P V with P (128 x 64 f16) in shared memory, K-major with 128-byte swizzle, and f16 V.
 template <int D>
 __device__ __forceinline__ void issue_pv_ss(uint32_t acc_tmem, uint32_t p_base, uint32_t v_base, bool accumulate) {
   const uint64_t pd = smem_desc(p_base, 16, 1024, kSwizzle128B);
   const uint64_t vd = smem_desc(v_base, Tiles<D>::kKVMain, 1024, kSwizzle128B);
   const uint32_t acc0 = accumulate ? 1u : 0u;
-  mma_ss_w(acc_tmem, pd, vd, kIdescPV64, acc0);
+  mma_ss_w(acc_tmem, pd, vd, kIdescPV64F16, acc0);
 #pragma unroll
-  for (int ks = 1; ks < kBN / 16; ++ks) mma_ss_w(acc_tmem, pd + 2 * ks, vd + 128 * ks, kIdescPV64, 1u);
+  for (int ks = 1; ks < kBN / 16; ++ks) mma_ss_w(acc_tmem, pd + 2 * ks, vd + 128 * ks, kIdescPV64F16, 1u);
   if constexpr (Tiles<D>::kTail) {
     using T = Tiles<D>;
     const uint64_t vt = smem_desc(v_base + T::kKVMain, T::kKVTail, T::kTailSBO, T::kTailSwizzle);
-    mma_ss_w(acc_tmem + 64, pd, vt, T::kIdescPVTail, acc0);
+    mma_ss_w(acc_tmem + 64, pd, vt, T::kIdescPVTailF16, acc0);
 #pragma unroll
     for (int ks = 1; ks < kBN / 16; ++ks)
-      mma_ss_w(acc_tmem + 64, pd + 2 * ks, vt + T::kTailRow * ks, T::kIdescPVTail, 1u);
+      mma_ss_w(acc_tmem + 64, pd + 2 * ks, vt + T::kTailRow * ks, T::kIdescPVTailF16, 1u);
   }
 }
 
@@ -1023,11 +1028,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       const uint32_t v_base = sbase + L::kOffStage0 + (j % NS) * T::kStageBytes + T::kKVBytes;
       const uint32_t sbuf = tmem + (j & 1) * 64;
       if (!masked_any) {  // kept by every row: P in the S buffer
-        issue_pv<D>(tmem + L::kOKCol, sbuf, v_base, ok_started);
+        issue_pv<D, true>(tmem + L::kOKCol, sbuf, v_base, ok_started);
         ok_started = true;
       } else {
-        issue_pv<D>(tmem + L::kOUCol, sbuf, v_base, ou_started);   // bf16(p)
-        issue_pv<D>(tmem + L::kOUCol, sbuf + 32, v_base, true);    // p - bf16(p)
+        issue_pv<D, true>(tmem + L::kOUCol, sbuf, v_base, ou_started);  // masked rows' P (kept rows 0)
         ou_started = true;
         if (kept_any) {  // mixed: the kept rows' P is in shared memory
           issue_pv_ss<D>(tmem + L::kOKCol, sbase + L::kOffPK, v_base, ok_started);
@@ -1101,7 +1105,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           s[c] = ex2_approx(x0);
           s[c + 1] = ex2_approx(x1);
           zz = f2_add(zz, f2_pack(s[c], s[c + 1]));
-          pk[c / 2] = pack_bf16x2(s[c], s[c + 1]);
+          pk[c / 2] = pack_f16x2(s[c], s[c + 1]);
         }
         float z0, z1;
         f2_unpack(zz, z0, z1);
@@ -1113,20 +1117,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         tmem_st32(sbuf, pk);  // kept by every row
       } else {
         if (!kept) {
-          uint32_t lo[32];  // residual p - bf16(p), so U keeps ~16 mantissa bits of p
-          const uint64_t m1 = f2_pack(-1.f, -1.f);
-#pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            float r0, r1;  // p - bf16(p), exact in fp32
-            f2_unpack(f2_fma(f2_pack(bf16_lo_to_f32(pk[c / 2]), bf16_hi_to_f32(pk[c / 2])), m1, f2_pack(s[c], s[c + 1])),
-                      r0, r1);
-            lo[c / 2] = pack_bf16x2(r0, r1);
-          }
           tmem_st32(sbuf, pk);
-          tmem_st32(sbuf + 32, lo);
         } else {
           tmem_st32_zero(sbuf);
-          tmem_st32_zero(sbuf + 32);
         }
         if (kept_any) {
           // Mixed tile: the kept rows' P (masked rows zero) into the shared-memory tile, once
@@ -1201,6 +1194,29 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
+}
+
+// f16 copy of V for the capture kernel's PV products, 8 elements per thread and step.  A
+// finite value outside the f16 range (|v| > 65504) records RT_ERR_RANGE in the device
+// status word, so the capture kernel after it does nothing.
+__global__ void __launch_bounds__(256) convert_v_f16_kernel(const uint4* __restrict__ v, uint4* __restrict__ v16,
+                                                            size_t n8) {
+  if (device_status_set()) return;  // an earlier kernel failed
+  bool range = true;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint4 x = __ldg(v + i);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t h[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a = bf16_lo_to_f32(w[k]), b = bf16_hi_to_f32(w[k]);
+      range = range && !(fabsf(a) > 65504.f && fabsf(a) != INFINITY) && !(fabsf(b) > 65504.f && fabsf(b) != INFINITY);
+      h[k] = pack_f16x2(a, b);
+    }
+    v16[i] = make_uint4(h[0], h[1], h[2], h[3]);
+  }
+  if (!range) record_device_status(RT_ERR_RANGE);
 }
 
 // Failure-detection self test: wait on a barrier nothing completes.

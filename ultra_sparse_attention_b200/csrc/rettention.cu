@@ -78,15 +78,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor [bh][N][D] viewed as 3-D (D, N, bh); box of `box_cols` x `box_rows` x 1.
-bool make_map(CUtensorMap* m, const void* base, const Dims& d, int box_cols, int box_rows, bool swizzle128) {
+// bf16 (or f16) tensor [bh][N][D] viewed as 3-D (D, N, bh); box of `box_cols` x `box_rows` x 1.
+bool make_map(CUtensorMap* m, const void* base, const Dims& d, int box_cols, int box_rows, bool swizzle128,
+              CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d.D), static_cast<cuuint64_t>(d.N), static_cast<cuuint64_t>(d.bh)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d.D * 2), static_cast<cuuint64_t>(d.N * d.D * 2)};
   cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(m, type, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -99,16 +100,19 @@ struct Maps {
 
 // Q and O boxes are `q_rows` high: a whole 128-row tile for the capture kernel, one
 // query block for the sparse kernel (whose tiles may pair any two blocks of a head).
-bool make_maps(Maps* m, const Dims& d, const void* q, const void* k, const void* v, const void* out, int q_rows) {
+// V is f16 for the capture kernel (v_f16), bf16 otherwise.
+bool make_maps(Maps* m, const Dims& d, const void* q, const void* k, const void* v, const void* out, int q_rows,
+               bool v_f16 = false) {
   std::memset(m, 0, sizeof(*m));
+  const CUtensorMapDataType vt = v_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   bool ok = make_map(&m->q, q, d, 64, q_rows, true) && make_map(&m->k, k, d, 64, rt::kBN, true) &&
-            make_map(&m->v, v, d, 64, rt::kBN, true) && make_map(&m->o, out, d, 64, q_rows, true);
+            make_map(&m->v, v, d, 64, rt::kBN, true, vt) && make_map(&m->o, out, d, 64, q_rows, true);
   if (d.D > 64) {
     // Columns 64..D-1: 16 of them (32-byte swizzle) for D = 80, 64 (128-byte swizzle) for D = 128.
     const int tc = static_cast<int>(d.D) - 64;
     const bool wide = tc == 64;
     ok = ok && make_map(&m->q_tail, q, d, tc, q_rows, wide) && make_map(&m->k_tail, k, d, tc, rt::kBN, wide) &&
-         make_map(&m->v_tail, v, d, tc, rt::kBN, wide) && make_map(&m->o_tail, out, d, tc, q_rows, wide);
+         make_map(&m->v_tail, v, d, tc, rt::kBN, wide, vt) && make_map(&m->o_tail, out, d, tc, q_rows, wide);
   } else {
     m->q_tail = m->q;
     m->k_tail = m->k;
@@ -281,6 +285,7 @@ const char* rt_status_string(rt_status status) {
     case RT_ERR_UNSUPPORTED: return "RT_ERR_UNSUPPORTED: head dim, block size or size outside the supported set";
     case RT_ERR_CUDA: return "RT_ERR_CUDA: a CUDA call or kernel launch failed";
     case RT_ERR_TIMEOUT: return "RT_ERR_TIMEOUT: a kernel wait ran out and the kernel stopped";
+    case RT_ERR_RANGE: return "RT_ERR_RANGE: an input value outside the range the kernels compute in";
   }
   return "unknown rt_status";
 }
@@ -325,8 +330,20 @@ rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void*
       !aligned(stat_zkept, 4))
     return RT_ERR_INVALID_ARGUMENT;
   if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // The PV products run on f16 P and an f16 copy of V (a transient workspace).
+  const size_t v_elems = static_cast<size_t>(d.bh) * d.N * d.D;
+  void* v16 = nullptr;
+  if (!workspace_alloc(&v16, v_elems * 2, s)) return RT_ERR_CUDA;
   Maps m;
-  if (!make_maps(&m, d, q, k, v, out, rt::kBM)) return RT_ERR_CUDA;
+  if (!make_maps(&m, d, q, k, v16, out, rt::kBM, true)) {
+    cudaFreeAsync(v16, s);
+    return RT_ERR_CUDA;
+  }
+  const size_t n8 = v_elems / 8;  // D is a multiple of 16
+  const unsigned cgrid = static_cast<unsigned>(std::min<size_t>((n8 + 255) / 256, 8 * static_cast<size_t>(sm_count())));
+  rt::convert_v_f16_kernel<<<cgrid, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), n8);
+  st = launch_status();
   AttnArgs a{};
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
@@ -340,7 +357,9 @@ rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void*
   a.n_blocks = static_cast<int>(d.n_blocks);
   a.n_heads = static_cast<int>(d.bh);
   a.scale_log2 = scale * rt::kLog2e;
-  return dispatch_attention<true>(d, m, a, reinterpret_cast<cudaStream_t>(stream));
+  if (st == RT_OK) st = dispatch_attention<true>(d, m, a, s);
+  if (cudaFreeAsync(v16, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
+  return st;
 }
 
 rt_status rt_attn_sparse_reshape(const rt_shape* shape, const void* q, const void* k, const void* v, float scale,
