@@ -50,7 +50,8 @@
  * RT_ERR_CUDA.  Kernels never trap: every wait inside a kernel is bounded;
  * when one runs out the kernel records RT_ERR_TIMEOUT in a device status word
  * (read it with rt_take_device_error), leaves its outputs unspecified and
- * returns.  The CSR must be readable where row_ptr points: row_ptr holds
+ * returns.  A V value outside the f16 range at the capture step records
+ * RT_ERR_RANGE there the same way (see rt_attn_full_capture).  The CSR must be readable where row_ptr points: row_ptr holds
  * B*H*n_blocks + 1 entries and 0 <= row_ptr[r] <= row_ptr[r+1] <= the length
  * of col_idx (the library cannot see that length).  Beyond that, malformed
  * contents (block indices out of range, unsorted or repeated entries, rows
