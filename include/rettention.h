@@ -146,7 +146,8 @@ rt_status rt_build_block_mask(const rt_shape *shape, const void *q, const void *
  * mantissa bits of p (a relative error below 2^-12).  V must therefore lie in
  * the f16 range: a finite |v| above 65504 records RT_ERR_RANGE in the device
  * status word (read it with rt_take_device_error) and the outputs are left
- * unspecified.
+ * unspecified; values below 2^-14 in magnitude become f16 subnormals (spacing
+ * 2^-24), so the 2^-12 bound holds for V of ordinary activation magnitude.
  *
  * q, k, v       bf16 [B,H,N,D] device.
  * row_ptr, col_idx  CSR of kept blocks (for example from rt_build_block_mask).
