@@ -115,3 +115,13 @@ def test_python_binding_rejects_cpu_tensors():
     q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         usa.rt_build_block_mask(q, q, head_dim=64, block_size=64, scale=0.125, keep_blocks=1)
+
+
+def test_source_hash_covers_code_not_comments():
+    """The build stamp (and the DRAM traffic keyed to it) changes with the code only."""
+    from ultra_sparse_attention_b200 import build as b
+    src = 'int a = 1; // note\n/* block\n note */ const char* s = "x // kept /* kept */";\nchar q = \'"\';  int  b;'
+    assert b.code_text(src) == 'int a = 1; const char* s = "x // kept /* kept */"; char q = \'"\'; int b;'
+    edited = src.replace("// note", "// another note\n// and a line more").replace("  int", "\n\nint")
+    assert b.code_text(edited) == b.code_text(src)
+    assert b.code_text(src.replace("a = 1", "a = 2")) != b.code_text(src)

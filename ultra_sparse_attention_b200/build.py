@@ -2,7 +2,10 @@
 
 The library is rebuilt when the hash of its sources, of the public header or
 of the compiler flags changes; the hash is kept beside the .so, so a copy of
-the tree with different file times does not trigger a rebuild.
+the tree with different file times does not trigger a rebuild.  The hash
+covers the code only: comments and the amount of white space are left out,
+so a documentation edit neither rebuilds the library nor makes measurements
+keyed to the hash (the DRAM traffic in profiles/) look stale.
 """
 from __future__ import annotations
 
@@ -33,12 +36,36 @@ def _sources() -> list[str]:
     return files
 
 
+def code_text(text: str) -> str:
+    """C/C++/CUDA source without its comments, white space runs collapsed to one space."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":  # string or character literal, copied as is
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_hash() -> str:
     h = hashlib.sha256(" ".join(NVCC_FLAGS).encode())
     for f in _sources():
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            h.update(code_text(fh.read()).encode())
     return h.hexdigest()
 
 
