@@ -50,8 +50,7 @@
  * RT_ERR_CUDA.  Kernels never trap: every wait inside a kernel is bounded;
  * when one runs out the kernel records RT_ERR_TIMEOUT in a device status word
  * (read it with rt_take_device_error), leaves its outputs unspecified and
- * returns.  A V value outside the f16 range at the capture step records
- * RT_ERR_RANGE there the same way (see rt_attn_full_capture).  The CSR must be readable where row_ptr points: row_ptr holds
+ * returns.  The CSR must be readable where row_ptr points: row_ptr holds
  * B*H*n_blocks + 1 entries and 0 <= row_ptr[r] <= row_ptr[r+1] <= the length
  * of col_idx (the library cannot see that length).  Beyond that, malformed
  * contents (block indices out of range, unsorted or repeated entries, rows
@@ -67,15 +66,14 @@
 extern "C" {
 #endif
 
-#define RT_ABI_VERSION 3
+#define RT_ABI_VERSION 4
 
 typedef enum rt_status {
     RT_OK = 0,
     RT_ERR_INVALID_ARGUMENT = 1,
     RT_ERR_UNSUPPORTED = 2,
     RT_ERR_CUDA = 3,
-    RT_ERR_TIMEOUT = 4,
-    RT_ERR_RANGE = 5
+    RT_ERR_TIMEOUT = 4
 } rt_status;
 
 /* Same type as cudaStream_t, spelled without the CUDA headers. */
@@ -141,13 +139,12 @@ rt_status rt_build_block_mask(const rt_shape *shape, const void *q, const void *
  *   out_i    = sum_j exp(s_ij - m_i) * v_j / Z_full_i       (full attention, bf16)
  *
  * The P V products take the probabilities in f16 with an f16 copy of V, made
- * by the call in a transient device workspace of B*H*N*D*2 bytes from the
- * library's stream-ordered pool: every term of U and out is rounded to 11
- * mantissa bits of p (a relative error below 2^-12).  V must therefore lie in
- * the f16 range: a finite |v| above 65504 records RT_ERR_RANGE in the device
- * status word (read it with rt_take_device_error) and the outputs are left
- * unspecified; values below 2^-14 in magnitude become f16 subnormals (spacing
- * 2^-24), so the 2^-12 bound holds for V of ordinary activation magnitude.
+ * by the call in a transient device workspace of B*H*N*D*2 + B*H*4 bytes from
+ * the library's stream-ordered pool: every term of U and out is rounded to 11
+ * mantissa bits of p (a relative error below 2^-12).  The copy is scaled per
+ * (batch, head) by the power of two that puts max |v| in [2^14, 2^15) and the
+ * scale is taken out exactly afterwards, so any finite V keeps 11 mantissa
+ * bits down to 2^-30 of its head's largest |v|.
  *
  * q, k, v       bf16 [B,H,N,D] device.
  * row_ptr, col_idx  CSR of kept blocks (for example from rt_build_block_mask).
@@ -240,8 +237,7 @@ int32_t rt_abi_version(void);
 /*
  * rt_take_device_error -- read and clear the device status word of the
  * current CUDA device.  Waits for all work on the device to finish first.
- * *code receives RT_OK or the first error a kernel recorded (RT_ERR_TIMEOUT, or
- * RT_ERR_RANGE from rt_attn_full_capture).
+ * *code receives RT_OK or the first error a kernel recorded (RT_ERR_TIMEOUT).
  * While the word holds an error, this library's kernels return at once
  * without touching their outputs, so clear it before going on.
  */

@@ -32,8 +32,8 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    assert usa.rt_abi_version() == 3
-    for code in range(6):
+    assert usa.rt_abi_version() == 4
+    for code in range(5):
         s = usa.rt_status_string(code)
         assert s.startswith("RT_")
     assert usa.rt_status_string(99) == "unknown rt_status"

@@ -436,30 +436,33 @@ def test_timeout_self_test_reports_and_recovers(cuda_device):
     assert float(x.sum()) == 4.0
 
 
-def test_capture_reports_values_outside_the_f16_range(cuda_device):
-    """The capture's PV products run on an f16 copy of V: a finite |v| above 65504 records
-    RT_ERR_RANGE, the next kernels of the library skip, and after the status is read a
-    capture of in-range values matches the oracle; infinities are not a range error."""
+@pytest.mark.parametrize("v_scale", [1.0e5, 3.0e-7])
+def test_capture_with_large_and_tiny_v(cuda_device, v_scale):
+    """The capture's PV products run on an f16 copy of V scaled per head by a power of two:
+    V far above the f16 range (1e5) or far below its normal range (3e-7) gives the same
+    relative accuracy as unit-scale V, against the oracle on the same bf16 inputs; one head
+    mixes a single huge value into unit-scale V (its scale follows the max)."""
     N, d, D, bs = 1000, 64, 64, 64
     w = _wl(N, d, D, bs, std=1.0, seed=41, drift=0.05)
     (h0, _), (d0, _) = _inputs(w, cuda_device)
-    rp, ci = random_csr(w.batch * w.heads, w.n_blocks, 4, seed=43, forced=1)
-    kw = dict(head_dim=d, block_size=bs, scale=w.scale, row_ptr=to_dev(rp, cuda_device), col_idx=to_dev(ci, cuda_device))
-    assert usa.rt_take_device_error() == 0
-    v_big = d0[2].clone()
-    v_big[1, 2, 777, 5] = 1.0e5
-    usa.rt_attn_full_capture(d0[0], d0[1], v_big, **kw)
-    assert usa.rt_take_device_error() == usa.RT_ERR_RANGE
-    assert usa.rt_take_device_error() == 0
-    v_inf = d0[2].clone()
-    v_inf[0, 0, 3, 0] = float("inf")
-    usa.rt_attn_full_capture(d0[0], d0[1], v_inf, **kw)
-    assert usa.rt_take_device_error() == 0
-    out, st = usa.rt_attn_full_capture(*d0, **kw)
+    v = (h0[2].float() * v_scale).to(torch.bfloat16)
+    v[1, 2] = h0[2][1, 2]
+    v[1, 2, 777, 5] = 6.0e4 if v_scale > 1 else 1.0
+    bh = w.batch * w.heads
+    rp, ci = random_csr(bh, w.n_blocks, 4, seed=43, forced=1)
+    out, st = usa.rt_attn_full_capture(d0[0], d0[1], v.to(cuda_device), head_dim=d, block_size=bs, scale=w.scale,
+                                       row_ptr=to_dev(rp, cuda_device), col_idx=to_dev(ci, cuda_device))
     torch.cuda.synchronize()
     assert usa.rt_take_device_error() == 0
-    orc = oracle.full_capture(*h0, d, bs, w.scale, rp, ci)
-    compare_out(out.reshape(-1, D), orc["o"], d, "capture O after a range error")
+    orc = oracle.full_capture(h0[0], h0[1], v, d, bs, w.scale, rp, ci)
+    orc_abs = oracle.full_capture(h0[0], h0[1], v.abs(), d, bs, w.scale, rp, ci)["u"]
+    # outputs compared at unit scale, head by head (the mixed head at its own scale)
+    head_scale = np.full(bh, v_scale)
+    head_scale[1 * w.heads + 2] = 1.0
+    row_scale = np.repeat(head_scale, N)[:, None]
+    got = out.reshape(-1, D).float().cpu().numpy().astype(np.float64) / row_scale
+    compare_out(torch.as_tensor(got), orc["o"] / row_scale, d, f"capture O, V x {v_scale:g}")
+    compare_stats(st, np.arange(bh * N), orc, orc_abs, d, f"capture stats, V x {v_scale:g}")
 
 
 # ------------------------------------------------------------------ maximum size

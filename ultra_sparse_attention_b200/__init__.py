@@ -48,7 +48,6 @@ RT_ERR_INVALID_ARGUMENT = 1
 RT_ERR_UNSUPPORTED = 2
 RT_ERR_CUDA = 3
 RT_ERR_TIMEOUT = 4
-RT_ERR_RANGE = 5
 
 
 class RtError(RuntimeError):

@@ -98,12 +98,30 @@ struct AttnArgs {
   // sparse step: the query blocks of each 128-row tile, int32 [B*H][n_tiles][2]
   // (-1: empty half); null = the neighbouring blocks
   const int32_t* tile_blocks;
+  // capture step: per (batch, head) the bits of max |v|, which fix the power-of-two scale
+  // of the f16 copy of V (see v_scale_exp)
+  const uint32_t* v_amax;
   int N;
   int d;
   int n_blocks;
   int n_heads;       // B*H
   float scale_log2;  // softmax scale * log2(e)
 };
+
+// Power-of-two exponent k of the capture's f16 copy of V for a head whose max |v| has the
+// float bits `amax`: max |v| * 2^k lies in [2^14, 2^15), well inside f16 (max 65504), so
+// every finite bf16 value down to 2^-30 of the head's largest keeps 11 mantissa bits.  A
+// head of zeros or with a non-finite max is not scaled.  k in [-113, 126] keeps 2^k normal.
+__host__ __device__ constexpr int v_scale_exp(uint32_t amax) {
+  return (((amax >> 23) & 0xFFu) == 0xFFu || amax == 0u)
+             ? 0
+             : (14 - (static_cast<int>((amax >> 23) & 0xFFu) - 127) > 126 ? 126
+                                                                         : 14 - (static_cast<int>((amax >> 23) & 0xFFu) - 127));
+}
+
+__device__ __forceinline__ float exp2_int(int k) {  // 2^k for k in [-126, 127]
+  return __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+}
 
 __host__ __device__ constexpr int attn_words(int n_blocks) { return (n_blocks + 31) / 32; }
 __host__ __device__ constexpr int key_tiles(int N) { return (N + kBN - 1) / kBN; }
@@ -846,9 +864,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 // One CTA per 128-row query tile, every key tile in order.  Each key tile's
 // P V goes to O_kept (rows whose query block keeps the tile's block) and/or
 // to U (the other rows).  The PV products take P in f16 with V in f16 (an f16
-// copy of V made by convert_v_f16_kernel before the launch): P keeps 11
-// mantissa bits, a rounding error below 2^-12 of each term of U, in one
-// product per key tile.
+// copy of V made by convert_v_f16_kernel before the launch, scaled per head
+// by a power of two that puts max |v| in [2^14, 2^15), undone exactly in the
+// epilogue): P keeps 11 mantissa bits, a rounding error below 2^-12 of each
+// term of U, in one product per key tile.
 //
 // S is double-buffered in TMEM, so QK^T(j+1) runs while the softmax works on
 // tile j: the MMA warp issues QK^T(j+1) as soon as PV(j-1) -- the last reader
@@ -1143,9 +1162,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     if (ok) ok = warp_wait(&sh.o_full, 0, abort_flag);
     tc_fence_after();
     if (ok) {
-      const float adj = ex2_approx(m_run - m_seen);  // <= 1: refer the cache to the true row max
+      // O and U were accumulated on V * 2^k; 2^-k (exact) takes the head's scale back out.
+      const float unscale = exp2_int(-v_scale_exp(a.v_amax[bh]));
+      const float adjz = ex2_approx(m_run - m_seen);  // <= 1: refer the cache to the true row max
+      const float adj = adjz * unscale;
       const float zsum = zk + zm;
-      const float inv = zsum > 0.f ? 1.f / zsum : 0.f;
+      const float inv = zsum > 0.f ? unscale / zsum : 0.f;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 16) {
         float okv[16], ouv[16];
@@ -1179,10 +1201,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           for (int q4 = 0; q4 < 4; ++q4) ud[q4] = make_float4(uo[4 * q4], uo[4 * q4 + 1], uo[4 * q4 + 2], uo[4 * q4 + 3]);
         }
       }
-      if (valid) {
+      if (valid) {  // the sums carry no V scale
         a.out_m[row_g] = m_seen * kLn2;
-        a.out_zfull[row_g] = (zk + zm) * adj;
-        a.out_zkept[row_g] = zk * adj;
+        a.out_zfull[row_g] = (zk + zm) * adjz;
+        a.out_zkept[row_g] = zk * adjz;
       }
     }
   }
@@ -1196,27 +1218,40 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   }
 }
 
-// f16 copy of V for the capture kernel's PV products, 8 elements per thread and step.  A
-// finite value outside the f16 range (|v| > 65504) records RT_ERR_RANGE in the device
-// status word, so the capture kernel after it does nothing.
-__global__ void __launch_bounds__(256) convert_v_f16_kernel(const uint4* __restrict__ v, uint4* __restrict__ v16,
-                                                            size_t n8) {
+// Per (batch, head) max |v| into amax (float bits, atomic max; zeroed before).  grid (x, B*H).
+__global__ void __launch_bounds__(256) v_absmax_kernel(const uint4* __restrict__ v, size_t per_head8,
+                                                       uint32_t* __restrict__ amax) {
   if (device_status_set()) return;  // an earlier kernel failed
-  bool range = true;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+  const uint4* vh = v + blockIdx.y * per_head8;
+  float m = 0.f;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < per_head8;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const uint4 x = __ldg(v + i);
+    const uint4 x = __ldg(vh + i);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m = fmaxf(m, fmaxf(fabsf(bf16_lo_to_f32(w[k])), fabsf(bf16_hi_to_f32(w[k]))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax + blockIdx.y, __float_as_uint(m));
+}
+
+// f16 copy of V * 2^k (k per head from amax, see v_scale_exp), 8 elements per thread and
+// step.  grid (x, B*H).
+__global__ void __launch_bounds__(256) convert_v_f16_kernel(const uint4* __restrict__ v, uint4* __restrict__ v16,
+                                                            size_t per_head8, const uint32_t* __restrict__ amax) {
+  if (device_status_set()) return;  // an earlier kernel failed
+  const float scale = exp2_int(v_scale_exp(amax[blockIdx.y]));
+  const size_t base = blockIdx.y * per_head8;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < per_head8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint4 x = __ldg(v + base + i);
     const uint32_t w[4] = {x.x, x.y, x.z, x.w};
     uint32_t h[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float a = bf16_lo_to_f32(w[k]), b = bf16_hi_to_f32(w[k]);
-      range = range && !(fabsf(a) > 65504.f && fabsf(a) != INFINITY) && !(fabsf(b) > 65504.f && fabsf(b) != INFINITY);
-      h[k] = pack_f16x2(a, b);
-    }
-    v16[i] = make_uint4(h[0], h[1], h[2], h[3]);
+    for (int k = 0; k < 4; ++k) h[k] = pack_f16x2(bf16_lo_to_f32(w[k]) * scale, bf16_hi_to_f32(w[k]) * scale);
+    v16[base + i] = make_uint4(h[0], h[1], h[2], h[3]);
   }
-  if (!range) record_device_status(RT_ERR_RANGE);
 }
 
 // Failure-detection self test: wait on a barrier nothing completes.

@@ -285,7 +285,6 @@ const char* rt_status_string(rt_status status) {
     case RT_ERR_UNSUPPORTED: return "RT_ERR_UNSUPPORTED: head dim, block size or size outside the supported set";
     case RT_ERR_CUDA: return "RT_ERR_CUDA: a CUDA call or kernel launch failed";
     case RT_ERR_TIMEOUT: return "RT_ERR_TIMEOUT: a kernel wait ran out and the kernel stopped";
-    case RT_ERR_RANGE: return "RT_ERR_RANGE: an input value outside the range the kernels compute in";
   }
   return "unknown rt_status";
 }
@@ -331,22 +330,37 @@ rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void*
     return RT_ERR_INVALID_ARGUMENT;
   if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // The PV products run on f16 P and an f16 copy of V (a transient workspace).
-  const size_t v_elems = static_cast<size_t>(d.bh) * d.N * d.D;
-  void* v16 = nullptr;
-  if (!workspace_alloc(&v16, v_elems * 2, s)) return RT_ERR_CUDA;
+  // The PV products run on f16 P and an f16 copy of V scaled per head by a power of two
+  // (transient workspace: the copy, then the per-head max |v|).
+  const size_t per_head8 = static_cast<size_t>(d.N) * d.D / 8;  // D is a multiple of 16
+  const size_t v16_bytes = static_cast<size_t>(d.bh) * per_head8 * 16;
+  void* ws = nullptr;
+  if (!workspace_alloc(&ws, v16_bytes + static_cast<size_t>(d.bh) * 4, s)) return RT_ERR_CUDA;
+  void* v16 = ws;
+  uint32_t* amax = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + v16_bytes);
   Maps m;
   if (!make_maps(&m, d, q, k, v16, out, rt::kBM, true)) {
-    cudaFreeAsync(v16, s);
+    cudaFreeAsync(ws, s);
     return RT_ERR_CUDA;
   }
-  const size_t n8 = v_elems / 8;  // D is a multiple of 16
-  const unsigned cgrid = static_cast<unsigned>(std::min<size_t>((n8 + 255) / 256, 8 * static_cast<size_t>(sm_count())));
-  rt::convert_v_f16_kernel<<<cgrid, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), n8);
-  st = launch_status();
+  const size_t per_head_blocks = (per_head8 + 255) / 256;
+  const size_t want = (8 * static_cast<size_t>(sm_count()) + d.bh - 1) / d.bh;
+  const dim3 cgrid(static_cast<unsigned>(std::max<size_t>(1, std::min(per_head_blocks, want))),
+                   static_cast<unsigned>(d.bh));
+  st = cudaMemsetAsync(amax, 0, static_cast<size_t>(d.bh) * 4, s) == cudaSuccess ? RT_OK : RT_ERR_CUDA;
+  if (st == RT_OK) {
+    rt::v_absmax_kernel<<<cgrid, 256, 0, s>>>(static_cast<const uint4*>(v), per_head8, amax);
+    st = launch_status();
+  }
+  if (st == RT_OK) {
+    rt::convert_v_f16_kernel<<<cgrid, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16),
+                                                   per_head8, amax);
+    st = launch_status();
+  }
   AttnArgs a{};
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
+  a.v_amax = amax;
   a.out_m = stat_m;
   a.out_zfull = stat_zfull;
   a.out_zkept = stat_zkept;
@@ -358,7 +372,7 @@ rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void*
   a.n_heads = static_cast<int>(d.bh);
   a.scale_log2 = scale * rt::kLog2e;
   if (st == RT_OK) st = dispatch_attention<true>(d, m, a, s);
-  if (cudaFreeAsync(v16, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
+  if (cudaFreeAsync(ws, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
   return st;
 }
 
