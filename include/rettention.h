@@ -60,13 +60,14 @@
 #ifndef RETTENTION_H
 #define RETTENTION_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
 extern "C" {
 #endif
 
-#define RT_ABI_VERSION 4
+#define RT_ABI_VERSION 5
 
 typedef enum rt_status {
     RT_OK = 0,
@@ -139,8 +140,8 @@ rt_status rt_build_block_mask(const rt_shape *shape, const void *q, const void *
  *   out_i    = sum_j exp(s_ij - m_i) * v_j / Z_full_i       (full attention, bf16)
  *
  * The P V products take the probabilities in f16 with an f16 copy of V, made
- * by the call in a transient device workspace of B*H*N*D*2 + B*H*4 bytes from
- * the library's stream-ordered pool: every term of U and out is rounded to 11
+ * by the call in a device workspace of B*H*N*D*2 + B*H*4 bytes (see
+ * rt_workspace_bytes): every term of U and out is rounded to 11
  * mantissa bits of p (a relative error below 2^-12).  The copy is scaled per
  * (batch, head) by the power of two that puts max |v| in [2^14, 2^15) and the
  * scale is taken out exactly afterwards, so any finite V keeps 11 mantissa
@@ -151,11 +152,17 @@ rt_status rt_build_block_mask(const rt_shape *shape, const void *q, const void *
  * out           out, bf16 [B,H,N,D] device.
  * stat_m, stat_zfull, stat_zkept  out, fp32 [B,H,N] device.
  * stat_u        out, fp32 [B,H,N,D] device.
+ * workspace     optional (may be NULL), device, 16-byte aligned, at least the
+ *               capture size rt_workspace_bytes gives (workspace_bytes says
+ *               how large it is; a smaller one is RT_ERR_INVALID_ARGUMENT).
+ *               Used only while the call's work runs on `stream`.  NULL takes
+ *               a transient buffer from the library's stream-ordered pool.
  */
 rt_status rt_attn_full_capture(const rt_shape *shape, const void *q, const void *k, const void *v,
                                float scale, const int32_t *row_ptr, const int32_t *col_idx,
                                void *out, float *stat_m, float *stat_zfull, float *stat_zkept,
-                               float *stat_u, rt_stream_t stream);
+                               float *stat_u, void *workspace, size_t workspace_bytes,
+                               rt_stream_t stream);
 
 /*
  * rt_attn_sparse_reshape -- block-sparse attention with the statistical reshape.
@@ -219,14 +226,28 @@ rt_status rt_attn_sparse_reshape(const rt_shape *shape, const void *q, const voi
  *
  * row_ptr, col_idx  the CSR (as for rt_attn_sparse_reshape).
  * tile_blocks   out, int32 [B*H][ceil(N / 128)][2] device.
- * Malformed CSR contents give a valid table of unspecified quality.  At block
- * size 64 takes a transient device workspace of B*H*n_blocks*16 bytes (the
- * candidates of step 1) from the library's stream-ordered pool, as
- * rt_build_block_mask does.
+ * workspace     optional (may be NULL), device, 16-byte aligned: at block size
+ *               64 the candidates of step 1 need B*H*n_blocks*16 bytes (the
+ *               pairing size rt_workspace_bytes gives; a smaller workspace is
+ *               RT_ERR_INVALID_ARGUMENT).  NULL takes a transient buffer from
+ *               the library's stream-ordered pool.
+ * Malformed CSR contents give a valid table of unspecified quality.
  */
 rt_status rt_pair_query_blocks(const rt_shape *shape, const int32_t *row_ptr,
-                               const int32_t *col_idx, int32_t *tile_blocks,
-                               rt_stream_t stream);
+                               const int32_t *col_idx, int32_t *tile_blocks, void *workspace,
+                               size_t workspace_bytes, rt_stream_t stream);
+
+/*
+ * rt_workspace_bytes -- device workspace sizes for a shape.
+ *
+ * *capture_bytes (if not NULL) receives what rt_attn_full_capture needs,
+ * *pairing_bytes (if not NULL) what rt_pair_query_blocks needs (0 at block
+ * size 128).  With these passed in, rt_build_block_mask_static,
+ * rt_pair_query_blocks, rt_attn_full_capture and rt_attn_sparse_reshape run a
+ * whole denoising cycle without the library allocating device memory.
+ * Validates the shape like the other calls; launches nothing.
+ */
+rt_status rt_workspace_bytes(const rt_shape *shape, size_t *capture_bytes, size_t *pairing_bytes);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *rt_status_string(rt_status status);

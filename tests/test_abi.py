@@ -32,7 +32,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    assert usa.rt_abi_version() == 4
+    assert usa.rt_abi_version() == 5
     for code in range(5):
         s = usa.rt_status_string(code)
         assert s.startswith("RT_")
@@ -54,13 +54,14 @@ def _sparse(lib, shape, stats=(None, None, None, None), out=A16, scale=0.125, ti
     return lib.rt_attn_sparse_reshape(ctypes.byref(shape), A16, A16, A16, scale, A16, A16, tiles, *stats, out, None)
 
 
-def _pair(lib, shape, rp=A16, ci=A16, tiles=A16):
-    return lib.rt_pair_query_blocks(ctypes.byref(shape) if shape is not None else None, rp, ci, tiles, None)
-
-
-def _capture(lib, shape, u=A16, m=A16):
-    return lib.rt_attn_full_capture(ctypes.byref(shape), A16, A16, A16, 0.125, A16, A16, A16, m, A16, A16, u,
+def _pair(lib, shape, rp=A16, ci=A16, tiles=A16, ws=None, ws_bytes=0):
+    return lib.rt_pair_query_blocks(ctypes.byref(shape) if shape is not None else None, rp, ci, tiles, ws, ws_bytes,
                                     None)
+
+
+def _capture(lib, shape, u=A16, m=A16, ws=None, ws_bytes=0):
+    return lib.rt_attn_full_capture(ctypes.byref(shape), A16, A16, A16, 0.125, A16, A16, A16, m, A16, A16, u,
+                                    ws, ws_bytes, None)
 
 
 def test_mask_argument_validation():
@@ -125,3 +126,21 @@ def test_source_hash_covers_code_not_comments():
     edited = src.replace("// note", "// another note\n// and a line more").replace("  int", "\n\nint")
     assert b.code_text(edited) == b.code_text(src)
     assert b.code_text(src.replace("a = 1", "a = 2")) != b.code_text(src)
+
+
+def test_workspace_sizes_and_validation():
+    """rt_workspace_bytes gives the capture's f16 copy of V plus its per-head maxima and the
+    pairing's candidates; a caller workspace that is too small or misaligned is refused
+    before any CUDA call."""
+    cap, pair = usa.rt_workspace_bytes(2, 3, 1000, head_dim=72, head_dim_padded=80, block_size=64)
+    assert cap == 2 * 3 * 1000 * 80 * 2 + 2 * 3 * 4
+    assert pair == 2 * 3 * 16 * 16  # 16 blocks of 64, eight int16 candidates each
+    assert usa.rt_workspace_bytes(2, 3, 1000, head_dim=72, head_dim_padded=80, block_size=128)[1] == 0
+    with pytest.raises(usa.RtError):
+        usa.rt_workspace_bytes(2, 3, 1000, head_dim=72, head_dim_padded=96, block_size=64)
+    lib = usa.load_library()
+    ok = RtShape(2, 3, 1000, 72, 80, 64)
+    assert _capture(lib, ok, ws=A16, ws_bytes=cap - 1) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _capture(lib, ok, ws=A4, ws_bytes=cap) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _pair(lib, ok, ws=A16, ws_bytes=pair - 1) == usa.RT_ERR_INVALID_ARGUMENT
+    assert _pair(lib, ok, ws=MIS, ws_bytes=pair) == usa.RT_ERR_INVALID_ARGUMENT

@@ -79,3 +79,38 @@ def test_static_mask_rejects_shapes_beyond_the_workspace(cuda_device):
     q = torch.zeros(1, 64, 17776, 64, dtype=torch.bfloat16, device=cuda_device)
     with pytest.raises(ValueError):
         usa.rt_build_block_mask_static(q, q, head_dim=64, block_size=64, scale=0.125, keep_blocks=9)
+
+
+@pytest.mark.parametrize("bs,D,d", [(64, 64, 64), (128, 80, 72)])
+def test_cycle_with_caller_workspaces_equals_pool_cycle(cuda_device, bs, D, d):
+    """A whole denoising cycle without the library allocating: the static mask, the pairing
+    and the capture with caller workspaces (sized by rt_workspace_bytes, filled with garbage
+    first), then the sparse step; every output equals the pool-allocating cycle bit for bit."""
+    from ultra_sparse_attention_b200.workloads import Workload, denoising_inputs
+    from fractions import Fraction
+    w = Workload(name="case", batch=2, heads=3, seq_len=1000, head_dim=d, head_dim_padded=D, block_size=bs,
+                 keep=(Fraction(1, 4),), forced_prefix_tokens=70, steps=2, capture_every=2, drift_sigma=0.05,
+                 kind="iid", iid_std=1.0, seed=5)
+    steps = list(denoising_inputs(w, 2))
+    d0 = [x.to(cuda_device) for x in steps[0][1:]]
+    d1 = [x.to(cuda_device) for x in steps[1][1:]]
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale)
+    keep = w.keep_blocks()
+    cap_b, pair_b = usa.rt_workspace_bytes(2, 3, 1000, head_dim=d, head_dim_padded=D, block_size=bs)
+    ws_cap = torch.randint(0, 255, (cap_b,), dtype=torch.uint8, device=cuda_device)
+    ws_pair = torch.randint(0, 255, (max(pair_b, 16),), dtype=torch.uint8, device=cuda_device)
+
+    def cycle(static):
+        mask = usa.rt_build_block_mask_static if static else usa.rt_build_block_mask
+        rp, ci = mask(d0[0], d0[1], keep_blocks=keep, forced_prefix_tokens=w.forced_prefix_tokens, **kw)
+        tiles = usa.rt_pair_query_blocks(d0[0], rp, ci, head_dim=d, block_size=bs,
+                                         workspace=ws_pair if static else None)
+        out0, st = usa.rt_attn_full_capture(*d0, row_ptr=rp, col_idx=ci, workspace=ws_cap if static else None, **kw)
+        out1 = usa.rt_attn_sparse_reshape(*d1, row_ptr=rp, col_idx=ci, stats=st, tile_blocks=tiles, **kw)
+        return [rp, ci, tiles, out0, st.m, st.zfull, st.zkept, st.u, out1]
+
+    got, want = cycle(True), cycle(False)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    for g, x in zip(got, want):
+        assert torch.equal(g.view(torch.uint8), x.view(torch.uint8))

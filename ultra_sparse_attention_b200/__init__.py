@@ -32,6 +32,7 @@ __all__ = [
     "rt_attn_full_capture",
     "rt_attn_sparse_reshape",
     "rt_pair_query_blocks",
+    "rt_workspace_bytes",
     "rt_status_string",
     "rt_abi_version",
     "rt_take_device_error",
@@ -82,9 +83,11 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
             vp, i32, f32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_int64
             shp = ctypes.POINTER(RtShape)
             lib.rt_build_block_mask.argtypes = [shp, vp, vp, f32, i32, i32, vp, vp, vp, vp]
-            lib.rt_attn_full_capture.argtypes = [shp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp]
+            sz = ctypes.c_size_t
+            lib.rt_attn_full_capture.argtypes = [shp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
             lib.rt_attn_sparse_reshape.argtypes = [shp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
-            lib.rt_pair_query_blocks.argtypes = [shp, vp, vp, vp, vp]
+            lib.rt_pair_query_blocks.argtypes = [shp, vp, vp, vp, vp, sz, vp]
+            lib.rt_workspace_bytes.argtypes = [shp, ctypes.POINTER(sz), ctypes.POINTER(sz)]
             lib.rt_status_string.argtypes = [ctypes.c_int]
             lib.rt_status_string.restype = ctypes.c_char_p
             lib.rt_abi_version.argtypes = []
@@ -94,7 +97,8 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.rt_build_block_mask_static.argtypes = [shp, vp, vp, f32, i32, i32, vp, vp, vp, vp]
             lib.rt_build_block_mask_static.restype = ctypes.c_int
             for fn in ("rt_build_block_mask", "rt_attn_full_capture", "rt_attn_sparse_reshape",
-                       "rt_pair_query_blocks", "rt_take_device_error", "rt_selftest_wait_timeout"):
+                       "rt_pair_query_blocks", "rt_workspace_bytes", "rt_take_device_error",
+                       "rt_selftest_wait_timeout"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -120,6 +124,10 @@ class Stats:
 
 def _ptr(t: torch.Tensor | None):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _nbytes(t: torch.Tensor | None) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
 
 
 def _stream_handle(device: torch.device, stream) -> ctypes.c_void_p:
@@ -206,8 +214,12 @@ def rt_build_block_mask(q: torch.Tensor, k: torch.Tensor, *, head_dim: int, bloc
 
 def rt_attn_full_capture(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, head_dim: int, block_size: int,
                          scale: float, row_ptr: torch.Tensor, col_idx: torch.Tensor,
-                         out: torch.Tensor | None = None, stats: Stats | None = None, stream=None):
-    """Full attention at a capture step plus the statistics cache.  Returns (out, stats)."""
+                         out: torch.Tensor | None = None, stats: Stats | None = None,
+                         workspace: torch.Tensor | None = None, stream=None):
+    """Full attention at a capture step plus the statistics cache.  Returns (out, stats).
+
+    ``workspace`` (uint8, device, at least rt_workspace_bytes(...)[0] bytes) keeps the
+    library from taking a transient buffer from its pool."""
     name = "rt_attn_full_capture"
     dims = _check_qkv(name, q, k, v)
     B, H, N, D = dims
@@ -223,12 +235,14 @@ def rt_attn_full_capture(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, h
     _check_stats(name, stats, dims, dev)
     _check_buf(name, "row_ptr", row_ptr, torch.int32, dev)
     _check_buf(name, "col_idx", col_idx, torch.int32, dev)
+    if workspace is not None:
+        _check_buf(name, "workspace", workspace, torch.uint8, dev)
     shape = _shape(dims, head_dim, block_size)
     with torch.cuda.device(dev):
         _call(load_library().rt_attn_full_capture(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale),
                                                   _ptr(row_ptr), _ptr(col_idx), _ptr(out), _ptr(stats.m),
                                                   _ptr(stats.zfull), _ptr(stats.zkept), _ptr(stats.u),
-                                                  _stream_handle(dev, stream)),
+                                                  _ptr(workspace), _nbytes(workspace), _stream_handle(dev, stream)),
               name)
     return out, stats
 
@@ -270,10 +284,13 @@ def _tile_table_shape(dims) -> tuple[int, int, int]:
 
 
 def rt_pair_query_blocks(q: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor, *, head_dim: int,
-                         block_size: int, tile_blocks: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                         block_size: int, tile_blocks: torch.Tensor | None = None,
+                         workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Group each head's query blocks into the sparse kernel's 128-row tiles (``q`` gives the shape).
 
-    Returns int32 [B*H, ceil(N/128), 2]: the query blocks of each tile, -1 for an empty half."""
+    Returns int32 [B*H, ceil(N/128), 2]: the query blocks of each tile, -1 for an empty half.
+    ``workspace`` (uint8, device, at least rt_workspace_bytes(...)[1] bytes) keeps the
+    library from taking a transient buffer from its pool."""
     name = "rt_pair_query_blocks"
     dims = _check_qkv(name, q)
     dev = q.device
@@ -282,12 +299,25 @@ def rt_pair_query_blocks(q: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.
     _check_buf(name, "tile_blocks", tile_blocks, torch.int32, dev, shape=_tile_table_shape(dims))
     _check_buf(name, "row_ptr", row_ptr, torch.int32, dev)
     _check_buf(name, "col_idx", col_idx, torch.int32, dev)
+    if workspace is not None:
+        _check_buf(name, "workspace", workspace, torch.uint8, dev)
     shape = _shape(dims, head_dim, block_size)
     with torch.cuda.device(dev):
         _call(load_library().rt_pair_query_blocks(ctypes.byref(shape), _ptr(row_ptr), _ptr(col_idx),
-                                                  _ptr(tile_blocks), _stream_handle(dev, stream)),
+                                                  _ptr(tile_blocks), _ptr(workspace), _nbytes(workspace),
+                                                  _stream_handle(dev, stream)),
               name)
     return tile_blocks
+
+
+def rt_workspace_bytes(batch: int, heads: int, seq_len: int, *, head_dim: int, head_dim_padded: int,
+                       block_size: int) -> tuple[int, int]:
+    """Device workspace bytes of (rt_attn_full_capture, rt_pair_query_blocks) for a shape."""
+    shape = RtShape(batch, heads, seq_len, head_dim, head_dim_padded, block_size)
+    cap, pair = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _call(load_library().rt_workspace_bytes(ctypes.byref(shape), ctypes.byref(cap), ctypes.byref(pair)),
+          "rt_workspace_bytes")
+    return int(cap.value), int(pair.value)
 
 
 def rt_take_device_error() -> int:

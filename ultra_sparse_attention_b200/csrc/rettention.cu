@@ -273,6 +273,16 @@ rt_status static_pool_address(float** out) {
   return RT_OK;
 }
 
+// Workspace of rt_attn_full_capture: the f16 copy of V, then the per-head max |v|.
+size_t capture_workspace_bytes(const Dims& d) {
+  return static_cast<size_t>(d.bh) * d.N * d.D * 2 + static_cast<size_t>(d.bh) * 4;
+}
+
+// Workspace of rt_pair_query_blocks: the candidates of step 1 (none at block size 128).
+size_t pairing_workspace_bytes(const Dims& d) {
+  return d.bs == 64 ? static_cast<size_t>(d.bh) * d.n_blocks * rt::kPairCands * 2 : 0;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -316,9 +326,19 @@ rt_status rt_build_block_mask(const rt_shape* shape, const void* q, const void* 
   return st;
 }
 
+rt_status rt_workspace_bytes(const rt_shape* shape, size_t* capture_bytes, size_t* pairing_bytes) {
+  Dims d;
+  rt_status st = check_shape(shape, &d);
+  if (st != RT_OK) return st;
+  if (capture_bytes) *capture_bytes = capture_workspace_bytes(d);
+  if (pairing_bytes) *pairing_bytes = pairing_workspace_bytes(d);
+  return RT_OK;
+}
+
 rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void* k, const void* v, float scale,
                                const int32_t* row_ptr, const int32_t* col_idx, void* out, float* stat_m,
-                               float* stat_zfull, float* stat_zkept, float* stat_u, rt_stream_t stream) {
+                               float* stat_zfull, float* stat_zkept, float* stat_u, void* workspace,
+                               size_t workspace_bytes, rt_stream_t stream) {
   Dims d;
   rt_status st = check_shape(shape, &d);
   if (st != RT_OK) return st;
@@ -329,18 +349,21 @@ rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void*
       !aligned(stat_zkept, 4))
     return RT_ERR_INVALID_ARGUMENT;
   if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
+  if (workspace && (!aligned(workspace, 16) || workspace_bytes < capture_workspace_bytes(d)))
+    return RT_ERR_INVALID_ARGUMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // The PV products run on f16 P and an f16 copy of V scaled per head by a power of two
-  // (transient workspace: the copy, then the per-head max |v|).
+  // (workspace: the copy, then the per-head max |v|; the caller's, or from the pool).
   const size_t per_head8 = static_cast<size_t>(d.N) * d.D / 8;  // D is a multiple of 16
   const size_t v16_bytes = static_cast<size_t>(d.bh) * per_head8 * 16;
-  void* ws = nullptr;
-  if (!workspace_alloc(&ws, v16_bytes + static_cast<size_t>(d.bh) * 4, s)) return RT_ERR_CUDA;
+  const bool own = workspace == nullptr;
+  void* ws = workspace;
+  if (own && !workspace_alloc(&ws, capture_workspace_bytes(d), s)) return RT_ERR_CUDA;
   void* v16 = ws;
   uint32_t* amax = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + v16_bytes);
   Maps m;
   if (!make_maps(&m, d, q, k, v16, out, rt::kBM, true)) {
-    cudaFreeAsync(ws, s);
+    if (own) cudaFreeAsync(ws, s);
     return RT_ERR_CUDA;
   }
   const size_t per_head_blocks = (per_head8 + 255) / 256;
@@ -372,7 +395,7 @@ rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void*
   a.n_heads = static_cast<int>(d.bh);
   a.scale_log2 = scale * rt::kLog2e;
   if (st == RT_OK) st = dispatch_attention<true>(d, m, a, s);
-  if (cudaFreeAsync(ws, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
+  if (own && cudaFreeAsync(ws, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
   return st;
 }
 
@@ -411,12 +434,14 @@ rt_status rt_attn_sparse_reshape(const rt_shape* shape, const void* q, const voi
 }
 
 rt_status rt_pair_query_blocks(const rt_shape* shape, const int32_t* row_ptr, const int32_t* col_idx,
-                               int32_t* tile_blocks, rt_stream_t stream) {
+                               int32_t* tile_blocks, void* workspace, size_t workspace_bytes, rt_stream_t stream) {
   Dims d;
   rt_status st = check_shape(shape, &d);
   if (st != RT_OK) return st;
   if (!row_ptr || !col_idx || !tile_blocks) return RT_ERR_INVALID_ARGUMENT;
   if (!aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(tile_blocks, 4)) return RT_ERR_INVALID_ARGUMENT;
+  if (workspace && (!aligned(workspace, 16) || workspace_bytes < pairing_workspace_bytes(d)))
+    return RT_ERR_INVALID_ARGUMENT;
   const int nb = static_cast<int>(d.n_blocks);
   const int n_tiles = rt::query_tiles(static_cast<int>(d.N));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -425,7 +450,8 @@ rt_status rt_pair_query_blocks(const rt_shape* shape, const int32_t* row_ptr, co
                                                                                  static_cast<int>(d.bs), tile_blocks);
     return launch_status();
   }
-  // Candidates of every query block go through a transient workspace (int16 [B*H][n_blocks][8]).
+  // Candidates of every query block go through a workspace (int16 [B*H][n_blocks][8]): the
+  // caller's, or from the pool.
   const size_t cand_smem = rt::pair_candidates_smem_bytes(nb), match_smem = rt::pair_match_smem_bytes(nb);
   // Block i's kept-set bitmap lives in registers, in the smallest of these word counts that holds it.
   const int words = (nb + 31) / 32;
@@ -440,9 +466,9 @@ rt_status rt_pair_query_blocks(const rt_shape* shape, const int32_t* row_ptr, co
       cudaFuncSetAttribute(rt::pair_match_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(match_smem)) != cudaSuccess)
     return RT_ERR_CUDA;
-  int16_t* cand = nullptr;
-  if (!workspace_alloc(reinterpret_cast<void**>(&cand), static_cast<size_t>(d.bh) * nb * rt::kPairCands * 2, s))
-    return RT_ERR_CUDA;
+  const bool own = workspace == nullptr;
+  int16_t* cand = static_cast<int16_t*>(workspace);
+  if (own && !workspace_alloc(reinterpret_cast<void**>(&cand), pairing_workspace_bytes(d), s)) return RT_ERR_CUDA;
   dim3 grid(static_cast<unsigned>((nb + rt::kCandBlocks - 1) / rt::kCandBlocks), static_cast<unsigned>(d.bh));
   cand_kernel<<<grid, rt::kPairThreads, cand_smem, s>>>(row_ptr, col_idx, nb, cand);
   st = launch_status();
@@ -451,7 +477,7 @@ rt_status rt_pair_query_blocks(const rt_shape* shape, const int32_t* row_ptr, co
                                                                                           tile_blocks);
     st = launch_status();
   }
-  if (cudaFreeAsync(cand, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
+  if (own && cudaFreeAsync(cand, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
   return st;
 }
 
