@@ -93,10 +93,9 @@ typedef struct rt_shape {
 /*
  * rt_build_block_mask -- choose the key blocks each query block keeps.
  *
- * The project page's Abstract describes sparse attention as including "only a
- * subset of tokens or patches", down to 3.1% of them; it does not say how the
- * subset is chosen.  This call uses block mean pooling and a per-query-block
- * top-k:
+ * The project page's Abstract has the sparse step attend to a small subset of
+ * the tokens, down to 3.1% of them; it does not say how the subset is chosen.
+ * This call uses block mean pooling and a per-query-block top-k:
  *   pooled_q[b,h,qb] = mean of q over the real tokens of query block qb
  *                      (logical columns only); pooled_k likewise;
  *   score[qb,kb]     = scale * <pooled_q[qb], pooled_k[kb]>;
@@ -127,8 +126,8 @@ rt_status rt_build_block_mask(const rt_shape *shape, const void *q, const void *
 /*
  * rt_attn_full_capture -- full attention at a capture step, and the cache.
  *
- * The teaser reshapes sparse attention "with cached statistics across
- * denoising steps"; the mechanism highlight names the cached quantities: the
+ * The teaser corrects sparse attention with statistics kept from an earlier
+ * denoising step; the mechanism highlight names the cached quantities: the
  * stable ratio between sparse and full softmax denominators and the residual
  * contribution of the masked-out tokens.  For every query row i, with
  * s_ij = scale * q_i . k_j over all keys j < N and K(i) the keys of the blocks
@@ -141,8 +140,12 @@ rt_status rt_build_block_mask(const rt_shape *shape, const void *q, const void *
  *
  * The P V products take the probabilities in f16 with an f16 copy of V, made
  * by the call in a device workspace of B*H*N*D*2 + B*H*4 bytes (see
- * rt_workspace_bytes): every term of U and out is rounded to 11
- * mantissa bits of p (a relative error below 2^-12).  The copy is scaled per
+ * rt_workspace_bytes).  The kept and the masked keys of a row are summed as
+ * two separate online softmaxes, each against a reference of its own, and p
+ * enters f16 as p * 2^7 with p <= 2^8: every term of U down to 2^-21 of the
+ * row's largest masked term keeps 11 mantissa bits (a relative error below
+ * 2^-12), smaller ones an absolute error below 2^-32 of that term, however
+ * far the row's maximum lies above its masked scores.  The copy is scaled per
  * (batch, head) by the power of two that puts max |v| in [2^14, 2^15) and the
  * scale is taken out exactly afterwards, so any finite V keeps 11 mantissa
  * bits down to 2^-30 of its head's largest |v|.
@@ -294,7 +297,14 @@ rt_status rt_selftest_wait_timeout(int64_t timeout_ns, rt_stream_t stream);
  *
  * The first call on a device looks up the workspace's device address on that
  * device (with the device current); make that first call before capturing
- * the stream into a CUDA graph.  All calls on a device share the one
+ * the stream into a CUDA graph.  The address is remembered per CUDA context:
+ * after cudaDeviceReset (a new primary context, the module loaded again at a
+ * new address) the next call looks it up again.  The library's first call of
+ * any kind on a device loads its module there (under CUDA's lazy loading),
+ * and that load is what places the 8 MiB array and the kernels in device
+ * memory; a caller whose memory budget is fixed later, or who must never see
+ * a call allocate, should make one call (this one, or rt_workspace_bytes
+ * followed by this one) at start-up.  All calls on a device share the one
  * workspace and it keeps the last call's contents; nothing in it needs to
  * start at zero (every call overwrites what it reads).  Calls that overlap on
  * the GPU (different streams, or different host threads, without ordering

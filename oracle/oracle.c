@@ -7,11 +7,12 @@
  *
  * What it follows (Re-ttention: Ultra Sparse Visual Generation via Attention
  * Statistical Reshape, project page):
- *   - teaser: sparse attention is reshaped "with cached statistics across
- *     denoising steps" so that it recovers the full attention distribution;
+ *   - teaser: sparse attention is corrected with statistics kept from an
+ *     earlier denoising step, so that it recovers the full attention
+ *     distribution;
  *   - Abstract: only a subset of tokens enters the sparse step, and the
- *     reshape corrects the "probabilistic normalization shift" using the
- *     prior softmax distribution history;
+ *     reshape undoes the shift that normalising over that subset causes,
+ *     using the softmax statistics of an earlier step;
  *   - mechanism highlight: the full/sparse softmax-denominator ratio is reused
  *     and the residual contribution of masked-out tokens is cached.
  * The pages give no formula, mask rule or precision.  The readings taken here

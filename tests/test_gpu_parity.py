@@ -465,6 +465,75 @@ def test_capture_with_large_and_tiny_v(cuda_device, v_scale):
     compare_stats(st, np.arange(bh * N), orc, orc_abs, d, f"capture stats, V x {v_scale:g}")
 
 
+# ------------------------------------------------------------------ sharply peaked rows
+def _csr_with_block(bh, nb, keep, seed, block):
+    """Random kept sets that all contain `block` (sorted): int32 row_ptr, col_idx."""
+    rng = np.random.default_rng(seed)
+    others = np.array([b for b in range(nb) if b != block])
+    sets = [sorted({block} | set(int(x) for x in rng.choice(others, size=keep - 1, replace=False)))
+            for _ in range(bh * nb)]
+    row_ptr = np.array([0] + list(np.cumsum([len(s) for s in sets])), np.int32)
+    col_idx = np.array([kb for s in sets for kb in s], np.int32)
+    return row_ptr, col_idx
+
+
+def _capture_vs_oracle(cuda_device, h, d, bs, scale, rp, ci, what):
+    q, k, v = (x.to(cuda_device) for x in h)
+    out, st = usa.rt_attn_full_capture(q, k, v, head_dim=d, block_size=bs, scale=scale,
+                                       row_ptr=to_dev(rp, cuda_device), col_idx=to_dev(ci, cuda_device))
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    orc = oracle.full_capture(*h, d, bs, scale, rp, ci)
+    orc_abs = oracle.full_capture(h[0], h[1], h[2].abs(), d, bs, scale, rp, ci)["u"]
+    D = q.shape[-1]
+    bh, N = q.shape[0] * q.shape[1], q.shape[2]
+    compare_out(out.reshape(-1, D), orc["o"], d, f"{what}: capture O")
+    compare_stats(st, np.arange(bh * N), orc, orc_abs, d, f"{what}: capture stats")
+
+
+@pytest.mark.parametrize("N,d,D,bs", [(1000, 64, 64, 64), (1000, 72, 80, 64), (896, 64, 64, 128),
+                                      (1000, 128, 128, 64)])
+@pytest.mark.parametrize("gain", [3.0, 5.0])
+def test_capture_sharp_scores(cuda_device, N, d, D, bs, gain):
+    """Q scaled by 3 and 5: scores spread over tens of nats, so most terms of U and of the
+    kept sum lie many binades below the row's largest term; statistics and output must
+    still meet the tolerances against the oracle on the same bf16 inputs."""
+    w = _wl(N, d, D, bs, std=1.2, seed=5 * N + d + int(gain))
+    (h0, _), _ = _inputs(w, cuda_device)
+    q = (h0[0].float() * gain).to(torch.bfloat16)
+    bh = w.batch * w.heads
+    rp, ci = random_csr(bh, w.n_blocks, max(2, w.n_blocks // 4), seed=N + int(gain), forced=1)
+    _capture_vs_oracle(cuda_device, (q, h0[1], h0[2]), d, bs, w.scale, rp, ci, f"Q x {gain:g}")
+
+
+@pytest.mark.parametrize("gap", [10.0, 14.0, 16.0, 18.0, 22.0, 30.0])
+@pytest.mark.parametrize("N,d,D,bs,peak", [(2000, 64, 64, 64, 0), (2000, 64, 64, 64, 1500), (2000, 72, 80, 128, 1100),
+                                           (2000, 128, 128, 64, 700)])
+def test_capture_peaked_rows(cuda_device, N, d, D, bs, peak, gap):
+    """Every row's maximum sits on one key (token `peak`, in a block that every query block
+    keeps) about `gap` nats above all other keys, the masked ones among them: U is then a
+    sum of many terms each near e^-gap of the row's largest, whose total still decides the
+    tolerance.  Q shares a direction u; the peak key is c*u, the others small noise."""
+    g = torch.Generator().manual_seed(int(gap * 10) + N + peak)
+    B, H = 1, 2
+    scale = 1.0 / np.sqrt(d)
+    u = torch.randn(d, generator=g)
+    q = u + 0.3 * torch.randn(B, H, N, d, generator=g)
+    k = 0.5 * torch.randn(B, H, N, d, generator=g)
+    c = gap / (scale * float(u @ u))
+    k[:, :, peak] = c * u
+    v = torch.randn(B, H, N, d, generator=g)
+
+    def pad(x):
+        out = torch.zeros(B, H, N, D)
+        out[..., :d] = x
+        return out.to(torch.bfloat16)
+
+    nb = -(-N // bs)
+    rp, ci = _csr_with_block(B * H, nb, max(2, nb // 4), seed=N + peak, block=peak // bs)
+    _capture_vs_oracle(cuda_device, (pad(q), pad(k), pad(v)), d, bs, scale, rp, ci, f"peak gap {gap:g} nats")
+
+
 # ------------------------------------------------------------------ maximum size
 def test_cycle_at_the_block_limit(cuda_device):
     """One mask + capture + sparse cycle at the largest supported block count (2048 blocks

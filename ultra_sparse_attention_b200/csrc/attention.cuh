@@ -52,6 +52,7 @@ constexpr float kRescaleUp = 8.f;    // log2 units
 constexpr float kRescaleDown = 64.f; // log2 units
 constexpr float kSumUp = 0x1p8f;      // 2^kRescaleUp
 constexpr float kSumDown = 0x1p-64f;  // 2^-kRescaleDown
+constexpr float kPBias = 7.f;         // capture: f16 P carries p * 2^7 (p <= 2^8, so <= 2^15)
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 
 // Tile byte sizes for head dim D (bf16 Q/K/V tiles).  A tile is its 64-column
@@ -866,8 +867,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 // to U (the other rows).  The PV products take P in f16 with V in f16 (an f16
 // copy of V made by convert_v_f16_kernel before the launch, scaled per head
 // by a power of two that puts max |v| in [2^14, 2^15), undone exactly in the
-// epilogue): P keeps 11 mantissa bits, a rounding error below 2^-12 of each
-// term of U, in one product per key tile.
+// epilogue), in one product per key tile.  The kept and the masked keys of a
+// row are two online softmaxes with references of their own, and P enters f16
+// as p * 2^7 (p <= 2^8 under the lazy reference, so P <= 2^15): a masked term
+// down to 2^-21 of the row's largest masked term keeps 11 mantissa bits (a
+// rounding error below 2^-12), a smaller one an absolute error below 2^-32 of
+// it, wherever the row's maximum lies.
 //
 // S is double-buffered in TMEM, so QK^T(j+1) runs while the softmax works on
 // tile j: the MMA warp issues QK^T(j+1) as soon as PV(j-1) -- the last reader
@@ -1082,7 +1087,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const size_t row_g = static_cast<size_t>(bh) * a.N + (valid ? i : 0);
     const float C = a.scale_log2;
     const uint32_t* my_bm = bitmaps + (grp < nqb_here ? grp : 0) * words;
-    float m_run = -INFINITY, m_seen = -INFINITY, zk = 0.f, zm = 0.f;
+    // The kept keys (O_kept, Z_kept) and the masked keys (U, the masked sum) are two online
+    // softmaxes with references of their own (log2 units): each set's p stays within 2^8 of
+    // its own largest term, so the f16 P of the masked rows keeps its precision even when the
+    // row's maximum sits in a kept block far above every masked score.
+    float m_k = -INFINITY, m_u = -INFINITY;        // lazy references
+    float seen_k = -INFINITY, seen_u = -INFINITY;  // largest score seen in each set
+    float zk = 0.f, zm = 0.f;                      // sums of the biased p of each set
     bool ok = true;
     int mixed = 0;  // mixed key tiles so far
     for (int j = 0; j < Tn; ++j) {
@@ -1095,27 +1106,34 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       float s[64];
       tmem_ld64(sbuf, s);
       mask_tail(s, j * kBN, a.N);
-      m_seen = fmaxf(m_seen, row_max64(s) * C);
-      float ref = m_run;
+      const float prev = kept ? m_k : m_u;
+      const float seen = fmaxf(kept ? seen_k : seen_u, row_max64(s) * C);
+      float ref = prev;
       bool need = false;
-      if (m_run == -INFINITY) ref = m_seen;
-      else if (m_seen > m_run + kRescaleUp) { need = true; ref = m_seen; }
+      if (prev == -INFINITY) ref = seen;
+      else if (seen > prev + kRescaleUp) { need = true; ref = seen; }
       if (__any_sync(0xffffffffu, need)) {
         // PV(j-1) done: its commit also freed the K/V stage of tile j-1.
         if (j > 0 && !warp_wait(&sh.kv_empty[(j - 1) % NS], ((j - 1) / NS) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const float f = need ? ex2_approx(m_run - ref) : 1.f;
-        tmem_row_scale<D>(tmem + lane_off + L::kOKCol, f);
-        tmem_row_scale<D>(tmem + lane_off + L::kOUCol, f);
-        zk *= f;
-        zm *= f;
+        const float f = need ? ex2_approx(prev - ref) : 1.f;
+        tmem_row_scale<D>(tmem + lane_off + (kept ? L::kOKCol : L::kOUCol), f);  // warp-uniform choice
+        if (kept) zk *= f;
+        else zm *= f;
       }
-      m_run = ref;
-      // p = 2^(s*C - m'), two lanes of f32x2 arithmetic at a time; s now holds p.
+      if (kept) {
+        m_k = ref;
+        seen_k = seen;
+      } else {
+        m_u = ref;
+        seen_u = seen;
+      }
+      const float m_run = ref;
+      // p = 2^(s*C - m' + kPBias), two lanes of f32x2 arithmetic at a time; s now holds p.
       uint32_t pk[32];
       float zt;
       {
-        const uint64_t C2 = f2_pack(C, C), nref = f2_pack(-m_run, -m_run);
+        const uint64_t C2 = f2_pack(C, C), nref = f2_pack(kPBias - m_run, kPBias - m_run);
         uint64_t zz = f2_pack(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
@@ -1164,10 +1182,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     if (ok) {
       // O and U were accumulated on V * 2^k; 2^-k (exact) takes the head's scale back out.
       const float unscale = exp2_int(-v_scale_exp(a.v_amax[bh]));
-      const float adjz = ex2_approx(m_run - m_seen);  // <= 1: refer the cache to the true row max
-      const float adj = adjz * unscale;
-      const float zsum = zk + zm;
-      const float inv = zsum > 0.f ? unscale / zsum : 0.f;
+      // Refer both sets to the true row max M and take the bias out (exact powers of two
+      // apart from ex2's rounding; a set with no term has reference -inf and weight 0).
+      const float M = fmaxf(seen_k, seen_u);
+      const float adjk = ex2_approx(m_k - kPBias - M);
+      const float adju = ex2_approx(m_u - kPBias - M);
+      const float zkept = zk * adjk, zfull = zkept + zm * adju;
+      const float inv = zfull > 0.f ? unscale / zfull : 0.f;
+      const float adj = adju * unscale;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 16) {
         float okv[16], ouv[16];
@@ -1187,8 +1209,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
           for (int c = 0; c < 16; c += 2) {
             const bool in0 = c0 + c < a.d, in1 = c0 + c + 1 < a.d;
-            const float o0 = in0 ? (okv[c] + ouv[c]) * inv : 0.f;
-            const float o1 = in1 ? (okv[c + 1] + ouv[c + 1]) * inv : 0.f;
+            const float o0 = in0 ? fmaf(okv[c], adjk, ouv[c] * adju) * inv : 0.f;
+            const float o1 = in1 ? fmaf(okv[c + 1], adjk, ouv[c + 1] * adju) * inv : 0.f;
             w[c / 2] = pack_bf16x2(o0, o1);
             uo[c] = in0 ? ouv[c] * adj : 0.f;
             uo[c + 1] = in1 ? ouv[c + 1] * adj : 0.f;
@@ -1202,9 +1224,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         }
       }
       if (valid) {  // the sums carry no V scale
-        a.out_m[row_g] = m_seen * kLn2;
-        a.out_zfull[row_g] = (zk + zm) * adjz;
-        a.out_zkept[row_g] = zk * adjz;
+        a.out_m[row_g] = M * kLn2;
+        a.out_zfull[row_g] = zfull;
+        a.out_zkept[row_g] = zkept;
       }
     }
   }

@@ -1,7 +1,7 @@
 // mask_builder.cuh -- which key blocks each query block keeps.
 //
-// Re-ttention project page, Abstract: the sparse step attends to "only a
-// subset of tokens or patches" (as few as 3.1%).  The subset rule used here:
+// Re-ttention project page, Abstract: the sparse step attends to a small
+// subset of the tokens (down to 3.1% of them).  The subset rule used here:
 // mean-pool each block of Q and K, score every (query block, key block) pair
 // by the scaled dot product of the pooled vectors, keep the forced prefix
 // blocks plus the best-scoring others, ties to the lower block index, and

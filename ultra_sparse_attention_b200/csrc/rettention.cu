@@ -257,19 +257,60 @@ rt_status mask_for_dim(const Dims& d, const void* q, const void* k, float scale,
 
 constexpr int kMaxDevices = 64;
 std::mutex g_static_pool_mutex;
-float* g_static_pool_addr[kMaxDevices] = {};
+struct StaticPoolEntry {
+  unsigned long long ctx_id;  // the CUDA context the address belongs to (0: none yet)
+  float* addr;
+};
+StaticPoolEntry g_static_pool_addr[kMaxDevices] = {};
 
-// Device address of g_static_pool on the current device, looked up once per device.
+// Unique id of the calling thread's current CUDA context (0 if there is none or the driver
+// cannot say).  Context ids are never reused within a process, so an address cached under an
+// id stays valid exactly as long as that context lives.
+unsigned long long current_context_id() {
+  using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+  using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_static_pool on the current device.  It is looked up with
+// cudaGetSymbolAddress the first time the device's current context calls, and again
+// whenever that context has changed (after cudaDeviceReset the runtime creates a new
+// primary context and loads the module again, at a new address).  Without a context id
+// the address is looked up on every call.
 rt_status static_pool_address(float** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RT_ERR_CUDA;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_static_pool_mutex);
-  if (g_static_pool_addr[dev] == nullptr) {
+  StaticPoolEntry& e = g_static_pool_addr[dev];
+  if (ctx == 0 || e.ctx_id != ctx || e.addr == nullptr) {
+    // The lookup makes the device's primary context current if no context was (a thread's
+    // first runtime call), so the id is taken again after it.
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_pool) != cudaSuccess || p == nullptr) return RT_ERR_CUDA;
-    g_static_pool_addr[dev] = static_cast<float*>(p);
+    e.addr = static_cast<float*>(p);
+    e.ctx_id = current_context_id();
   }
-  *out = g_static_pool_addr[dev];
+  *out = e.addr;
   return RT_OK;
 }
 
