@@ -350,13 +350,16 @@ def run_ours(args, rank, world, local):
          e2e["ms_per_step"] if e2e else 0.0], device, world)
     return {"w": w, "keep": keep, "keep_ratio": keep_ratio, "total_ms": total_ms, "mask_ms": mask_ms,
             "pair_ms": pair_ms, "capture_ms": cap_ms, "sparse_ms": sp_ms, "e2e": e2e, "e2e_ms": e2e_ms, "clocks": clk, "nums": nums,
-            "host1": host1, "host0": host0}
+            "host1": host1, "host0": host0, "gpu": {"row_ptr": rp, "col_idx": ci, "out0": out0, "out1": out1,
+                                                    "stats": stats}}
 
 
 # --------------------------------------------------------------------------- configuration sweep
-def run_sweep(args, device) -> list:
+def run_sweep(args, device, checker=None) -> list:
     """Per-kernel times of one mask + capture + sparse cycle on every workload
-    (the 5B shape at every keep ratio), L2 flushed between cycles."""
+    (the 5B shape at every keep ratio), L2 flushed between cycles.  With a
+    `checker` (the CPU-baseline leg's OracleChecker) each row also carries the
+    oracle's error figures on sampled rows of that cycle's outputs."""
     import ultra_sparse_attention_b200 as usa
 
     peaks, _ = load_peaks()
@@ -370,8 +373,10 @@ def run_sweep(args, device) -> list:
         ratio = w.keep[0] if ratio is None else ratio
         keep = w.keep_blocks(ratio)
         steps = denoising_inputs(w, 2)
-        q0, k0, v0 = (x.to(device) for x in next(steps)[1:])
-        q1, k1, v1 = (x.to(device) for x in next(steps)[1:])
+        host0 = next(steps)[1:]
+        host1 = next(steps)[1:]
+        q0, k0, v0 = (x.to(device) for x in host0)
+        q1, k1, v1 = (x.to(device) for x in host1)
         kw = dict(head_dim=w.head_dim, block_size=w.block_size, scale=w.scale)
         times = {"mask": [], "pair": [], "capture": [], "sparse": []}
         rp = ci = tb = None
@@ -383,9 +388,9 @@ def run_sweep(args, device) -> list:
             ev[1].record(stream)
             tb = usa.rt_pair_query_blocks(q0, rp, ci, head_dim=w.head_dim, block_size=w.block_size)
             ev[2].record(stream)
-            _, st = usa.rt_attn_full_capture(q0, k0, v0, row_ptr=rp, col_idx=ci, **kw)
+            out0, st = usa.rt_attn_full_capture(q0, k0, v0, row_ptr=rp, col_idx=ci, **kw)
             ev[3].record(stream)
-            usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rp, col_idx=ci, stats=st, tile_blocks=tb, **kw)
+            out1 = usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rp, col_idx=ci, stats=st, tile_blocks=tb, **kw)
             ev[4].record(stream)
             if it >= args.sweep_warmup:
                 for i, k in enumerate(("mask", "pair", "capture", "sparse")):
@@ -417,7 +422,9 @@ def run_sweep(args, device) -> list:
                     "capture_tflops": cap, "capture_frac_of_bf16_peak": cap / peaks["bf16_tflops"],
                     "reshape_rel_l2_vs_full": err_r, "plain_sparse_rel_l2_vs_full": err_p,
                     "steps": args.sweep_steps, "warmup": args.sweep_warmup, "l2": "flushed between cycles"})
-        del q0, k0, v0, q1, k1, v1, st, rp, ci, tb
+        if checker is not None:
+            out[-1]["oracle_check"] = checker.check(w, keep, host0, host1, rp, ci, out0, st, out1)
+        del q0, k0, v0, q1, k1, v1, st, rp, ci, tb, out0, out1, host0, host1
     return out
 
 
@@ -454,6 +461,53 @@ class OracleSample:
         secs = min(self.time_step() for _ in range(repeats))
         return {"value": self.dense_flops / secs / 1e12, "unit": UNIT, "cores": self.threads, "kind": "oracle",
                 "sample": self.desc}
+
+
+class OracleChecker:
+    """Part of the CPU-baseline leg: the GPU outputs of a cycle against the fp64 oracle on a
+    few sampled rows (capture output and statistics, sparse output), with the oracle's own
+    block mask.  Rows are sampled only from query blocks whose kept sets the GPU mask and the
+    oracle's agree on (a near tie may make them differ; the count is reported)."""
+
+    def __init__(self, rows: int = 64, seed: int = 1):
+        import oracle
+        self.oracle, self.rows, self.seed = oracle, rows, seed
+
+    def check(self, w, keep, host0, host1, rp_gpu, ci_gpu, out0, st, out1) -> dict:
+        orc = self.oracle
+        d, bs, D, N = w.head_dim, w.block_size, w.head_dim_padded, w.seq_len
+        rp_o, ci_o = orc.build_block_mask(host0[0], host0[1], d, bs, w.scale, keep, w.forced_prefix_tokens)
+        rp_g = rp_gpu.cpu().numpy() if torch.is_tensor(rp_gpu) else rp_gpu
+        ci_g = ci_gpu.cpu().numpy() if torch.is_tensor(ci_gpu) else ci_gpu
+        nb = w.n_blocks
+        n_qb = w.batch * w.heads * nb
+        same = np.array([np.array_equal(ci_g[rp_g[r]:rp_g[r + 1]], ci_o[rp_o[r]:rp_o[r + 1]]) for r in range(n_qb)])
+        rng = np.random.default_rng(self.seed)
+        cand = rng.choice(w.batch * w.heads * N, size=min(w.batch * w.heads * N, 8 * self.rows), replace=False)
+        cand = cand[same[(cand // N) * nb + (cand % N) // bs]]
+        rows = np.sort(cand[:self.rows]).astype(np.int64)
+        cap = orc.full_capture(*host0, d, bs, w.scale, rp_o, ci_o, rows=rows)
+        cap_abs = orc.full_capture(host0[0], host0[1], host0[2].abs(), d, bs, w.scale, rp_o, ci_o, rows=rows)["u"]
+        sp = orc.sparse_reshape(*host1, d, bs, w.scale, rp_o, ci_o, cap, rows=rows)
+        sel = torch.as_tensor(rows, device=out0.device)
+
+        def errs(got, want):
+            g = got.reshape(-1, D)[sel].double().cpu().numpy()[:, :d]
+            e = np.abs(g - want)
+            return {"max_abs_unit_scale": float(np.max(e / np.maximum(1.0, np.abs(want)))),
+                    "mean_abs": float(e.mean())}
+
+        zf = st.zfull.reshape(-1)[sel].double().cpu().numpy()
+        zk = st.zkept.reshape(-1)[sel].double().cpu().numpy()
+        m = st.m.reshape(-1)[sel].double().cpu().numpy()
+        u = st.u.reshape(-1, D)[sel].double().cpu().numpy()[:, :d]
+        bound = 1e-3 * cap_abs / cap["zfull"][:, None] + 1e-7
+        stats = {"ratio_rel": float(np.max(np.abs((zf / zk) / (cap["zfull"] / cap["zkept"]) - 1))),
+                 "lse_abs": float(np.max(np.abs(m + np.log(zf) - cap["m"] - np.log(cap["zfull"])))),
+                 "u_err_over_bound": float(np.max(np.abs(u / zf[:, None] - cap["u"] / cap["zfull"][:, None]) / bound))}
+        return {"rows": int(len(rows)), "mask_rows_differing": int(n_qb - int(same.sum())),
+                "capture_o": errs(out0, cap["o"]), "capture_stats": stats, "sparse_o": errs(out1, sp),
+                "tolerance": "o: max-abs 1.5e-2 at unit scale, mean-abs 1.5e-3; stats: 1e-3 relative"}
 
 
 def run_reference(args, rank, world):
@@ -504,12 +558,19 @@ def main():
     r = run_ours(args, rank, world, local)
     if rank == 0:
         peaks, peak_src = load_peaks()
+        # The CPU-baseline leg (rank 0 at one GPU): the oracle's timed sample, and its error
+        # check of the GPU outputs on sampled rows of the main cycle and of every sweep cycle.
+        cpu_leg = not args.no_cpu_baseline and world == 1
+        checker = OracleChecker() if cpu_leg else None
         sweep = None
         if not args.no_sweep and world == 1:
-            sweep = run_sweep(args, torch.device("cuda", local))
+            sweep = run_sweep(args, torch.device("cuda", local), checker)
         cpu = None
-        if not args.no_cpu_baseline and world == 1:
+        if cpu_leg:
             cpu = OracleSample(r["w"], r["keep"], r["host0"], r["host1"], args.cpu_rows).baseline()
+            g = r["gpu"]
+            cpu["oracle_check"] = checker.check(r["w"], r["keep"], r["host0"], r["host1"], g["row_ptr"],
+                                                g["col_idx"], g["out0"], g["stats"], g["out1"])
         print(json.dumps(build_line(args, r, world, peaks, peak_src, sweep, cpu)), flush=True)
     if world > 1:
         torch.distributed.barrier()
@@ -562,6 +623,27 @@ def build_line(args, r: dict, world: int, peaks: dict, peak_src: str, sweep, cpu
         ach = kernels["rt_build_block_mask"]["achieved_gbs"]
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": f"hbm_gbs ({peak_src})"}
+    # The kernel the target is stated for: the sparse step on its executed (kept-block) flops,
+    # beside its achieved HBM bandwidth on the algorithmic bytes.
+    sp_ach = exec_tflops
+    roof_sparse = {"kernel": "rt_attn_sparse_reshape", "bound": "tensor", "achieved": sp_ach,
+                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": sp_ach / peaks["bf16_tflops"],
+                   "traffic": stored_traffic("sparse_reshape_kernel", wl_tag),
+                   "peak_source": f"bf16_tflops ({peak_src}, burst)",
+                   "per_launch": f"{nums['executed_flops'] / 1e12:.4f} TFLOP executed (kept blocks, 4*d*rows*cols)",
+                   "hbm_achieved_gbs": nums["sparse_bytes"] / sp_s / 1e9,
+                   "hbm_frac": nums["sparse_bytes"] / sp_s / 1e9 / peaks["hbm_gbs"],
+                   "algorithmic_bytes": nums["sparse_bytes"], "target_frac": 0.5}
+    kept_tokens = nums["executed_flops"] / nums["dense_flops"]
+    claims = [
+        {"claim": "full-attention quality with as few as 3.1% of the tokens", "source":
+         "Re-ttention project page, Abstract", "hardware": "not stated",
+         "here": f"{r['keep']}/{w.n_blocks} key blocks per query block = {100.0 * r['keep'] / w.n_blocks:.2f}% of the "
+                 f"keys; {100.0 * kept_tokens:.2f}% of the dense score work executed"},
+        {"claim": "over 95% of the attention computation skipped", "source": "Re-ttention project page, teaser",
+         "hardware": "not stated", "here": f"{100.0 * (1.0 - kept_tokens):.2f}% of the dense QK^T and PV flops skipped "
+                                           "in the sparse step"},
+    ]
     e2e = None
     if r["e2e"]:
         e2e = {"value": job_throughput(nums["dense_flops"], world, r["e2e_ms"]), "unit": UNIT,
@@ -578,7 +660,8 @@ def build_line(args, r: dict, world: int, peaks: dict, peak_src: str, sweep, cpu
         "sparse_step_ms": r["sparse_ms"], "full_step_ms": r["mask_ms"] + r["pair_ms"] + r["capture_ms"],
         "dense_equiv_tflops": nums["dense_flops"] / sp_s / 1e12, "executed_tflops": exec_tflops,
         "tensor_pct_of_bf16_peak": 100.0 * exec_tflops / peaks["bf16_tflops"],
-        "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+        "roofline": roof, "roofline_sparse": roof_sparse, "pages_claims": claims,
+        "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": r["clocks"],
         "peaks": {**peaks, "source": peak_src},
         "sweep": sweep,

@@ -119,3 +119,51 @@ def test_reference_line_has_the_contract_keys():
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert bench.run_reference(A, 1, 2) is None
+
+
+def test_sparse_roofline_and_page_claims():
+    r = _measurement(1)
+    peaks = dict(bench.FALLBACK_PEAKS)
+    line = bench.build_line(_Args, r, 1, peaks, "fallback", None, None)
+    rs = line["roofline_sparse"]
+    assert rs["kernel"] == "rt_attn_sparse_reshape" and rs["bound"] == "tensor" and rs["unit"] == "TFLOP/s"
+    assert rs["achieved"] == pytest.approx(r["nums"]["executed_flops"] / 0.25e-3 / 1e12)
+    assert rs["frac"] == pytest.approx(rs["achieved"] / peaks["bf16_tflops"])
+    assert rs["hbm_frac"] == pytest.approx(r["nums"]["sparse_bytes"] / 0.25e-3 / 1e9 / peaks["hbm_gbs"])
+    claims = line["pages_claims"]
+    assert len(claims) == 2 and all(c["hardware"] == "not stated" and c["source"] for c in claims)
+    assert "3.1%" in claims[0]["claim"] and "95%" in claims[1]["claim"]
+
+
+def test_oracle_checker_on_oracle_outputs():
+    """The checker's error figures are those of bf16-rounded oracle outputs: within the
+    tolerances, with no mask row differing when it is given the oracle's own CSR."""
+    import torch
+
+    import oracle
+    w = bench.WORKLOADS["tiny"]
+    steps = list(bench.denoising_inputs(w, 2))
+    h0, h1 = steps[0][1:], steps[1][1:]
+    keep = w.keep_blocks()
+    d, bs, D, N = w.head_dim, w.block_size, w.head_dim_padded, w.seq_len
+    rp, ci = oracle.build_block_mask(h0[0], h0[1], d, bs, w.scale, keep, 0)
+    cap = oracle.full_capture(*h0, d, bs, w.scale, rp, ci)
+    sp = oracle.sparse_reshape(*h1, d, bs, w.scale, rp, ci, cap)
+    B, H = w.batch, w.heads
+
+    def as_out(x):
+        t = torch.zeros(B * H * N, D)
+        t[:, :d] = torch.as_tensor(x, dtype=torch.float32)
+        return t.to(torch.bfloat16).reshape(B, H, N, D)
+
+    u = torch.zeros(B * H * N, D)
+    u[:, :d] = torch.as_tensor(cap["u"], dtype=torch.float32)
+    st = bench.OracleChecker  # the checker only reads .m .zfull .zkept .u
+    stats = type("S", (), {"m": torch.as_tensor(cap["m"], dtype=torch.float32),
+                           "zfull": torch.as_tensor(cap["zfull"], dtype=torch.float32),
+                           "zkept": torch.as_tensor(cap["zkept"], dtype=torch.float32), "u": u})()
+    res = st(rows=32).check(w, keep, h0, h1, rp, ci, as_out(cap["o"]), stats, as_out(sp))
+    assert res["rows"] == 32 and res["mask_rows_differing"] == 0
+    for k in ("capture_o", "sparse_o"):
+        assert res[k]["max_abs_unit_scale"] <= 2 ** -8 and res[k]["mean_abs"] <= 1.5e-3
+    assert res["capture_stats"]["ratio_rel"] < 1e-6 and res["capture_stats"]["u_err_over_bound"] < 0.01

@@ -121,3 +121,84 @@ def test_full_size_cycle_matches_oracle(cuda_device, name, keep):
         err_reshape = np.linalg.norm(g_rows - full) / np.linalg.norm(full)
         err_plain = np.linalg.norm(p_rows - full) / np.linalg.norm(full)
         assert err_reshape < 0.5 * err_plain, (name, err_reshape, err_plain)
+
+
+# ------------------------------------------------------------------ the farthest step of each schedule
+def _schedule_cases():
+    """(workload, farthest sparse step after the capture at step 0): the last step before the
+    next capture, where the inputs have drifted furthest from the cached statistics."""
+    out = []
+    for name in ("tiny", "image", "video2b", "long"):
+        w = WORKLOADS[name]
+        out.append((name, min(w.capture_every, w.steps) - 1))
+    return out
+
+
+@pytest.mark.parametrize("name,t_far", _schedule_cases(), ids=[f"{n}-t{t}" for n, t in _schedule_cases()])
+def test_farthest_sparse_step_of_the_schedule(cuda_device, name, t_far):
+    """Mask and capture at step 0, then the sparse step at the end of the capture's reuse
+    window (image t4, video2b t4, long t9, tiny t2) with the step-0 statistics, on sampled
+    rows against the oracle (same CSR, the oracle's own step-0 statistics); the reshape must
+    still be much closer to full attention of that step than plain sparse attention."""
+    w = WORKLOADS[name]
+    d, bs, D = w.head_dim, w.block_size, w.head_dim_padded
+    bh, N = w.batch * w.heads, w.seq_len
+    h0 = hf = None
+    for t, q, k, v in denoising_inputs(w, t_far + 1):
+        if t == 0:
+            h0 = (q, k, v)
+        hf = (q, k, v)
+    d0 = [x.to(cuda_device) for x in h0]
+    df = [x.to(cuda_device) for x in hf]
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale)
+    keep = w.keep_blocks()
+    rp, ci = usa.rt_build_block_mask(d0[0], d0[1], keep_blocks=keep, forced_prefix_tokens=w.forced_prefix_tokens, **kw)
+    tiles = usa.rt_pair_query_blocks(d0[0], rp, ci, head_dim=d, block_size=bs)
+    _, st = usa.rt_attn_full_capture(*d0, row_ptr=rp, col_idx=ci, **kw)
+    out = usa.rt_attn_sparse_reshape(*df, row_ptr=rp, col_idx=ci, stats=st, tile_blocks=tiles, **kw)
+    plain = usa.rt_attn_sparse_reshape(*df, row_ptr=rp, col_idx=ci, stats=None, tile_blocks=tiles, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    rp_h, ci_h = rp.cpu().numpy(), ci.cpu().numpy()
+    rows = sample_rows(bh, N, SAMPLE_ROWS, seed=100 + t_far)
+    orc0 = oracle.full_capture(*h0, d, bs, w.scale, rp_h, ci_h, rows=rows)
+    want = oracle.sparse_reshape(*hf, d, bs, w.scale, rp_h, ci_h, orc0, rows=rows)
+    sel = torch.as_tensor(rows, device=cuda_device)
+    got = out.reshape(-1, D)[sel]
+    compare_out(got, want, d, f"{name} sparse O at step {t_far}")
+    full = oracle.full_capture(*hf, d, bs, w.scale, rp_h, ci_h, rows=rows)["o"]
+    g_rows = got.double().cpu().numpy()[:, :d]
+    p_rows = plain.reshape(-1, D)[sel].double().cpu().numpy()[:, :d]
+    err_reshape = np.linalg.norm(g_rows - full) / np.linalg.norm(full)
+    err_plain = np.linalg.norm(p_rows - full) / np.linalg.norm(full)
+    assert err_reshape < 0.5 * err_plain, (name, t_far, err_reshape, err_plain)
+
+
+# ------------------------------------------------------------------ one whole head
+@pytest.mark.parametrize("name", ["image", "video2b", "video5b", "long"])
+def test_whole_head_matches_oracle(cuda_device, name):
+    """Every row of one head (b = 0, h = H/2) of the full-size workload: the capture step's
+    output and statistics, and the sparse step after it, against the oracle."""
+    w, h0, h1 = _host_inputs(name)
+    d, bs, D = w.head_dim, w.block_size, w.head_dim_padded
+    N = w.seq_len
+    head = w.heads // 2  # batch 0
+    rows = head * N + np.arange(N, dtype=np.int64)
+    d0 = [x.to(cuda_device) for x in h0]
+    d1 = [x.to(cuda_device) for x in h1]
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale)
+    keep = w.keep_blocks()
+    rp, ci = usa.rt_build_block_mask(d0[0], d0[1], keep_blocks=keep, forced_prefix_tokens=w.forced_prefix_tokens, **kw)
+    tiles = usa.rt_pair_query_blocks(d0[0], rp, ci, head_dim=d, block_size=bs)
+    out0, st = usa.rt_attn_full_capture(*d0, row_ptr=rp, col_idx=ci, **kw)
+    out1 = usa.rt_attn_sparse_reshape(*d1, row_ptr=rp, col_idx=ci, stats=st, tile_blocks=tiles, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    rp_h, ci_h = rp.cpu().numpy(), ci.cpu().numpy()
+    sel = torch.as_tensor(rows, device=cuda_device)
+    orc = oracle.full_capture(*h0, d, bs, w.scale, rp_h, ci_h, rows=rows)
+    orc_abs = oracle.full_capture(h0[0], h0[1], h0[2].abs(), d, bs, w.scale, rp_h, ci_h, rows=rows)["u"]
+    compare_out(out0.reshape(-1, D)[sel], orc["o"], d, f"{name} head {head} capture O")
+    compare_stats(st, rows, orc, orc_abs, d, f"{name} head {head} capture stats")
+    want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp_h, ci_h, orc, rows=rows)
+    compare_out(out1.reshape(-1, D)[sel], want, d, f"{name} head {head} sparse O")
