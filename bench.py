@@ -203,9 +203,11 @@ def workload_numbers(w, keep: int, row_ptr, col_idx):
     dense = 4.0 * bh * N * N * d
     executed = 4.0 * d * kept_work(row_ptr, col_idx, N, w.block_size, bh)
     sparse_bytes = bh * N * (D * 2 * 2 + D * 4 + 12) + 2 * bh * N * D * 2  # Q, O, U, stats; K and V once
+    sparse_bytes_c = bh * N * (D * 2 * 2 + D * 2 + 16) + 2 * bh * N * D * 2  # the same with f16 U and its row scale
     capture_bytes = 3 * bh * N * D * 2 + bh * N * (D * 2 + D * 4 + 12)     # Q, K, V; O, U, stats
     mask_bytes = 2 * bh * N * D * 2                                       # Q and K read once
     return {"dense_flops": dense, "executed_flops": executed, "sparse_bytes": sparse_bytes,
+            "sparse_bytes_compressed": sparse_bytes_c,
             "capture_bytes": capture_bytes, "mask_bytes": mask_bytes}
 
 
@@ -289,6 +291,28 @@ def run_ours(args, rank, world, local):
     if usa.rt_take_device_error() != 0:
         raise RuntimeError("a kernel reported a device error in the timed region")
 
+    # The sparse step reading the compressed residual cache (f16 U with a per-row scale),
+    # timed on its own after the main loop: the same launch on the same inputs.
+    _, stats_c = usa.rt_attn_full_capture(q0, k0, v0, row_ptr=row_ptr, col_idx=col_idx, compressed=True, **kw)
+    out1c = torch.empty_like(q1)
+    for _ in range(args.warmup):
+        usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=row_ptr, col_idx=col_idx, stats=stats_c, tile_blocks=tiles,
+                                   out=out1c, **kw)
+    ev_c = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for a, b in ev_c:
+        a.record(stream)
+        usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=row_ptr, col_idx=col_idx, stats=stats_c, tile_blocks=tiles,
+                                   out=out1c, **kw)
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    sparse_c_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_c)
+    if usa.rt_take_device_error() != 0:
+        raise RuntimeError("a kernel reported a device error in the compressed-cache loop")
+    del stats_c, out1c
+
     rp, ci = row_ptr.cpu().numpy(), col_idx.cpu().numpy()
     nums = workload_numbers(w, keep, rp, ci)
     nums["key_tiles_per_query_tile"] = key_tiles_per_query_tile(rp, ci, tiles.cpu().numpy(), nb, w.block_size, B * H, N)
@@ -345,11 +369,12 @@ def run_ours(args, rank, world, local):
                "d2h_bytes_per_step": int(h_out[0].numel() * h_out[0].element_size())}
         del d_in, d_out
 
-    total_ms, mask_ms, pair_ms, cap_ms, sp_ms, e2e_ms = max_over_ranks(
+    total_ms, mask_ms, pair_ms, cap_ms, sp_ms, e2e_ms, sp_c_ms = max_over_ranks(
         [total_ms, per_kernel["mask"], per_kernel["pair"], per_kernel["capture"], per_kernel["sparse"],
-         e2e["ms_per_step"] if e2e else 0.0], device, world)
+         e2e["ms_per_step"] if e2e else 0.0, sparse_c_ms], device, world)
     return {"w": w, "keep": keep, "keep_ratio": keep_ratio, "total_ms": total_ms, "mask_ms": mask_ms,
-            "pair_ms": pair_ms, "capture_ms": cap_ms, "sparse_ms": sp_ms, "e2e": e2e, "e2e_ms": e2e_ms, "clocks": clk, "nums": nums,
+            "pair_ms": pair_ms, "capture_ms": cap_ms, "sparse_ms": sp_ms, "sparse_compressed_ms": sp_c_ms,
+            "e2e": e2e, "e2e_ms": e2e_ms, "clocks": clk, "nums": nums,
             "host1": host1, "host0": host0, "gpu": {"row_ptr": rp, "col_idx": ci, "out0": out0, "out1": out1,
                                                     "stats": stats}}
 
@@ -378,7 +403,7 @@ def run_sweep(args, device, checker=None) -> list:
         q0, k0, v0 = (x.to(device) for x in host0)
         q1, k1, v1 = (x.to(device) for x in host1)
         kw = dict(head_dim=w.head_dim, block_size=w.block_size, scale=w.scale)
-        times = {"mask": [], "pair": [], "capture": [], "sparse": []}
+        times = {"mask": [], "pair": [], "capture": [], "sparse": [], "sparse_c": []}
         rp = ci = tb = None
         for it in range(args.sweep_warmup + args.sweep_steps):
             flush.zero_()
@@ -395,6 +420,17 @@ def run_sweep(args, device, checker=None) -> list:
             if it >= args.sweep_warmup:
                 for i, k in enumerate(("mask", "pair", "capture", "sparse")):
                     times[k].append((ev[i], ev[i + 1]))
+        # the sparse step on the compressed cache (same mask and tiles), L2 flushed likewise
+        _, st_c = usa.rt_attn_full_capture(q0, k0, v0, row_ptr=rp, col_idx=ci, compressed=True, **kw)
+        for it in range(args.sweep_warmup + args.sweep_steps):
+            flush.zero_()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            e[0].record(stream)
+            usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rp, col_idx=ci, stats=st_c, tile_blocks=tb, **kw)
+            e[1].record(stream)
+            if it >= args.sweep_warmup:
+                times["sparse_c"].append((e[0], e[1]))
+        del st_c
         # How close the reshaped sparse step comes to full attention of its own inputs (the
         # capture kernel's output on them), against plain block-sparse attention.
         full1, _ = usa.rt_attn_full_capture(q1, k1, v1, row_ptr=rp, col_idx=ci, **kw)
@@ -415,6 +451,7 @@ def run_sweep(args, device, checker=None) -> list:
         out.append({"workload": name, "shape": f"B={w.batch} H={w.heads} N={w.seq_len} d={w.head_dim} D={w.head_dim_padded} "
                                                f"block={w.block_size}",
                     "keep": f"{keep}/{w.n_blocks} ({ratio})", "sparse_step_ms": ms["sparse"],
+                    "sparse_step_ms_compressed_cache": ms["sparse_c"],
                     "full_step_ms": ms["mask"] + ms["pair"] + ms["capture"], "mask_ms": ms["mask"],
                     "pair_ms": ms["pair"], "capture_ms": ms["capture"],
                     "dense_equiv_tflops": nums["dense_flops"] / sp_s / 1e12, "executed_tflops": exe,
@@ -602,6 +639,17 @@ def build_line(args, r: dict, world: int, peaks: dict, peak_src: str, sweep, cpu
                                    "key_tiles_per_query_tile": nums.get("key_tiles_per_query_tile"),
                                    "key_tiles_per_query_tile_neighbours": nums.get("key_tiles_per_query_tile_neighbours")},
     }
+    if r.get("sparse_compressed_ms"):
+        spc_s = r["sparse_compressed_ms"] / 1e3
+        exc = nums["executed_flops"] / spc_s / 1e12
+        kernels["rt_attn_sparse_reshape_u16"] = {
+            "ms": r["sparse_compressed_ms"], "bound": "tensor+hbm", "executed_tflops": exc,
+            "tensor_frac_of_bf16_peak": exc / peaks["bf16_tflops"],
+            "dense_equiv_tflops": nums["dense_flops"] / spc_s / 1e12,
+            "achieved_gbs": nums["sparse_bytes_compressed"] / spc_s / 1e9,
+            "algorithmic_bytes": nums["sparse_bytes_compressed"],
+            "what": "the sparse step reading the compressed residual cache (f16 U, one power-of-two scale per row), "
+                    "timed in its own loop after the main one"}
     # dominant kernel of the step (by device time)
     dom = max(("rt_attn_full_capture", r["capture_ms"]), ("rt_attn_sparse_reshape", r["sparse_ms"]),
               ("rt_build_block_mask", r["mask_ms"]), key=lambda t: t[1])[0]

@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define RT_ABI_VERSION 5
+#define RT_ABI_VERSION 6
 
 typedef enum rt_status {
     RT_OK = 0,
@@ -205,6 +205,41 @@ rt_status rt_attn_sparse_reshape(const rt_shape *shape, const void *q, const voi
                                  const float *stat_m, const float *stat_zfull,
                                  const float *stat_zkept, const float *stat_u, void *out,
                                  rt_stream_t stream);
+
+/*
+ * rt_attn_full_capture_u16, rt_attn_sparse_reshape_u16 -- the same two steps
+ * with a compressed residual cache.
+ *
+ * The mechanism highlight caches the residual contribution of the masked-out
+ * tokens; at a few per cent of kept keys that cache (U, D values per row) is
+ * the largest stream the sparse step reads.  These variants store U as f16
+ * with one power-of-two scale per row instead of fp32, which halves it:
+ *   U_i = stat_u16_i * stat_u_scale_i,
+ * where stat_u_scale_i = 2^-k is chosen so that the row's largest |U_i[c]|
+ * times 2^k lies in [2^14, 2^15) (a row without masked keys gets scale 1 and
+ * zeros).  Every element down to 2^-28 of its row's largest keeps 11 mantissa
+ * bits (relative error below 2^-12, inside the 1e-3 statistics tolerance).
+ * m, Z_full and Z_kept stay fp32.  Everything else -- arguments, layouts,
+ * results, errors -- is as for rt_attn_full_capture and rt_attn_sparse_reshape.
+ *
+ * stat_u16      f16 bits [B,H,N,D] device (16-byte aligned; columns d..D-1 zero):
+ *               written by the capture call, read by the sparse call.
+ * stat_u_scale  fp32 [B,H,N] device: written / read likewise.
+ * The sparse variant requires all five statistics pointers (plain block-sparse
+ * attention is rt_attn_sparse_reshape with NULL statistics).
+ */
+rt_status rt_attn_full_capture_u16(const rt_shape *shape, const void *q, const void *k,
+                                   const void *v, float scale, const int32_t *row_ptr,
+                                   const int32_t *col_idx, void *out, float *stat_m,
+                                   float *stat_zfull, float *stat_zkept, uint16_t *stat_u16,
+                                   float *stat_u_scale, void *workspace, size_t workspace_bytes,
+                                   rt_stream_t stream);
+rt_status rt_attn_sparse_reshape_u16(const rt_shape *shape, const void *q, const void *k,
+                                     const void *v, float scale, const int32_t *row_ptr,
+                                     const int32_t *col_idx, const int32_t *tile_blocks,
+                                     const float *stat_m, const float *stat_zfull,
+                                     const float *stat_zkept, const uint16_t *stat_u16,
+                                     const float *stat_u_scale, void *out, rt_stream_t stream);
 
 /*
  * rt_pair_query_blocks -- group the query blocks of each head into the

@@ -32,7 +32,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    assert usa.rt_abi_version() == 5
+    assert usa.rt_abi_version() == 6
     for code in range(5):
         s = usa.rt_status_string(code)
         assert s.startswith("RT_")
@@ -144,3 +144,29 @@ def test_workspace_sizes_and_validation():
     assert _capture(lib, ok, ws=A4, ws_bytes=cap) == usa.RT_ERR_INVALID_ARGUMENT
     assert _pair(lib, ok, ws=A16, ws_bytes=pair - 1) == usa.RT_ERR_INVALID_ARGUMENT
     assert _pair(lib, ok, ws=MIS, ws_bytes=pair) == usa.RT_ERR_INVALID_ARGUMENT
+
+
+def test_compressed_cache_argument_validation():
+    """The f16-U variants validate like the fp32 ones, and need U's scale array."""
+    lib = usa.load_library()
+    ok = RtShape(2, 3, 1000, 72, 80, 64)
+
+    def cap16(u16=A16, us=A16, m=A16, shape=ok):
+        return lib.rt_attn_full_capture_u16(ctypes.byref(shape), A16, A16, A16, 0.125, A16, A16, A16, m, A16, A16,
+                                            u16, us, None, 0, None)
+
+    def sp16(stats=(A16, A16, A16, A16, A16), shape=ok, out=A16):
+        return lib.rt_attn_sparse_reshape_u16(ctypes.byref(shape), A16, A16, A16, 0.125, A16, A16, None, *stats,
+                                              out, None)
+
+    assert cap16(u16=None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert cap16(us=None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert cap16(u16=A4) == usa.RT_ERR_INVALID_ARGUMENT       # U must be 16-byte aligned
+    assert cap16(us=MIS) == usa.RT_ERR_INVALID_ARGUMENT
+    assert cap16(m=MIS) == usa.RT_ERR_INVALID_ARGUMENT
+    assert cap16(shape=RtShape(2, 3, 1000, 72, 96, 64)) == usa.RT_ERR_UNSUPPORTED
+    assert sp16(stats=(None, None, None, None, None)) == usa.RT_ERR_INVALID_ARGUMENT  # all five needed
+    assert sp16(stats=(A16, A16, A16, A16, None)) == usa.RT_ERR_INVALID_ARGUMENT
+    assert sp16(stats=(A16, A16, A16, A4, A16)) == usa.RT_ERR_INVALID_ARGUMENT
+    assert sp16(out=None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert sp16(shape=RtShape(2, 3, 1000, 72, 80, 32)) == usa.RT_ERR_UNSUPPORTED

@@ -108,6 +108,17 @@ def test_full_size_cycle_matches_oracle(cuda_device, name, keep):
         nh = min(2, bh)
         np.testing.assert_array_equal(tiles_h[:nh], pair_query_blocks(rp_h, ci_h, nh, nb, bs, tiles_h.shape[1]))
     assert torch.equal(out1p.view(torch.int16), out1.view(torch.int16))
+    # the same cycle with the compressed residual cache (f16 U, one scale per row)
+    out0c, stc = usa.rt_attn_full_capture(*d0, row_ptr=rp, col_idx=ci, compressed=True, **kw)
+    out1c = usa.rt_attn_sparse_reshape(*d1, row_ptr=rp, col_idx=ci, stats=stc, tile_blocks=tiles, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    assert torch.equal(out0c.view(torch.int16), out0.view(torch.int16))
+    compare_stats(usa.Stats(stc.m, stc.zfull, stc.zkept, stc.residual()), rows, orc, orc_abs, d,
+                  f"{name} capture stats (compressed cache)")
+    compare_out(out1c.reshape(-1, D)[torch.as_tensor(rows, device=cuda_device)], want, d,
+                f"{name} sparse O (compressed cache)")
+    del out0c, stc, out1c
     full = oracle.full_capture(*h1, d, bs, w.scale, rp_h, ci_h, rows=rows)["o"]
     if keep == nb:
         compare_out(got, full, d, f"{name} keep-all sparse step vs full attention")

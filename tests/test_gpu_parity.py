@@ -618,3 +618,112 @@ def test_binding_rejects_mismatched_buffers(cuda_device):
         usa.rt_attn_sparse_reshape(q, q, q, row_ptr=rp.cpu(), col_idx=ci, stats=st, **kw)  # device
     torch.cuda.synchronize()
     assert usa.rt_take_device_error() == 0
+
+
+# ------------------------------------------------------------------ compressed residual cache (f16 U, row scale)
+def _decoded(st):
+    """The statistics with U decoded to fp32 (compare_stats reads .u)."""
+    return usa.Stats(st.m, st.zfull, st.zkept, st.residual())
+
+
+@pytest.mark.parametrize("N,d,D,bs", CASES)
+@pytest.mark.parametrize("keep_frac", [Fraction(1, 4), Fraction(1, 1)])
+def test_compressed_capture_matches_oracle(cuda_device, N, d, D, bs, keep_frac):
+    """The f16 cache with one power-of-two scale per row, decoded, against the oracle's U at
+    the unchanged statistics tolerance; output and the other statistics as before."""
+    w = _wl(N, d, D, bs, std=1.2, seed=7 * N + d)
+    (h0, _), (d0, _) = _inputs(w, cuda_device)
+    bh, nb = w.batch * w.heads, w.n_blocks
+    keep = w.keep_blocks(keep_frac)
+    rp, ci = random_csr(bh, nb, keep, seed=N)
+    out, st = usa.rt_attn_full_capture(*d0, head_dim=d, block_size=bs, scale=w.scale, compressed=True,
+                                       row_ptr=to_dev(rp, cuda_device), col_idx=to_dev(ci, cuda_device))
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    assert st.compressed and st.u.dtype == torch.float16
+    orc = oracle.full_capture(*h0, d, bs, w.scale, rp, ci)
+    orc_abs = oracle.full_capture(h0[0], h0[1], h0[2].abs(), d, bs, w.scale, rp, ci)["u"]
+    compare_out(out.reshape(-1, D), orc["o"], d, "capture O (compressed cache)")
+    compare_stats(_decoded(st), np.arange(bh * N), orc, orc_abs, d, "capture stats (compressed cache)")
+    if keep == nb:
+        assert torch.all(st.u == 0) and torch.all(st.u_scale == 1)
+
+
+@pytest.mark.parametrize("N,d,D,bs", [(1000, 64, 64, 64), (1000, 72, 80, 128), (1000, 128, 128, 64)])
+def test_compressed_cache_is_the_fp32_cache_rounded(cuda_device, N, d, D, bs):
+    """Both capture variants compute the same fp32 U; the compressed one stores it as
+    f16(U * 2^k) with 2^-k in u_scale and the row's largest |U| * 2^k in [2^14, 2^15):
+    bit for bit, and the output and the other statistics are identical."""
+    w = _wl(N, d, D, bs, std=1.2, seed=3 * N + d)
+    (_, _), (d0, _) = _inputs(w, cuda_device)
+    bh, nb = w.batch * w.heads, w.n_blocks
+    rp, ci = random_csr(bh, nb, max(1, nb // 4), seed=N + 5)
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale, row_ptr=to_dev(rp, cuda_device),
+              col_idx=to_dev(ci, cuda_device))
+    o32, s32 = usa.rt_attn_full_capture(*d0, **kw)
+    o16, s16 = usa.rt_attn_full_capture(*d0, compressed=True, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    assert torch.equal(o32.view(torch.int16), o16.view(torch.int16))
+    for a, b in ((s32.m, s16.m), (s32.zfull, s16.zfull), (s32.zkept, s16.zkept)):
+        assert torch.equal(a, b)
+    sc = s16.u_scale
+    mant, _ = torch.frexp(sc)
+    assert torch.all(mant == 0.5), "scales are powers of two"
+    want = (s32.u / sc[..., None]).to(torch.float16)
+    assert torch.equal(want.view(torch.int16), s16.u.view(torch.int16))
+    amax = s16.u.float().abs().amax(-1)
+    nz = s32.u.abs().amax(-1) > 0
+    assert torch.all((amax[nz] >= 2.0 ** 14) & (amax[nz] <= 2.0 ** 15))
+
+
+@pytest.mark.parametrize("N,d,D,bs", CASES)
+def test_sparse_with_compressed_cache_matches_oracle(cuda_device, N, d, D, bs):
+    """Capture with the compressed cache, then the sparse step on drifted inputs reading it:
+    against the oracle's sparse step with its own fp64 statistics."""
+    w = _wl(N, d, D, bs, std=1.2, seed=11 * N + d, drift=0.05)
+    (h0, h1), (d0, d1) = _inputs(w, cuda_device)
+    bh, nb = w.batch * w.heads, w.n_blocks
+    keep = w.keep_blocks(Fraction(1, 4))
+    rp, ci = random_csr(bh, nb, keep, seed=N + 1)
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale, row_ptr=to_dev(rp, cuda_device),
+              col_idx=to_dev(ci, cuda_device))
+    _, st = usa.rt_attn_full_capture(*d0, compressed=True, **kw)
+    tiles = usa.rt_pair_query_blocks(d0[0], kw["row_ptr"], kw["col_idx"], head_dim=d, block_size=bs)
+    out = usa.rt_attn_sparse_reshape(*d1, stats=st, tile_blocks=tiles, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    st_o = oracle.full_capture(*h0, d, bs, w.scale, rp, ci)
+    want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp, ci, st_o)
+    compare_out(out.reshape(-1, D), want, d, "sparse O (compressed cache)")
+    # unchanged inputs: the sparse step reading the compressed cache recovers the capture output
+    o0 = usa.rt_attn_sparse_reshape(*d0, stats=st, tile_blocks=tiles, **kw)
+    torch.cuda.synchronize()
+    compare_out(o0.reshape(-1, D), st_o["o"], d, "sparse on unchanged inputs (compressed cache)")
+
+
+@pytest.mark.parametrize("gap", [14.0, 18.0, 30.0])
+def test_compressed_capture_peaked_rows(cuda_device, gap):
+    """The peaked rows with the compressed cache: each row's scale follows its own largest
+    |U|, however small U is next to the row's maximum."""
+    N, d, D, bs, peak = 2000, 64, 64, 64, 1500
+    g = torch.Generator().manual_seed(int(gap * 10) + N + peak)
+    B, H = 1, 2
+    scale = 1.0 / np.sqrt(d)
+    u = torch.randn(d, generator=g)
+    q = (u + 0.3 * torch.randn(B, H, N, d, generator=g)).to(torch.bfloat16)
+    k = 0.5 * torch.randn(B, H, N, d, generator=g)
+    k[:, :, peak] = gap / (scale * float(u @ u)) * u
+    k = k.to(torch.bfloat16)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    nb = -(-N // bs)
+    rp, ci = _csr_with_block(B * H, nb, nb // 4, seed=N + peak, block=peak // bs)
+    dq, dk, dv = (x.to(cuda_device) for x in (q, k, v))
+    out, st = usa.rt_attn_full_capture(dq, dk, dv, head_dim=d, block_size=bs, scale=scale, compressed=True,
+                                       row_ptr=to_dev(rp, cuda_device), col_idx=to_dev(ci, cuda_device))
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    orc = oracle.full_capture(q, k, v, d, bs, scale, rp, ci)
+    orc_abs = oracle.full_capture(q, k, v.abs(), d, bs, scale, rp, ci)["u"]
+    compare_out(out.reshape(-1, D), orc["o"], d, f"peak gap {gap:g}: capture O (compressed)")
+    compare_stats(_decoded(st), np.arange(B * H * N), orc, orc_abs, d, f"peak gap {gap:g}: stats (compressed)")

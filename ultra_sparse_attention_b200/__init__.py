@@ -86,6 +86,10 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
             sz = ctypes.c_size_t
             lib.rt_attn_full_capture.argtypes = [shp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
             lib.rt_attn_sparse_reshape.argtypes = [shp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            lib.rt_attn_full_capture_u16.argtypes = [shp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                                     vp]
+            lib.rt_attn_sparse_reshape_u16.argtypes = [shp, vp, vp, vp, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                                       vp]
             lib.rt_pair_query_blocks.argtypes = [shp, vp, vp, vp, vp, sz, vp]
             lib.rt_workspace_bytes.argtypes = [shp, ctypes.POINTER(sz), ctypes.POINTER(sz)]
             lib.rt_status_string.argtypes = [ctypes.c_int]
@@ -97,6 +101,7 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.rt_build_block_mask_static.argtypes = [shp, vp, vp, f32, i32, i32, vp, vp, vp, vp]
             lib.rt_build_block_mask_static.restype = ctypes.c_int
             for fn in ("rt_build_block_mask", "rt_attn_full_capture", "rt_attn_sparse_reshape",
+                       "rt_attn_full_capture_u16", "rt_attn_sparse_reshape_u16",
                        "rt_pair_query_blocks", "rt_workspace_bytes", "rt_take_device_error",
                        "rt_selftest_wait_timeout"):
                 getattr(lib, fn).restype = ctypes.c_int
@@ -114,12 +119,24 @@ def rt_abi_version() -> int:
 
 @dataclass
 class Stats:
-    """Statistics cache of a capture step (fp32, device)."""
+    """Statistics cache of a capture step (device).
+
+    ``u`` is fp32, or f16 for the compressed cache, where the residual numerator is
+    ``u * u_scale[..., None]`` with one power-of-two scale per row."""
 
     m: torch.Tensor       # [B, H, N]   row max of the scaled scores
     zfull: torch.Tensor   # [B, H, N]   full softmax denominator
     zkept: torch.Tensor   # [B, H, N]   kept-key part of it
-    u: torch.Tensor       # [B, H, N, D] masked-out residual numerator
+    u: torch.Tensor       # [B, H, N, D] masked-out residual numerator (fp32, or f16 with u_scale)
+    u_scale: torch.Tensor | None = None  # [B, H, N] fp32, compressed cache only
+
+    @property
+    def compressed(self) -> bool:
+        return self.u.dtype == torch.float16
+
+    def residual(self) -> torch.Tensor:
+        """U as fp32 [B, H, N, D] (decoded from the compressed form if needed)."""
+        return self.u.float() * self.u_scale[..., None] if self.compressed else self.u
 
 
 def _ptr(t: torch.Tensor | None):
@@ -167,7 +184,11 @@ def _check_stats(name: str, st: "Stats", dims, device: torch.device):
     B, H, N, D = dims
     for what, t in (("stats.m", st.m), ("stats.zfull", st.zfull), ("stats.zkept", st.zkept)):
         _check_buf(name, what, t, torch.float32, device, shape=(B, H, N))
-    _check_buf(name, "stats.u", st.u, torch.float32, device, shape=(B, H, N, D))
+    if isinstance(st.u, torch.Tensor) and st.u.dtype == torch.float16:
+        _check_buf(name, "stats.u", st.u, torch.float16, device, shape=(B, H, N, D))
+        _check_buf(name, "stats.u_scale", st.u_scale, torch.float32, device, shape=(B, H, N))
+    else:
+        _check_buf(name, "stats.u", st.u, torch.float32, device, shape=(B, H, N, D))
 
 
 def _shape(dims, head_dim: int, block_size: int) -> RtShape:
@@ -215,11 +236,13 @@ def rt_build_block_mask(q: torch.Tensor, k: torch.Tensor, *, head_dim: int, bloc
 def rt_attn_full_capture(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, head_dim: int, block_size: int,
                          scale: float, row_ptr: torch.Tensor, col_idx: torch.Tensor,
                          out: torch.Tensor | None = None, stats: Stats | None = None,
-                         workspace: torch.Tensor | None = None, stream=None):
+                         workspace: torch.Tensor | None = None, compressed: bool = False, stream=None):
     """Full attention at a capture step plus the statistics cache.  Returns (out, stats).
 
-    ``workspace`` (uint8, device, at least rt_workspace_bytes(...)[0] bytes) keeps the
-    library from taking a transient buffer from its pool."""
+    ``compressed`` (or a ``stats`` whose ``u`` is f16) writes the compressed cache
+    (rt_attn_full_capture_u16).  ``workspace`` (uint8, device, at least
+    rt_workspace_bytes(...)[0] bytes) keeps the library from taking a transient
+    buffer from its pool."""
     name = "rt_attn_full_capture"
     dims = _check_qkv(name, q, k, v)
     B, H, N, D = dims
@@ -227,10 +250,9 @@ def rt_attn_full_capture(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, h
     if out is None:
         out = torch.empty_like(q)
     if stats is None:
-        stats = Stats(torch.empty(B, H, N, dtype=torch.float32, device=dev),
-                      torch.empty(B, H, N, dtype=torch.float32, device=dev),
-                      torch.empty(B, H, N, dtype=torch.float32, device=dev),
-                      torch.empty(B, H, N, D, dtype=torch.float32, device=dev))
+        f = lambda *shp, dt=torch.float32: torch.empty(*shp, dtype=dt, device=dev)
+        stats = (Stats(f(B, H, N), f(B, H, N), f(B, H, N), f(B, H, N, D, dt=torch.float16), f(B, H, N))
+                 if compressed else Stats(f(B, H, N), f(B, H, N), f(B, H, N), f(B, H, N, D)))
     _check_buf(name, "out", out, torch.bfloat16, dev, shape=dims)
     _check_stats(name, stats, dims, dev)
     _check_buf(name, "row_ptr", row_ptr, torch.int32, dev)
@@ -238,12 +260,16 @@ def rt_attn_full_capture(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, h
     if workspace is not None:
         _check_buf(name, "workspace", workspace, torch.uint8, dev)
     shape = _shape(dims, head_dim, block_size)
+    lib = load_library()
     with torch.cuda.device(dev):
-        _call(load_library().rt_attn_full_capture(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale),
-                                                  _ptr(row_ptr), _ptr(col_idx), _ptr(out), _ptr(stats.m),
-                                                  _ptr(stats.zfull), _ptr(stats.zkept), _ptr(stats.u),
-                                                  _ptr(workspace), _nbytes(workspace), _stream_handle(dev, stream)),
-              name)
+        head = (ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale), _ptr(row_ptr), _ptr(col_idx),
+                _ptr(out), _ptr(stats.m), _ptr(stats.zfull), _ptr(stats.zkept))
+        tail = (_ptr(workspace), _nbytes(workspace), _stream_handle(dev, stream))
+        if stats.compressed:
+            _call(lib.rt_attn_full_capture_u16(*head, _ptr(stats.u), _ptr(stats.u_scale), *tail),
+                  "rt_attn_full_capture_u16")
+        else:
+            _call(lib.rt_attn_full_capture(*head, _ptr(stats.u), *tail), name)
     return out, stats
 
 
@@ -269,12 +295,17 @@ def rt_attn_sparse_reshape(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
     _check_buf(name, "col_idx", col_idx, torch.int32, dev)
     shape = _shape(dims, head_dim, block_size)
     s = stats
+    lib = load_library()
     with torch.cuda.device(dev):
-        _call(load_library().rt_attn_sparse_reshape(
-            ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale), _ptr(row_ptr), _ptr(col_idx),
-            _ptr(tile_blocks), _ptr(s.m if s else None), _ptr(s.zfull if s else None), _ptr(s.zkept if s else None),
-            _ptr(s.u if s else None), _ptr(out), _stream_handle(dev, stream)),
-            name)
+        head = (ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale), _ptr(row_ptr), _ptr(col_idx),
+                _ptr(tile_blocks), _ptr(s.m if s else None), _ptr(s.zfull if s else None),
+                _ptr(s.zkept if s else None))
+        if s is not None and s.compressed:
+            _call(lib.rt_attn_sparse_reshape_u16(*head, _ptr(s.u), _ptr(s.u_scale), _ptr(out),
+                                                 _stream_handle(dev, stream)), "rt_attn_sparse_reshape_u16")
+        else:
+            _call(lib.rt_attn_sparse_reshape(*head, _ptr(s.u if s else None), _ptr(out), _stream_handle(dev, stream)),
+                  name)
     return out
 
 

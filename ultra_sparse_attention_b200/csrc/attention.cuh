@@ -90,11 +90,16 @@ struct AttnArgs {
   const float* stat_zfull;
   const float* stat_zkept;
   const float* stat_u;
+  // compressed cache: U as f16 bits [B*H, N, D] times a per-row power of two (fp32 [B*H, N])
+  const uint16_t* stat_u16;
+  const float* stat_u_scale;
   // capture step: statistics out
   float* out_m;
   float* out_zfull;
   float* out_zkept;
   float* out_u;
+  uint16_t* out_u16;     // compressed cache out (instead of out_u)
+  float* out_u_scale;
   __nv_bfloat16* out;
   // sparse step: the query blocks of each 128-row tile, int32 [B*H][n_tiles][2]
   // (-1: empty half); null = the neighbouring blocks
@@ -390,7 +395,7 @@ __host__ __device__ constexpr size_t sparse_smem_bytes(int N) {
   return 1024 + SparseLayout<D>::kOffLists + SparseLayout<D>::kNL * 2 * tile_list_cap(N) + sizeof(SparseShared);
 }
 
-template <int D, int BS>
+template <int D, int BS, bool kU16>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     sparse_reshape_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tq_tail,
                           const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tk_tail,
@@ -659,6 +664,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const int grp = r / BS;
     const float C = a.scale_log2;
     const uint64_t C2 = f2_pack(C, C);
+    constexpr int kUBytes = kU16 ? D * 2 : D * 4;  // one cached U row
     // Prefetch into L2 the row of U that the epilogue of tile i reads.
     auto prefetch_u = [&](int i) {
       if (!has_stats || i >= n_mine) return;
@@ -666,17 +672,19 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       const int row = qb * BS + r % BS;
       if (qb < 0 || row >= a.N) return;
       const size_t rg = static_cast<size_t>(bh) * a.N + row;
-      const unsigned char* u = reinterpret_cast<const unsigned char*>(a.stat_u + rg * D);
+      const unsigned char* u = kU16 ? reinterpret_cast<const unsigned char*>(a.stat_u16 + rg * D)
+                                    : reinterpret_cast<const unsigned char*>(a.stat_u + rg * D);
 #pragma unroll
-      for (int off = 0; off < D * 4; off += 128) prefetch_l2(u + off);
-      prefetch_l2(u + D * 4 - 4);
+      for (int off = 0; off < kUBytes; off += 128) prefetch_l2(u + off);
+      prefetch_l2(u + kUBytes - 4);
     };
-    // This row's cached m, Z_full and Z_kept for tile i, read a tile ahead into registers
-    // (the neutral 0, 1, 1 for rows past N or without statistics).
-    auto load_stats = [&](int i, float& m, float& zf, float& zk) {
+    // This row's cached m, Z_full, Z_kept (and U's scale) for tile i, read a tile ahead into
+    // registers (the neutral 0, 1, 1, 1 for rows past N or without statistics).
+    auto load_stats = [&](int i, float& m, float& zf, float& zk, float& us) {
       m = 0.f;
       zf = 1.f;
       zk = 1.f;
+      us = 1.f;
       if (!has_stats || i >= n_mine) return;
       const int t = tile_of(i), bh = t / n_qt, qb = tile_query_block<BS>(a, n_qt, bh, t % n_qt, r / BS);
       const int row = qb * BS + r % BS;
@@ -685,10 +693,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       m = __ldg(a.stat_m + rg);
       zf = __ldg(a.stat_zfull + rg);
       zk = __ldg(a.stat_zkept + rg);
+      if constexpr (kU16) us = __ldg(a.stat_u_scale + rg);
     };
     prefetch_u(0);
-    float next_m, next_zf, next_zk;
-    load_stats(0, next_m, next_zf, next_zk);
+    float next_m, next_zf, next_zk, next_us;
+    load_stats(0, next_m, next_zf, next_zk, next_us);
     int g = 0, e = 0;
     for (int i = 0; i < n_mine; ++i) {
       prefetch_u(i + 1);
@@ -697,8 +706,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       const int row = qb * BS + r % BS;
       const bool valid = qb >= 0 && row < a.N;
       const size_t row_g = static_cast<size_t>(bh) * a.N + (valid ? row : 0);
-      const float mc2 = next_m * kLog2e, zf_c = next_zf, zk_c = next_zk;
-      load_stats(i + 1, next_m, next_zf, next_zk);
+      const float mc2 = next_m * kLog2e, zf_c = next_zf, zk_c = next_zk, us_c = next_us;
+      load_stats(i + 1, next_m, next_zf, next_zk, next_us);
       float m_run = has_stats ? mc2 : -INFINITY;
       const int lb = i % NL;
       if (!warp_wait(&sh.list_full[lb], (i / NL) & 1, abort_flag)) break;
@@ -774,20 +783,31 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       constexpr int kUPre = D <= 80 ? D : 64;
       const bool has_u = has_stats && valid;
       const float4* up = reinterpret_cast<const float4*>(a.stat_u + row_g * D);
+      const uint4* up16 = reinterpret_cast<const uint4*>(a.stat_u16 + row_g * D);
       float u[kUPre];
 #pragma unroll
       for (int c = 0; c < kUPre; ++c) u[c] = 0.f;
       float fu = 0.f;
       if (has_u) {
+        if constexpr (kU16) {
 #pragma unroll
-        for (int q4 = 0; q4 < kUPre / 4; ++q4) {
-          const float4 x = __ldg(up + q4);
-          u[4 * q4 + 0] = x.x;
-          u[4 * q4 + 1] = x.y;
-          u[4 * q4 + 2] = x.z;
-          u[4 * q4 + 3] = x.w;
+          for (int q8 = 0; q8 < kUPre / 8; ++q8) {
+            const uint4 x = __ldg(up16 + q8);
+            const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) f16x2_to_f32(w4[h], u[8 * q8 + 2 * h], u[8 * q8 + 2 * h + 1]);
+          }
+        } else {
+#pragma unroll
+          for (int q4 = 0; q4 < kUPre / 4; ++q4) {
+            const float4 x = __ldg(up + q4);
+            u[4 * q4 + 0] = x.x;
+            u[4 * q4 + 1] = x.y;
+            u[4 * q4 + 2] = x.z;
+            u[4 * q4 + 3] = x.w;
+          }
         }
-        fu = ex2_approx(mc2 - m_run);
+        fu = ex2_approx(mc2 - m_run) * us_c;  // us_c: U's power-of-two scale (1 for fp32 U)
       }
       const float denom = has_stats ? z * (zf_c / zk_c) : z;
       const float inv = z > 0.f ? 1.f / denom : 0.f;
@@ -814,6 +834,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         if (c0 < kUPre) {
 #pragma unroll
           for (int c = 0; c < 16; ++c) uc[c] = u[(c0 < kUPre ? c0 : 0) + c];
+        } else if constexpr (kU16) {
+#pragma unroll
+          for (int q8 = 0; q8 < 2; ++q8) {
+            const uint4 x = has_u ? __ldg(up16 + c0 / 8 + q8) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) f16x2_to_f32(w4[h], uc[8 * q8 + 2 * h], uc[8 * q8 + 2 * h + 1]);
+          }
         } else {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
@@ -934,7 +962,7 @@ __device__ __forceinline__ void issue_pv_ss(uint32_t acc_tmem, uint32_t p_base, 
   }
 }
 
-template <int D, int BS>
+template <int D, int BS, bool kU16>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     full_capture_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tq_tail,
                         const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tk_tail,
@@ -1189,7 +1217,27 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       const float adju = ex2_approx(m_u - kPBias - M);
       const float zkept = zk * adjk, zfull = zkept + zm * adju;
       const float inv = zfull > 0.f ? unscale / zfull : 0.f;
-      const float adj = adju * unscale;
+      float adj = adju * unscale;
+      float u_scale = 1.f;
+      if constexpr (kU16) {
+        // Compressed cache: the row's U as f16 times a power of two 2^-k, with k chosen so
+        // that the row's largest |U| lands in [2^14, 2^15) (11 mantissa bits for every
+        // element down to 2^-28 of it).  First pass: the row's largest |U|.
+        float umax = 0.f;
+        if (ou_any) {
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 16) {
+            float ouv[16];
+            tmem_ld16(tmem + lane_off + L::kOUCol + c0, ouv);
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              if (c0 + c < a.d) umax = fmaxf(umax, fabsf(ouv[c]));
+          }
+        }
+        const int k = v_scale_exp(__float_as_uint(umax * adj));
+        u_scale = exp2_int(-k);
+        adj *= exp2_int(k);
+      }
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 16) {
         float okv[16], ouv[16];
@@ -1218,12 +1266,23 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           uint4* dst = reinterpret_cast<uint4*>(a.out + row_g * D + c0);
           dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
           dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          float4* ud = reinterpret_cast<float4*>(a.out_u + row_g * D + c0);
+          if constexpr (kU16) {
+            uint32_t h[8];
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) ud[q4] = make_float4(uo[4 * q4], uo[4 * q4 + 1], uo[4 * q4 + 2], uo[4 * q4 + 3]);
+            for (int c = 0; c < 16; c += 2) h[c / 2] = pack_f16x2(uo[c], uo[c + 1]);
+            uint4* ud = reinterpret_cast<uint4*>(a.out_u16 + row_g * D + c0);
+            ud[0] = make_uint4(h[0], h[1], h[2], h[3]);
+            ud[1] = make_uint4(h[4], h[5], h[6], h[7]);
+          } else {
+            float4* ud = reinterpret_cast<float4*>(a.out_u + row_g * D + c0);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              ud[q4] = make_float4(uo[4 * q4], uo[4 * q4 + 1], uo[4 * q4 + 2], uo[4 * q4 + 3]);
+          }
         }
       }
       if (valid) {  // the sums carry no V scale
+        if constexpr (kU16) a.out_u_scale[row_g] = u_scale;
         a.out_m[row_g] = M * kLn2;
         a.out_zfull[row_g] = zfull;
         a.out_zkept[row_g] = zkept;

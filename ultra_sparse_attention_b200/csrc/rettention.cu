@@ -177,47 +177,53 @@ bool set_smem(K kernel, size_t smem) {
                               static_cast<int>(cudaSharedmemCarveoutMaxShared)) == cudaSuccess;
 }
 
-template <int D, int BS>
+template <int D, int BS, bool kU16>
 rt_status launch_sparse(const Dims& d, const Maps& m, const AttnArgs& a, cudaStream_t stream) {
   // One persistent kernel; it builds each query tile's key-tile list from the CSR itself.
   const int N = static_cast<int>(d.N);
   const int64_t tiles = rt::query_tiles(N) * d.bh;
   const size_t smem = rt::sparse_smem_bytes<D>(N);
-  auto kernel = rt::sparse_reshape_kernel<D, BS>;
+  auto kernel = rt::sparse_reshape_kernel<D, BS, kU16>;
   if (!set_smem(kernel, smem)) return RT_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, 2 * sm_count()));
   kernel<<<grid, rt::kAttnThreads, smem, stream>>>(m.q, m.q_tail, m.k, m.k_tail, m.v, m.v_tail, m.o, m.o_tail, a);
   return launch_status();
 }
 
-template <int D, int BS>
+template <int D, int BS, bool kU16>
 rt_status launch_capture(const Dims& d, const Maps& m, const AttnArgs& a, cudaStream_t stream) {
   const size_t smem = rt::capture_smem_bytes<D>(static_cast<int>(d.n_blocks));
-  auto kernel = rt::full_capture_kernel<D, BS>;
+  auto kernel = rt::full_capture_kernel<D, BS, kU16>;
   if (!set_smem(kernel, smem)) return RT_ERR_CUDA;
   dim3 grid(static_cast<unsigned>(rt::query_tiles(static_cast<int>(d.N))), static_cast<unsigned>(d.bh));
   kernel<<<grid, rt::kAttnThreads, smem, stream>>>(m.q, m.q_tail, m.k, m.k_tail, m.v, m.v_tail, a);
   return launch_status();
 }
 
-template <bool kCapture>
-rt_status dispatch_attention(const Dims& d, const Maps& m, const AttnArgs& a, cudaStream_t s) {
+template <bool kCapture, bool kU16>
+rt_status dispatch_attention_u(const Dims& d, const Maps& m, const AttnArgs& a, cudaStream_t s) {
   if (kCapture) {
-    if (d.D == 64 && d.bs == 64) return launch_capture<64, 64>(d, m, a, s);
-    if (d.D == 64 && d.bs == 128) return launch_capture<64, 128>(d, m, a, s);
-    if (d.D == 80 && d.bs == 64) return launch_capture<80, 64>(d, m, a, s);
-    if (d.D == 80 && d.bs == 128) return launch_capture<80, 128>(d, m, a, s);
-    if (d.D == 128 && d.bs == 64) return launch_capture<128, 64>(d, m, a, s);
-    if (d.D == 128 && d.bs == 128) return launch_capture<128, 128>(d, m, a, s);
+    if (d.D == 64 && d.bs == 64) return launch_capture<64, 64, kU16>(d, m, a, s);
+    if (d.D == 64 && d.bs == 128) return launch_capture<64, 128, kU16>(d, m, a, s);
+    if (d.D == 80 && d.bs == 64) return launch_capture<80, 64, kU16>(d, m, a, s);
+    if (d.D == 80 && d.bs == 128) return launch_capture<80, 128, kU16>(d, m, a, s);
+    if (d.D == 128 && d.bs == 64) return launch_capture<128, 64, kU16>(d, m, a, s);
+    if (d.D == 128 && d.bs == 128) return launch_capture<128, 128, kU16>(d, m, a, s);
   } else {
-    if (d.D == 64 && d.bs == 64) return launch_sparse<64, 64>(d, m, a, s);
-    if (d.D == 64 && d.bs == 128) return launch_sparse<64, 128>(d, m, a, s);
-    if (d.D == 80 && d.bs == 64) return launch_sparse<80, 64>(d, m, a, s);
-    if (d.D == 80 && d.bs == 128) return launch_sparse<80, 128>(d, m, a, s);
-    if (d.D == 128 && d.bs == 64) return launch_sparse<128, 64>(d, m, a, s);
-    if (d.D == 128 && d.bs == 128) return launch_sparse<128, 128>(d, m, a, s);
+    if (d.D == 64 && d.bs == 64) return launch_sparse<64, 64, kU16>(d, m, a, s);
+    if (d.D == 64 && d.bs == 128) return launch_sparse<64, 128, kU16>(d, m, a, s);
+    if (d.D == 80 && d.bs == 64) return launch_sparse<80, 64, kU16>(d, m, a, s);
+    if (d.D == 80 && d.bs == 128) return launch_sparse<80, 128, kU16>(d, m, a, s);
+    if (d.D == 128 && d.bs == 64) return launch_sparse<128, 64, kU16>(d, m, a, s);
+    if (d.D == 128 && d.bs == 128) return launch_sparse<128, 128, kU16>(d, m, a, s);
   }
   return RT_ERR_UNSUPPORTED;
+}
+
+// kU16: the residual numerator U is cached as f16 with a per-row power-of-two scale.
+template <bool kCapture>
+rt_status dispatch_attention(const Dims& d, const Maps& m, const AttnArgs& a, bool u16, cudaStream_t s) {
+  return u16 ? dispatch_attention_u<kCapture, true>(d, m, a, s) : dispatch_attention_u<kCapture, false>(d, m, a, s);
 }
 
 // ------------------------------------------------------------------ mask launch
@@ -324,6 +330,118 @@ size_t pairing_workspace_bytes(const Dims& d) {
   return d.bs == 64 ? static_cast<size_t>(d.bh) * d.n_blocks * rt::kPairCands * 2 : 0;
 }
 
+// The capture call behind rt_attn_full_capture (fp32 U) and rt_attn_full_capture_u16
+// (f16 U with a per-row scale): exactly one of stat_u and stat_u16 is non-null.
+rt_status full_capture_impl(const rt_shape* shape, const void* q, const void* k, const void* v, float scale,
+                            const int32_t* row_ptr, const int32_t* col_idx, void* out, float* stat_m,
+                            float* stat_zfull, float* stat_zkept, float* stat_u, uint16_t* stat_u16,
+                            float* stat_u_scale, bool u16, void* workspace, size_t workspace_bytes,
+                            cudaStream_t s) {
+  Dims d;
+  rt_status st = check_shape(shape, &d);
+  if (st != RT_OK) return st;
+  if (!q || !k || !v || !row_ptr || !col_idx || !out || !stat_m || !stat_zfull || !stat_zkept)
+    return RT_ERR_INVALID_ARGUMENT;
+  if (u16 ? (!stat_u16 || !stat_u_scale) : !stat_u) return RT_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(stat_u, 16) ||
+      !aligned(stat_u16, 16) || !aligned(stat_u_scale, 4) || !aligned(row_ptr, 4) || !aligned(col_idx, 4) ||
+      !aligned(stat_m, 4) || !aligned(stat_zfull, 4) || !aligned(stat_zkept, 4))
+    return RT_ERR_INVALID_ARGUMENT;
+  if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
+  if (workspace && (!aligned(workspace, 16) || workspace_bytes < capture_workspace_bytes(d)))
+    return RT_ERR_INVALID_ARGUMENT;
+  // The PV products run on f16 P and an f16 copy of V scaled per head by a power of two
+  // (workspace: the copy, then the per-head max |v|; the caller's, or from the pool).
+  const size_t per_head8 = static_cast<size_t>(d.N) * d.D / 8;  // D is a multiple of 16
+  const size_t v16_bytes = static_cast<size_t>(d.bh) * per_head8 * 16;
+  const bool own = workspace == nullptr;
+  void* ws = workspace;
+  if (own && !workspace_alloc(&ws, capture_workspace_bytes(d), s)) return RT_ERR_CUDA;
+  void* v16 = ws;
+  uint32_t* amax = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + v16_bytes);
+  Maps m;
+  if (!make_maps(&m, d, q, k, v16, out, rt::kBM, true)) {
+    if (own) cudaFreeAsync(ws, s);
+    return RT_ERR_CUDA;
+  }
+  const size_t per_head_blocks = (per_head8 + 255) / 256;
+  const size_t want = (8 * static_cast<size_t>(sm_count()) + d.bh - 1) / d.bh;
+  const dim3 cgrid(static_cast<unsigned>(std::max<size_t>(1, std::min(per_head_blocks, want))),
+                   static_cast<unsigned>(d.bh));
+  st = cudaMemsetAsync(amax, 0, static_cast<size_t>(d.bh) * 4, s) == cudaSuccess ? RT_OK : RT_ERR_CUDA;
+  if (st == RT_OK) {
+    rt::v_absmax_kernel<<<cgrid, 256, 0, s>>>(static_cast<const uint4*>(v), per_head8, amax);
+    st = launch_status();
+  }
+  if (st == RT_OK) {
+    rt::convert_v_f16_kernel<<<cgrid, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16),
+                                                   per_head8, amax);
+    st = launch_status();
+  }
+  AttnArgs a{};
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.v_amax = amax;
+  a.out_m = stat_m;
+  a.out_zfull = stat_zfull;
+  a.out_zkept = stat_zkept;
+  a.out_u = stat_u;
+  a.out_u16 = stat_u16;
+  a.out_u_scale = stat_u_scale;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.N = static_cast<int>(d.N);
+  a.d = static_cast<int>(d.d);
+  a.n_blocks = static_cast<int>(d.n_blocks);
+  a.n_heads = static_cast<int>(d.bh);
+  a.scale_log2 = scale * rt::kLog2e;
+  if (st == RT_OK) st = dispatch_attention<true>(d, m, a, u16, s);
+  if (own && cudaFreeAsync(ws, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
+  return st;
+}
+
+// The sparse call behind rt_attn_sparse_reshape and rt_attn_sparse_reshape_u16: with
+// statistics, exactly one of stat_u and stat_u16 is non-null.
+rt_status sparse_reshape_impl(const rt_shape* shape, const void* q, const void* k, const void* v, float scale,
+                              const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_blocks,
+                              const float* stat_m, const float* stat_zfull, const float* stat_zkept,
+                              const float* stat_u, const uint16_t* stat_u16, const float* stat_u_scale, bool u16,
+                              void* out, cudaStream_t s) {
+  Dims d;
+  rt_status st = check_shape(shape, &d);
+  if (st != RT_OK) return st;
+  if (!q || !k || !v || !row_ptr || !col_idx || !out) return RT_ERR_INVALID_ARGUMENT;
+  if (u16) {
+    if (!stat_m || !stat_zfull || !stat_zkept || !stat_u16 || !stat_u_scale) return RT_ERR_INVALID_ARGUMENT;
+  } else {
+    const int nstats = (stat_m != nullptr) + (stat_zfull != nullptr) + (stat_zkept != nullptr) + (stat_u != nullptr);
+    if (nstats != 0 && nstats != 4) return RT_ERR_INVALID_ARGUMENT;
+  }
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(stat_u, 16) ||
+      !aligned(stat_u16, 16) || !aligned(stat_u_scale, 4) || !aligned(row_ptr, 4) || !aligned(col_idx, 4) ||
+      !aligned(tile_blocks, 4) || !aligned(stat_m, 4) || !aligned(stat_zfull, 4) || !aligned(stat_zkept, 4))
+    return RT_ERR_INVALID_ARGUMENT;
+  if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
+  Maps m;
+  if (!make_maps(&m, d, q, k, v, out, static_cast<int>(d.bs))) return RT_ERR_CUDA;
+  AttnArgs a{};
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.tile_blocks = tile_blocks;
+  a.stat_m = stat_m;
+  a.stat_zfull = stat_zfull;
+  a.stat_zkept = stat_zkept;
+  a.stat_u = stat_u;
+  a.stat_u16 = stat_u16;
+  a.stat_u_scale = stat_u_scale;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.N = static_cast<int>(d.N);
+  a.d = static_cast<int>(d.d);
+  a.n_blocks = static_cast<int>(d.n_blocks);
+  a.n_heads = static_cast<int>(d.bh);
+  a.scale_log2 = scale * rt::kLog2e;
+  return dispatch_attention<false>(d, m, a, u16, s);
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -380,98 +498,35 @@ rt_status rt_attn_full_capture(const rt_shape* shape, const void* q, const void*
                                const int32_t* row_ptr, const int32_t* col_idx, void* out, float* stat_m,
                                float* stat_zfull, float* stat_zkept, float* stat_u, void* workspace,
                                size_t workspace_bytes, rt_stream_t stream) {
-  Dims d;
-  rt_status st = check_shape(shape, &d);
-  if (st != RT_OK) return st;
-  if (!q || !k || !v || !row_ptr || !col_idx || !out || !stat_m || !stat_zfull || !stat_zkept || !stat_u)
-    return RT_ERR_INVALID_ARGUMENT;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(stat_u, 16) ||
-      !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(stat_m, 4) || !aligned(stat_zfull, 4) ||
-      !aligned(stat_zkept, 4))
-    return RT_ERR_INVALID_ARGUMENT;
-  if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
-  if (workspace && (!aligned(workspace, 16) || workspace_bytes < capture_workspace_bytes(d)))
-    return RT_ERR_INVALID_ARGUMENT;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // The PV products run on f16 P and an f16 copy of V scaled per head by a power of two
-  // (workspace: the copy, then the per-head max |v|; the caller's, or from the pool).
-  const size_t per_head8 = static_cast<size_t>(d.N) * d.D / 8;  // D is a multiple of 16
-  const size_t v16_bytes = static_cast<size_t>(d.bh) * per_head8 * 16;
-  const bool own = workspace == nullptr;
-  void* ws = workspace;
-  if (own && !workspace_alloc(&ws, capture_workspace_bytes(d), s)) return RT_ERR_CUDA;
-  void* v16 = ws;
-  uint32_t* amax = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + v16_bytes);
-  Maps m;
-  if (!make_maps(&m, d, q, k, v16, out, rt::kBM, true)) {
-    if (own) cudaFreeAsync(ws, s);
-    return RT_ERR_CUDA;
-  }
-  const size_t per_head_blocks = (per_head8 + 255) / 256;
-  const size_t want = (8 * static_cast<size_t>(sm_count()) + d.bh - 1) / d.bh;
-  const dim3 cgrid(static_cast<unsigned>(std::max<size_t>(1, std::min(per_head_blocks, want))),
-                   static_cast<unsigned>(d.bh));
-  st = cudaMemsetAsync(amax, 0, static_cast<size_t>(d.bh) * 4, s) == cudaSuccess ? RT_OK : RT_ERR_CUDA;
-  if (st == RT_OK) {
-    rt::v_absmax_kernel<<<cgrid, 256, 0, s>>>(static_cast<const uint4*>(v), per_head8, amax);
-    st = launch_status();
-  }
-  if (st == RT_OK) {
-    rt::convert_v_f16_kernel<<<cgrid, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16),
-                                                   per_head8, amax);
-    st = launch_status();
-  }
-  AttnArgs a{};
-  a.row_ptr = row_ptr;
-  a.col_idx = col_idx;
-  a.v_amax = amax;
-  a.out_m = stat_m;
-  a.out_zfull = stat_zfull;
-  a.out_zkept = stat_zkept;
-  a.out_u = stat_u;
-  a.out = static_cast<__nv_bfloat16*>(out);
-  a.N = static_cast<int>(d.N);
-  a.d = static_cast<int>(d.d);
-  a.n_blocks = static_cast<int>(d.n_blocks);
-  a.n_heads = static_cast<int>(d.bh);
-  a.scale_log2 = scale * rt::kLog2e;
-  if (st == RT_OK) st = dispatch_attention<true>(d, m, a, s);
-  if (own && cudaFreeAsync(ws, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
-  return st;
+  return full_capture_impl(shape, q, k, v, scale, row_ptr, col_idx, out, stat_m, stat_zfull, stat_zkept, stat_u,
+                           nullptr, nullptr, false, workspace, workspace_bytes,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+rt_status rt_attn_full_capture_u16(const rt_shape* shape, const void* q, const void* k, const void* v, float scale,
+                                   const int32_t* row_ptr, const int32_t* col_idx, void* out, float* stat_m,
+                                   float* stat_zfull, float* stat_zkept, uint16_t* stat_u16, float* stat_u_scale,
+                                   void* workspace, size_t workspace_bytes, rt_stream_t stream) {
+  return full_capture_impl(shape, q, k, v, scale, row_ptr, col_idx, out, stat_m, stat_zfull, stat_zkept, nullptr,
+                           stat_u16, stat_u_scale, true, workspace, workspace_bytes,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 rt_status rt_attn_sparse_reshape(const rt_shape* shape, const void* q, const void* k, const void* v, float scale,
                                  const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_blocks,
                                  const float* stat_m, const float* stat_zfull, const float* stat_zkept,
                                  const float* stat_u, void* out, rt_stream_t stream) {
-  Dims d;
-  rt_status st = check_shape(shape, &d);
-  if (st != RT_OK) return st;
-  if (!q || !k || !v || !row_ptr || !col_idx || !out) return RT_ERR_INVALID_ARGUMENT;
-  const int nstats = (stat_m != nullptr) + (stat_zfull != nullptr) + (stat_zkept != nullptr) + (stat_u != nullptr);
-  if (nstats != 0 && nstats != 4) return RT_ERR_INVALID_ARGUMENT;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(stat_u, 16) ||
-      !aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(tile_blocks, 4) || !aligned(stat_m, 4) ||
-      !aligned(stat_zfull, 4) || !aligned(stat_zkept, 4))
-    return RT_ERR_INVALID_ARGUMENT;
-  if (!scale_ok(scale)) return RT_ERR_INVALID_ARGUMENT;
-  Maps m;
-  if (!make_maps(&m, d, q, k, v, out, static_cast<int>(d.bs))) return RT_ERR_CUDA;
-  AttnArgs a{};
-  a.row_ptr = row_ptr;
-  a.col_idx = col_idx;
-  a.tile_blocks = tile_blocks;
-  a.stat_m = stat_m;
-  a.stat_zfull = stat_zfull;
-  a.stat_zkept = stat_zkept;
-  a.stat_u = stat_u;
-  a.out = static_cast<__nv_bfloat16*>(out);
-  a.N = static_cast<int>(d.N);
-  a.d = static_cast<int>(d.d);
-  a.n_blocks = static_cast<int>(d.n_blocks);
-  a.n_heads = static_cast<int>(d.bh);
-  a.scale_log2 = scale * rt::kLog2e;
-  return dispatch_attention<false>(d, m, a, reinterpret_cast<cudaStream_t>(stream));
+  return sparse_reshape_impl(shape, q, k, v, scale, row_ptr, col_idx, tile_blocks, stat_m, stat_zfull, stat_zkept,
+                             stat_u, nullptr, nullptr, false, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+rt_status rt_attn_sparse_reshape_u16(const rt_shape* shape, const void* q, const void* k, const void* v, float scale,
+                                     const int32_t* row_ptr, const int32_t* col_idx, const int32_t* tile_blocks,
+                                     const float* stat_m, const float* stat_zfull, const float* stat_zkept,
+                                     const uint16_t* stat_u16, const float* stat_u_scale, void* out,
+                                     rt_stream_t stream) {
+  return sparse_reshape_impl(shape, q, k, v, scale, row_ptr, col_idx, tile_blocks, stat_m, stat_zfull, stat_zkept,
+                             nullptr, stat_u16, stat_u_scale, true, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
 rt_status rt_pair_query_blocks(const rt_shape* shape, const int32_t* row_ptr, const int32_t* col_idx,
