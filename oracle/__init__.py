@@ -64,8 +64,9 @@ def _load():
                                              i64, vp, vp, vp, vp, vp, ctypes.c_int]
             lib.orc_sparse_reshape.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, f64, vp, vp,
                                                vp, vp, vp, vp, vp, i64, vp, ctypes.c_int]
+            lib.orc_block_mass.argtypes = [vp, vp, i64, i64, i64, i64, i64, f64, vp, ctypes.c_int]
             for fn in ("orc_pool_blocks", "orc_block_scores", "orc_select_blocks",
-                       "orc_full_capture", "orc_sparse_reshape"):
+                       "orc_full_capture", "orc_sparse_reshape", "orc_block_mass"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -133,6 +134,27 @@ def build_block_mask(q, k, d: int, bs: int, scale: float, keep: int, forced_toke
     s = block_scores(pool_blocks(q, d, bs), pool_blocks(k, d, bs), scale)
     row_ptr, col_idx = select_blocks(s, keep, bs, forced_tokens)
     return (row_ptr, col_idx, s) if return_scores else (row_ptr, col_idx)
+
+
+def block_mass(q, k, d: int, bs: int, scale: float, threads: int | None = None) -> np.ndarray:
+    """Exact attention mass of every (query block, key block) pair: fp64 [B*H, n_blocks, n_blocks],
+    the softmax probabilities of the block's query rows summed over the key block's keys."""
+    qa, ka = _bf16_bits(q), _bf16_bits(k)
+    bh, n, dpad = qa.shape
+    nb = -(-n // bs)
+    out = np.empty((bh, nb, nb), dtype=np.float64)
+    _check(_load().orc_block_mass(_ptr(qa), _ptr(ka), bh, n, dpad, d, bs, float(scale), _ptr(out),
+                                  threads or default_threads()), "block_mass")
+    return out
+
+
+def build_block_mask_exact(q, k, d: int, bs: int, scale: float, keep: int, forced_tokens: int,
+                           return_mass: bool = False):
+    """The mask from exact block masses: the same selection rule as the pooled mask, applied to
+    block_mass instead of the pooled block scores."""
+    a = block_mass(q, k, d, bs, scale)
+    row_ptr, col_idx = select_blocks(a, keep, bs, forced_tokens)
+    return (row_ptr, col_idx, a) if return_mass else (row_ptr, col_idx)
 
 
 # --------------------------------------------------------------------------

@@ -320,3 +320,75 @@ int orc_sparse_reshape(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
     p.cm = cm; p.czf = czf; p.czk = czk; p.cu = cu; p.out = out; p.mode = 1;
     return run_parallel(&p, threads);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Exact block attention mass (pinned: rows of a query block sum to its     */
+/* token count; uniform scores give rows*cols/n; brute force against torch  */
+/* softmax in fp64 summed over the blocks).                                  */
+/* mass[bh][qb][kb] = sum over query tokens i of block qb (i < n) and key   */
+/* tokens j of block kb (j < n) of softmax_j(scale * q_i . k_j), the        */
+/* softmax taken over all n keys of row i.  Selecting the top-k of these    */
+/* per query block (orc_select_blocks) keeps the key blocks that carry the  */
+/* most attention probability in the step they are computed from.          */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    const uint16_t *q, *k;
+    int64_t bh_count, n, dpad, d, bs;
+    double scale;
+    double *mass;
+    int64_t begin, end;          /* query-block ids bh*nb + qb handled by this worker */
+    int status;
+} mass_work;
+
+static void *mass_rows(void *arg) {
+    mass_work *w = arg;
+    int64_t nb = n_blocks_of(w->n, w->bs);
+    problem p = {0};             /* for dot_qk only */
+    p.n = w->n; p.dpad = w->dpad; p.d = w->d; p.scale = w->scale;
+    double *s = malloc(sizeof(double) * (size_t)w->n);
+    if (!s) { w->status = 3; return NULL; }
+    for (int64_t r = w->begin; r < w->end; ++r) {
+        int64_t bh = r / nb, qb = r % nb;
+        double *out = w->mass + r * nb;
+        for (int64_t kb = 0; kb < nb; ++kb) out[kb] = 0.0;
+        int64_t i1 = (qb + 1) * w->bs < w->n ? (qb + 1) * w->bs : w->n;
+        for (int64_t i = qb * w->bs; i < i1; ++i) {
+            double m = -INFINITY, z = 0.0;
+            for (int64_t j = 0; j < w->n; ++j) {
+                s[j] = dot_qk(&p, w->q, bh, i, w->k, j);
+                if (s[j] > m) m = s[j];
+            }
+            for (int64_t j = 0; j < w->n; ++j) z += exp(s[j] - m);
+            for (int64_t j = 0; j < w->n; ++j) out[j / w->bs] += exp(s[j] - m) / z;
+        }
+    }
+    free(s);
+    return NULL;
+}
+
+int orc_block_mass(const uint16_t *q, const uint16_t *k, int64_t bh_count, int64_t n, int64_t dpad,
+                   int64_t d, int64_t bs, double scale, double *mass, int threads) {
+    if (!q || !k || !mass || n <= 0 || d <= 0 || dpad < d || bs <= 0 || bh_count < 0) return 1;
+    int64_t rows = bh_count * n_blocks_of(n, bs);
+    if (threads < 1) threads = 1;
+    if (threads > 256) threads = 256;
+    if (threads > rows) threads = rows > 0 ? (int)rows : 1;
+    pthread_t tid[256];
+    mass_work w[256];
+    int64_t per = (rows + threads - 1) / threads;
+    int status = 0;
+    for (int t = 0; t < threads; ++t) {
+        w[t] = (mass_work){q, k, bh_count, n, dpad, d, bs, scale, mass, 0, 0, 0};
+        w[t].begin = t * per < rows ? t * per : rows;
+        w[t].end = (t + 1) * per < rows ? (t + 1) * per : rows;
+        if (threads == 1 || pthread_create(&tid[t], NULL, mass_rows, &w[t]) != 0) {
+            mass_rows(&w[t]);
+            tid[t] = 0;
+        }
+    }
+    for (int t = 0; t < threads; ++t)
+        if (threads > 1 && tid[t]) pthread_join(tid[t], NULL);
+    for (int t = 0; t < threads; ++t)
+        if (w[t].status) status = w[t].status;
+    return status;
+}

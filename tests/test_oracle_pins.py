@@ -301,3 +301,72 @@ def test_mask_step_composes_pool_score_select():
     np.testing.assert_allclose(s, w.scale * np.einsum("bqc,bkc->bqk", x, y), rtol=1e-12, atol=1e-15)
     for r in range(16):
         assert set(ci[2 * r:2 * r + 2]) == _brute_topk(s.reshape(16, 8)[r], 2, 0)
+
+
+# ------------------------------------------------------------------ exact block masses
+def _torch_block_mass(q, k, d, bs, scale):
+    """fp64 torch softmax over all keys, summed over query and key blocks (ragged tail)."""
+    B, H, N, _ = q.shape
+    qq = q[..., :d].double().reshape(B * H, N, d)
+    kk = k[..., :d].double().reshape(B * H, N, d)
+    p = torch.softmax(scale * qq @ kk.transpose(1, 2), dim=-1)       # [BH, N, N]
+    nb = -(-N // bs)
+    blk = torch.arange(N) // bs
+    a = torch.zeros(B * H, nb, N, dtype=torch.float64).index_add_(1, blk, p)   # sum query rows
+    return torch.zeros(B * H, nb, nb, dtype=torch.float64).index_add_(2, blk, a).numpy()
+
+
+@pytest.mark.parametrize("N,d,D,bs", [(200, 64, 64, 64), (300, 72, 80, 128), (128, 16, 64, 64)])
+def test_block_mass_matches_torch_softmax(N, d, D, bs):
+    q, k, _ = _rand_qkv(2, 2, N, d, D, std=1.3, seed=N + d)
+    scale = 1.0 / math.sqrt(d)
+    got = oracle.block_mass(q, k, d, bs, scale)
+    want = _torch_block_mass(q, k, d, bs, scale)
+    assert np.max(np.abs(got - want)) <= 1e-12
+    # a transposed operand (masses of K attending to Q) is a different matrix
+    swapped = oracle.block_mass(k, q, d, bs, scale)
+    assert np.max(np.abs(swapped - got)) > 1e-3
+
+
+def test_block_mass_rows_sum_to_the_block_size():
+    """Every query token's probabilities sum to 1, so a query block's masses sum to its
+    number of real tokens (the ragged tail block to its own count)."""
+    N, bs = 1000, 64
+    q, k, _ = _rand_qkv(1, 3, N, 64, 64, std=2.0, seed=5)
+    a = oracle.block_mass(q, k, 64, bs, 0.125)
+    rows = np.minimum(bs, N - np.arange(-(-N // bs)) * bs)
+    assert np.allclose(a.sum(-1), rows[None, :], rtol=0, atol=1e-10)
+    assert np.all(a >= 0)
+
+
+def test_block_mass_uniform_scores_closed_form():
+    """Q = 0: every score is 0, each probability 1/N, so mass = rows(qb) * cols(kb) / N."""
+    N, bs = 300, 64
+    q = torch.zeros(1, 2, N, 64, dtype=torch.bfloat16)
+    _, k, _ = _rand_qkv(1, 2, N, 64, 64, seed=2)
+    a = oracle.block_mass(q, k, 64, bs, 0.125)
+    sizes = np.minimum(bs, N - np.arange(-(-N // bs)) * bs).astype(np.float64)
+    want = np.outer(sizes, sizes) / N
+    assert np.max(np.abs(a - want[None])) <= 1e-11  # 4096 fp64 additions of 1/N per entry
+
+
+def test_exact_mask_keeps_the_block_of_a_dominant_key():
+    """A key aligned with every query (a large score for all rows) puts most of each row's
+    mass in its block; with keep = 1 every query block keeps exactly that block, with keep
+    = all every block, and the selection equals select_blocks on the masses."""
+    N, d, bs = 512, 64, 64
+    g = torch.Generator().manual_seed(9)
+    u = torch.randn(d, generator=g)
+    q = torch.zeros(1, 1, N, d)
+    q[..., :] = u + 0.2 * torch.randn(1, 1, N, d, generator=g)
+    k = 0.3 * torch.randn(1, 1, N, d, generator=g)
+    k[0, 0, 333] = 0.6 * u
+    q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    rp, ci, a = oracle.build_block_mask_exact(q, k, d, bs, 0.125, 1, 0, return_mass=True)
+    assert list(ci) == [333 // bs] * (N // bs)
+    rp_s, ci_s = oracle.select_blocks(a, 1, bs, 0)
+    assert np.array_equal(ci, ci_s) and np.array_equal(rp, rp_s)
+    _, ci_all = oracle.build_block_mask_exact(q, k, d, bs, 0.125, N // bs, 0)
+    assert list(ci_all) == list(range(N // bs)) * (N // bs)
+    _, ci_f = oracle.build_block_mask_exact(q, k, d, bs, 0.125, 2, 100)  # forced blocks 0, 1
+    assert list(ci_f) == [0, 1] * (N // bs)
