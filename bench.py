@@ -442,7 +442,40 @@ def run_sweep(args, device, checker=None) -> list:
         ref_norm = torch.linalg.vector_norm(full1.float()).item()
         err_r = torch.linalg.vector_norm(resh1.float() - full1.float()).item() / ref_norm
         err_p = torch.linalg.vector_norm(plain1.float() - full1.float()).item() / ref_norm
-        del full1, resh1, plain1
+        del resh1, plain1
+        # The same cycle with the mask chosen by exact block attention mass (one extra
+        # full-attention pass at the capture step): its time and the reshape's distance to full
+        # attention, beside the pooled mask's.
+        exact = None
+        if name != "tiny" and (name != "video5b" or ratio == w.keep[0]):
+            ex_ms = []
+            for it in range(args.sweep_warmup + 3):
+                flush.zero_()
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                e[0].record(stream)
+                rpx, cix = usa.rt_build_block_mask_exact(q0, k0, v0, keep_blocks=keep,
+                                                         forced_prefix_tokens=w.forced_prefix_tokens, **kw)
+                e[1].record(stream)
+                if it >= args.sweep_warmup:
+                    ex_ms.append((e[0], e[1]))
+            tbx = usa.rt_pair_query_blocks(q0, rpx, cix, head_dim=w.head_dim, block_size=w.block_size)
+            _, stx = usa.rt_attn_full_capture(q0, k0, v0, row_ptr=rpx, col_idx=cix, **kw)
+            reshx = usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rpx, col_idx=cix, stats=stx, tile_blocks=tbx, **kw)
+            plainx = usa.rt_attn_sparse_reshape(q1, k1, v1, row_ptr=rpx, col_idx=cix, stats=None, tile_blocks=tbx,
+                                                **kw)
+            torch.cuda.synchronize()
+            if usa.rt_take_device_error() != 0:
+                raise RuntimeError(f"a kernel reported a device error in the exact-mask cycle ({name})")
+            exact = {"mask_ms": statistics.mean(a.elapsed_time(b) for a, b in ex_ms),
+                     "reshape_rel_l2_vs_full": torch.linalg.vector_norm(reshx.float() - full1.float()).item() / ref_norm,
+                     "plain_sparse_rel_l2_vs_full":
+                         torch.linalg.vector_norm(plainx.float() - full1.float()).item() / ref_norm,
+                     "kept_sets_differing_from_pooled": float((cix.view(-1, keep) != ci.view(-1, keep)).any(1)
+                                                              .float().mean().item()),
+                     "what": "rt_build_block_mask_exact (one full-attention pass, block masses, top-k) "
+                             "instead of the pooled mask; same capture and sparse kernels"}
+            del rpx, cix, tbx, stx, reshx, plainx
+        del full1
         ms = {k: statistics.mean(a.elapsed_time(b) for a, b in v) for k, v in times.items()}
         nums = workload_numbers(w, keep, rp.cpu().numpy(), ci.cpu().numpy())
         sp_s, cap_s = ms["sparse"] / 1e3, ms["capture"] / 1e3
@@ -458,6 +491,7 @@ def run_sweep(args, device, checker=None) -> list:
                     "sparse_tensor_frac_of_bf16_peak": exe / peaks["bf16_tflops"],
                     "capture_tflops": cap, "capture_frac_of_bf16_peak": cap / peaks["bf16_tflops"],
                     "reshape_rel_l2_vs_full": err_r, "plain_sparse_rel_l2_vs_full": err_p,
+                    "exact_mass_mask": exact,
                     "steps": args.sweep_steps, "warmup": args.sweep_warmup, "l2": "flushed between cycles"})
         if checker is not None:
             out[-1]["oracle_check"] = checker.check(w, keep, host0, host1, rp, ci, out0, st, out1)

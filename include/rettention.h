@@ -242,6 +242,44 @@ rt_status rt_attn_sparse_reshape_u16(const rt_shape *shape, const void *q, const
                                      const float *stat_u_scale, void *out, rt_stream_t stream);
 
 /*
+ * rt_build_block_mask_exact -- choose the kept key blocks by their exact
+ * attention mass.
+ *
+ * The Abstract reshapes the sparse scores with the softmax distribution of an
+ * earlier step; the capture step computes every score, so the mask can be
+ * chosen from that distribution itself instead of from pooled block means.
+ * For every query block qb and key block kb of a head:
+ *   mass[qb,kb] = sum over the real query rows i of qb and keys j of kb of
+ *                 exp(s_ij - m_i) / Z_full_i,   s_ij = scale * q_i . k_j
+ * (the softmax probability the block's rows give the key block, over all N
+ * keys), and kept(qb) is selected from these masses by the same rule as in
+ * rt_build_block_mask: the forced prefix blocks, then the largest masses
+ * (equal masses: lower block index first), sorted ascending.
+ *
+ * The call makes one full-attention pass over Q and K (the capture kernel
+ * with no key block kept and no output stored: the cost of about one capture
+ * step), which writes each row's per-64-key-tile log-sum-exp, then reduces
+ * those to block masses and selects.  Use the CSR with rt_attn_full_capture
+ * on the same Q, K, V to get the statistics for it.
+ *
+ * q, k, v       bf16 [B,H,N,D] device (v feeds the pass but not the masses).
+ * keep_blocks, forced_prefix_tokens, row_ptr, col_idx  as for rt_build_block_mask.
+ * block_mass    optional out (may be NULL), fp32 [B,H,n_blocks,n_blocks] device.
+ * workspace     optional (may be NULL), device, 256-byte aligned, at least
+ *               rt_exact_mask_workspace_bytes (about 4*B*H*N*(ceil(N/64) + 3)
+ *               + 2*B*H*N*D bytes: 1.07 GB for B*H = 48, N = 17776, D = 64);
+ *               NULL takes a transient buffer from the library's pool.
+ */
+rt_status rt_build_block_mask_exact(const rt_shape *shape, const void *q, const void *k,
+                                    const void *v, float scale, int32_t keep_blocks,
+                                    int32_t forced_prefix_tokens, int32_t *row_ptr,
+                                    int32_t *col_idx, float *block_mass, void *workspace,
+                                    size_t workspace_bytes, rt_stream_t stream);
+
+/* Workspace size of rt_build_block_mask_exact for a shape (validates the shape). */
+rt_status rt_exact_mask_workspace_bytes(const rt_shape *shape, size_t *bytes);
+
+/*
  * rt_pair_query_blocks -- group the query blocks of each head into the
  * sparse kernel's 128-row tiles.
  *

@@ -64,7 +64,7 @@ def _load():
                                              i64, vp, vp, vp, vp, vp, ctypes.c_int]
             lib.orc_sparse_reshape.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, f64, vp, vp,
                                                vp, vp, vp, vp, vp, i64, vp, ctypes.c_int]
-            lib.orc_block_mass.argtypes = [vp, vp, i64, i64, i64, i64, i64, f64, vp, ctypes.c_int]
+            lib.orc_block_mass.argtypes = [vp, vp, i64, i64, i64, i64, i64, f64, vp, i64, vp, ctypes.c_int]
             for fn in ("orc_pool_blocks", "orc_block_scores", "orc_select_blocks",
                        "orc_full_capture", "orc_sparse_reshape", "orc_block_mass"):
                 getattr(lib, fn).restype = ctypes.c_int
@@ -136,15 +136,18 @@ def build_block_mask(q, k, d: int, bs: int, scale: float, keep: int, forced_toke
     return (row_ptr, col_idx, s) if return_scores else (row_ptr, col_idx)
 
 
-def block_mass(q, k, d: int, bs: int, scale: float, threads: int | None = None) -> np.ndarray:
+def block_mass(q, k, d: int, bs: int, scale: float, qblocks=None, threads: int | None = None) -> np.ndarray:
     """Exact attention mass of every (query block, key block) pair: fp64 [B*H, n_blocks, n_blocks],
-    the softmax probabilities of the block's query rows summed over the key block's keys."""
+    the softmax probabilities of the block's query rows summed over the key block's keys.
+    With ``qblocks`` (global query-block ids bh*n_blocks + qb) only those rows: [len, n_blocks]."""
     qa, ka = _bf16_bits(q), _bf16_bits(k)
     bh, n, dpad = qa.shape
     nb = -(-n // bs)
-    out = np.empty((bh, nb, nb), dtype=np.float64)
-    _check(_load().orc_block_mass(_ptr(qa), _ptr(ka), bh, n, dpad, d, bs, float(scale), _ptr(out),
-                                  threads or default_threads()), "block_mass")
+    qb = None if qblocks is None else np.ascontiguousarray(qblocks, dtype=np.int64)
+    out = np.empty((bh, nb, nb) if qb is None else (qb.size, nb), dtype=np.float64)
+    _check(_load().orc_block_mass(_ptr(qa), _ptr(ka), bh, n, dpad, d, bs, float(scale), _ptr(qb),
+                                  0 if qb is None else qb.size, _ptr(out), threads or default_threads()),
+           "block_mass")
     return out
 
 
@@ -215,4 +218,54 @@ def sparse_reshape(q, k, v, d: int, bs: int, scale: float, row_ptr, col_idx, sta
                                     _ptr(rp), _ptr(ci), _ptr(cm), _ptr(czf), _ptr(czk), _ptr(cu),
                                     _ptr(r), nr, _ptr(out), threads or default_threads())
     _check(rc, "sparse_reshape")
+    return out
+
+
+# --------------------------------------------------------------------------
+# Hilbert-curve token order (HilbertA blog page, "Introducing HilbertA", first
+# component, Reordering: tokens follow a Hilbert curve over the patch grid, so
+# neighbours on the grid stay neighbours in the sequence).  Pinned by the
+# curve's defining properties: a bijection onto the cells, consecutive cells
+# 4-adjacent, each quarter of the curve filling one quadrant, the order-1 curve.
+# --------------------------------------------------------------------------
+def hilbert_curve(k: int) -> list[tuple[int, int]]:
+    """Cells (x, y) of the 2^k x 2^k grid in Hilbert order, by the recursive definition:
+    the curve of side 2s visits the lower-left quadrant along the transposed curve of side s,
+    then the upper-left and upper-right quadrants along the curve itself, then the lower-right
+    quadrant along the anti-transposed curve; it starts at (0, 0) and ends at (2s - 1, 0)."""
+    if k == 0:
+        return [(0, 0)]
+    sub = hilbert_curve(k - 1)
+    s = 1 << (k - 1)
+    return ([(y, x) for x, y in sub] +
+            [(x, y + s) for x, y in sub] +
+            [(x + s, y + s) for x, y in sub] +
+            [(2 * s - 1 - y, s - 1 - x) for x, y in sub])
+
+
+def hilbert_order(grid_h: int, grid_w: int, frames: int = 1, prefix: int = 0) -> np.ndarray:
+    """Token permutation perm (int64 [prefix + frames*grid_h*grid_w]): position t of the
+    reordered sequence holds token perm[t] of the row-major one (cell (x, y) of frame f is
+    token prefix + f*grid_h*grid_w + y*grid_w + x).  The first `prefix` tokens (text) keep
+    their place; each frame's cells follow the Hilbert curve of the smallest power-of-two
+    square that holds the grid, skipping the square's cells outside it."""
+    k = 0
+    while (1 << k) < max(grid_h, grid_w):
+        k += 1
+    cells = [y * grid_w + x for x, y in hilbert_curve(k) if x < grid_w and y < grid_h]
+    hw = grid_h * grid_w
+    order = list(range(prefix))
+    for f in range(frames):
+        order += [prefix + f * hw + c for c in cells]
+    return np.array(order, dtype=np.int64)
+
+
+def permute_tokens(x, perm, inverse: bool = False):
+    """Reordered copy of a [B, H, N, D] tensor: out[..., t, :] = x[..., perm[t], :], or the
+    inverse, out[..., perm[t], :] = x[..., t, :]."""
+    p = torch.as_tensor(np.asarray(perm, dtype=np.int64))
+    if not inverse:
+        return x[..., p, :].clone()
+    out = torch.empty_like(x)
+    out[..., p, :] = x
     return out

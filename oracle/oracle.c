@@ -336,7 +336,8 @@ typedef struct {
     int64_t bh_count, n, dpad, d, bs;
     double scale;
     double *mass;
-    int64_t begin, end;          /* query-block ids bh*nb + qb handled by this worker */
+    const int64_t *qblocks;      /* listed query-block ids bh*nb + qb; NULL = all */
+    int64_t begin, end;          /* slots handled by this worker */
     int status;
 } mass_work;
 
@@ -347,9 +348,11 @@ static void *mass_rows(void *arg) {
     p.n = w->n; p.dpad = w->dpad; p.d = w->d; p.scale = w->scale;
     double *s = malloc(sizeof(double) * (size_t)w->n);
     if (!s) { w->status = 3; return NULL; }
-    for (int64_t r = w->begin; r < w->end; ++r) {
+    for (int64_t slot = w->begin; slot < w->end; ++slot) {
+        int64_t r = w->qblocks ? w->qblocks[slot] : slot;
+        if (r < 0 || r >= w->bh_count * nb) { w->status = 5; continue; }
         int64_t bh = r / nb, qb = r % nb;
-        double *out = w->mass + r * nb;
+        double *out = w->mass + slot * nb;
         for (int64_t kb = 0; kb < nb; ++kb) out[kb] = 0.0;
         int64_t i1 = (qb + 1) * w->bs < w->n ? (qb + 1) * w->bs : w->n;
         for (int64_t i = qb * w->bs; i < i1; ++i) {
@@ -366,10 +369,12 @@ static void *mass_rows(void *arg) {
     return NULL;
 }
 
+/* mass is [nq][nb] for the listed query blocks (qblocks), [bh*nb][nb] when qblocks is NULL. */
 int orc_block_mass(const uint16_t *q, const uint16_t *k, int64_t bh_count, int64_t n, int64_t dpad,
-                   int64_t d, int64_t bs, double scale, double *mass, int threads) {
-    if (!q || !k || !mass || n <= 0 || d <= 0 || dpad < d || bs <= 0 || bh_count < 0) return 1;
-    int64_t rows = bh_count * n_blocks_of(n, bs);
+                   int64_t d, int64_t bs, double scale, const int64_t *qblocks, int64_t nq, double *mass,
+                   int threads) {
+    if (!q || !k || !mass || n <= 0 || d <= 0 || dpad < d || bs <= 0 || bh_count < 0 || nq < 0) return 1;
+    int64_t rows = qblocks ? nq : bh_count * n_blocks_of(n, bs);
     if (threads < 1) threads = 1;
     if (threads > 256) threads = 256;
     if (threads > rows) threads = rows > 0 ? (int)rows : 1;
@@ -378,7 +383,7 @@ int orc_block_mass(const uint16_t *q, const uint16_t *k, int64_t bh_count, int64
     int64_t per = (rows + threads - 1) / threads;
     int status = 0;
     for (int t = 0; t < threads; ++t) {
-        w[t] = (mass_work){q, k, bh_count, n, dpad, d, bs, scale, mass, 0, 0, 0};
+        w[t] = (mass_work){q, k, bh_count, n, dpad, d, bs, scale, mass, qblocks, 0, 0, 0};
         w[t].begin = t * per < rows ? t * per : rows;
         w[t].end = (t + 1) * per < rows ? (t + 1) * per : rows;
         if (threads == 1 || pthread_create(&tid[t], NULL, mass_rows, &w[t]) != 0) {

@@ -170,3 +170,27 @@ def test_compressed_cache_argument_validation():
     assert sp16(stats=(A16, A16, A16, A4, A16)) == usa.RT_ERR_INVALID_ARGUMENT
     assert sp16(out=None) == usa.RT_ERR_INVALID_ARGUMENT
     assert sp16(shape=RtShape(2, 3, 1000, 72, 80, 32)) == usa.RT_ERR_UNSUPPORTED
+
+
+def test_exact_mask_argument_validation():
+    lib = usa.load_library()
+    ok = RtShape(1, 2, 512, 64, 64, 64)
+
+    def ex(shape=ok, q=A16, v=A16, keep=2, forced=0, rp=A16, mass=None, ws=None, ws_bytes=0, scale=0.125):
+        return lib.rt_build_block_mask_exact(ctypes.byref(shape), q, A16, v, scale, keep, forced, rp, A16, mass, ws,
+                                             ws_bytes, None)
+
+    n = ctypes.c_size_t(0)
+    assert lib.rt_exact_mask_workspace_bytes(ctypes.byref(ok), ctypes.byref(n)) == usa.RT_OK
+    assert n.value >= 2 * 512 * 8 * 4  # at least the per-tile log-sum-exps
+    assert ex(v=None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert ex(q=MIS) == usa.RT_ERR_INVALID_ARGUMENT
+    assert ex(rp=None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert ex(mass=MIS) == usa.RT_ERR_INVALID_ARGUMENT
+    assert ex(keep=0) == usa.RT_ERR_INVALID_ARGUMENT
+    assert ex(keep=9) == usa.RT_ERR_INVALID_ARGUMENT
+    assert ex(keep=1, forced=65) == usa.RT_ERR_INVALID_ARGUMENT
+    assert ex(scale=float("inf")) == usa.RT_ERR_INVALID_ARGUMENT
+    assert ex(ws=ctypes.c_void_p(0x10010), ws_bytes=n.value) == usa.RT_ERR_INVALID_ARGUMENT  # 256-byte alignment
+    assert ex(ws=ctypes.c_void_p(0x10000), ws_bytes=n.value - 1) == usa.RT_ERR_INVALID_ARGUMENT
+    assert ex(shape=RtShape(1, 2, 512, 64, 64, 32)) == usa.RT_ERR_UNSUPPORTED

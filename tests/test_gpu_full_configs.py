@@ -213,3 +213,54 @@ def test_whole_head_matches_oracle(cuda_device, name):
     compare_stats(st, rows, orc, orc_abs, d, f"{name} head {head} capture stats")
     want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp_h, ci_h, orc, rows=rows)
     compare_out(out1.reshape(-1, D)[sel], want, d, f"{name} head {head} sparse O")
+
+
+# ------------------------------------------------------------------ mask from exact block masses, full size
+@pytest.mark.parametrize("name", ["image", "video2b", "video5b", "long"])
+def test_full_size_exact_mask_cycle(cuda_device, name):
+    """The exact-mass mask at full size: masses and kept sets of sampled query blocks against
+    the oracle, then a capture + sparse cycle with that mask on sampled rows; the reshaped
+    step must stay much closer to full attention than plain sparse attention with the same
+    mask."""
+    w, h0, h1 = _host_inputs(name)
+    d, bs, D = w.head_dim, w.block_size, w.head_dim_padded
+    bh, N, nb = w.batch * w.heads, w.seq_len, w.n_blocks
+    keep = w.keep_blocks()
+    d0 = [x.to(cuda_device) for x in h0]
+    d1 = [x.to(cuda_device) for x in h1]
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale)
+    rp, ci, mass = usa.rt_build_block_mask_exact(*d0, keep_blocks=keep, forced_prefix_tokens=w.forced_prefix_tokens,
+                                                 block_mass=True, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    rng = np.random.default_rng(31)
+    qbs = np.unique(np.concatenate([[0, nb - 1, (bh - 1) * nb + nb - 1], rng.choice(bh * nb, 24, replace=False)]))
+    a64 = oracle.block_mass(h0[0], h0[1], d, bs, w.scale, qblocks=qbs)
+    tol = 1e-5 * (1.0 + float(np.max(a64)))
+    got = mass.reshape(-1, nb)[torch.as_tensor(qbs, device=cuda_device)].double().cpu().numpy()
+    assert np.max(np.abs(got - a64)) <= tol
+    rp_h, ci_h = rp.cpu().numpy(), ci.cpu().numpy()
+    sub_ci = np.concatenate([ci_h[rp_h[r]:rp_h[r + 1]] for r in qbs])
+    sub_rp = np.arange(len(qbs) + 1, dtype=np.int64) * keep
+    assert check_mask(sub_rp, sub_ci, a64, keep, bs, w.forced_prefix_tokens, tol) <= 1
+    # a cycle with the exact mask, checked against the oracle on sampled rows
+    tiles = usa.rt_pair_query_blocks(d0[0], rp, ci, head_dim=d, block_size=bs)
+    out0, st = usa.rt_attn_full_capture(*d0, row_ptr=rp, col_idx=ci, **kw)
+    out1 = usa.rt_attn_sparse_reshape(*d1, row_ptr=rp, col_idx=ci, stats=st, tile_blocks=tiles, **kw)
+    plain = usa.rt_attn_sparse_reshape(*d1, row_ptr=rp, col_idx=ci, stats=None, tile_blocks=tiles, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    rows = sample_rows(bh, N, SAMPLE_ROWS, seed=5)
+    sel = torch.as_tensor(rows, device=cuda_device)
+    orc = oracle.full_capture(*h0, d, bs, w.scale, rp_h, ci_h, rows=rows)
+    orc_abs = oracle.full_capture(h0[0], h0[1], h0[2].abs(), d, bs, w.scale, rp_h, ci_h, rows=rows)["u"]
+    compare_stats(st, rows, orc, orc_abs, d, f"{name} capture stats (exact mask)")
+    want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp_h, ci_h, orc, rows=rows)
+    got1 = out1.reshape(-1, D)[sel]
+    compare_out(got1, want, d, f"{name} sparse O (exact mask)")
+    full = oracle.full_capture(*h1, d, bs, w.scale, rp_h, ci_h, rows=rows)["o"]
+    g_rows = got1.double().cpu().numpy()[:, :d]
+    p_rows = plain.reshape(-1, D)[sel].double().cpu().numpy()[:, :d]
+    err_reshape = np.linalg.norm(g_rows - full) / np.linalg.norm(full)
+    err_plain = np.linalg.norm(p_rows - full) / np.linalg.norm(full)
+    assert err_reshape < 0.5 * err_plain, (name, err_reshape, err_plain)

@@ -727,3 +727,70 @@ def test_compressed_capture_peaked_rows(cuda_device, gap):
     orc_abs = oracle.full_capture(q, k, v.abs(), d, bs, scale, rp, ci)["u"]
     compare_out(out.reshape(-1, D), orc["o"], d, f"peak gap {gap:g}: capture O (compressed)")
     compare_stats(_decoded(st), np.arange(B * H * N), orc, orc_abs, d, f"peak gap {gap:g}: stats (compressed)")
+
+
+# ------------------------------------------------------------------ mask from exact block masses
+def mass_tol(a64):
+    """Bound on |fp32 GPU block mass - fp64 oracle mass| used for tie decisions."""
+    return 1e-5 * (1.0 + float(np.max(np.abs(a64))))
+
+
+@pytest.mark.parametrize("N,d,D,bs", CASES)
+@pytest.mark.parametrize("keep_frac", [Fraction(1, 4), Fraction(1, 1)])
+def test_exact_mask_matches_oracle(cuda_device, N, d, D, bs, keep_frac):
+    """Block masses from the capture pass against the oracle's fp64 softmax sums, and the
+    kept sets against the oracle's selection on them (near ties as for the pooled mask)."""
+    w = _wl(N, d, D, bs, std=1.3, seed=13 * N + d)
+    (h0, _), (d0, _) = _inputs(w, cuda_device)
+    nb = w.n_blocks
+    keep = w.keep_blocks(keep_frac)
+    forced = 70 if keep >= 2 else 0
+    rp, ci, mass = usa.rt_build_block_mask_exact(*d0, head_dim=d, block_size=bs, scale=w.scale, keep_blocks=keep,
+                                                 forced_prefix_tokens=forced, block_mass=True)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    a64 = oracle.block_mass(h0[0], h0[1], d, bs, w.scale)
+    tol = mass_tol(a64)
+    got = mass.double().cpu().numpy().reshape(a64.shape)
+    assert np.max(np.abs(got - a64)) <= tol, np.max(np.abs(got - a64))
+    differ = check_mask(rp.cpu().numpy(), ci.cpu().numpy(), a64, keep, bs, forced, tol)
+    assert differ <= max(1, (w.batch * w.heads * nb) // 100)
+
+
+def test_exact_mask_with_caller_workspace_is_identical(cuda_device):
+    """A caller workspace (filled with garbage first) gives the same masses and CSR as the
+    library's pool, and a too-small one is refused."""
+    N, d, D, bs = 1000, 72, 80, 64
+    w = _wl(N, d, D, bs, std=1.3, seed=77)
+    _, (d0, _) = _inputs(w, cuda_device)
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale, keep_blocks=4, forced_prefix_tokens=0, block_mass=True)
+    rp, ci, mass = usa.rt_build_block_mask_exact(*d0, **kw)
+    nbytes = usa.rt_exact_mask_workspace_bytes(w.batch, w.heads, N, head_dim=d, head_dim_padded=D, block_size=bs)
+    ws = torch.randint(0, 256, (nbytes,), dtype=torch.uint8, device=cuda_device)
+    rp2, ci2, mass2 = usa.rt_build_block_mask_exact(*d0, workspace=ws, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    assert torch.equal(rp, rp2) and torch.equal(ci, ci2) and torch.equal(mass, mass2)
+    with pytest.raises(usa.RtError):
+        usa.rt_build_block_mask_exact(*d0, workspace=ws[:nbytes - 256], **kw)
+
+
+def test_exact_mask_keeps_a_dominant_block(cuda_device):
+    """One key aligned with every query: with keep = 1 every query block keeps its block,
+    whatever the pooled block means say."""
+    N, d, bs = 1000, 64, 64
+    g = torch.Generator().manual_seed(9)
+    u = torch.randn(d, generator=g)
+    q = (u + 0.2 * torch.randn(1, 2, N, d, generator=g)).to(torch.bfloat16)
+    k = 0.3 * torch.randn(1, 2, N, d, generator=g)
+    k[:, :, 777] = 0.6 * u
+    k[:, :, 768:777] -= 0.3 * u  # the block's mean points away from the queries
+    k = k.to(torch.bfloat16)
+    v = torch.randn(1, 2, N, d, generator=g).to(torch.bfloat16)
+    rp, ci = usa.rt_build_block_mask_exact(q.to(cuda_device), k.to(cuda_device), v.to(cuda_device), head_dim=d,
+                                           block_size=bs, scale=0.125, keep_blocks=1)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    assert torch.all(ci == 777 // bs)
+    rp_o, ci_o = oracle.build_block_mask_exact(q, k, d, bs, 0.125, 1, 0)
+    assert np.array_equal(ci.cpu().numpy(), ci_o)

@@ -370,3 +370,75 @@ def test_exact_mask_keeps_the_block_of_a_dominant_key():
     assert list(ci_all) == list(range(N // bs)) * (N // bs)
     _, ci_f = oracle.build_block_mask_exact(q, k, d, bs, 0.125, 2, 100)  # forced blocks 0, 1
     assert list(ci_f) == [0, 1] * (N // bs)
+
+
+def test_block_mass_listed_query_blocks_match_all():
+    N, bs = 700, 64
+    q, k, _ = _rand_qkv(1, 2, N, 64, 64, std=1.5, seed=8)
+    full = oracle.block_mass(q, k, 64, bs, 0.125)
+    nb = -(-N // bs)
+    ids = np.array([0, 5, nb - 1, nb, 2 * nb - 1])
+    part = oracle.block_mass(q, k, 64, bs, 0.125, qblocks=ids)
+    assert np.array_equal(part, full.reshape(-1, nb)[ids])
+
+
+# ------------------------------------------------------------------ Hilbert token order
+def test_hilbert_order_one_is_the_u_shape():
+    assert oracle.hilbert_curve(1) == [(0, 0), (0, 1), (1, 1), (1, 0)]
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4, 6])
+def test_hilbert_curve_is_a_continuous_bijection_filling_quadrants(k):
+    cells = oracle.hilbert_curve(k)
+    n = 1 << k
+    assert sorted(cells) == [(x, y) for x in range(n) for y in range(n)]          # every cell once
+    for (x0, y0), (x1, y1) in zip(cells, cells[1:]):
+        assert abs(x1 - x0) + abs(y1 - y0) == 1                                  # 4-adjacent steps
+    assert cells[0] == (0, 0) and cells[-1] == (n - 1, 0)
+    s, q = n // 2, (n * n) // 4
+    quads = [(0, 0), (0, s), (s, s), (s, 0)]  # lower-left, upper-left, upper-right, lower-right
+    for i, (qx, qy) in enumerate(quads):
+        part = cells[i * q:(i + 1) * q]
+        assert all(qx <= x < qx + s and qy <= y < qy + s for x, y in part)
+
+
+def test_hilbert_order_permutation_with_prefix_frames_and_ragged_grid():
+    # a 3 x 5 grid inside the 8 x 8 curve, two frames, 4 text tokens in front
+    perm = oracle.hilbert_order(3, 5, frames=2, prefix=4)
+    assert sorted(perm.tolist()) == list(range(4 + 2 * 15))
+    assert perm[:4].tolist() == [0, 1, 2, 3]
+    f0, f1 = perm[4:19] - 4, perm[19:] - 19
+    assert np.array_equal(f0, f1)
+    # the cells keep the order they have on the enclosing curve
+    curve = [y * 5 + x for x, y in oracle.hilbert_curve(3) if x < 5 and y < 3]
+    assert f0.tolist() == curve
+    # a power-of-two grid is the pure curve: consecutive tokens are grid neighbours
+    p = oracle.hilbert_order(16, 16)
+    xy = [(t % 16, t // 16) for t in p]
+    assert all(abs(a[0] - b[0]) + abs(a[1] - b[1]) == 1 for a, b in zip(xy, xy[1:]))
+
+
+def test_hilbert_blocks_are_compact_squares():
+    """On a 64 x 64 grid every 64-token block of the Hilbert order is an 8 x 8 square
+    (the locality the reordering is for), where a row-major block is a 64 x 1 line."""
+    p = oracle.hilbert_order(64, 64)
+    for b in range(64):
+        xs = p[b * 64:(b + 1) * 64] % 64
+        ys = p[b * 64:(b + 1) * 64] // 64
+        assert xs.max() - xs.min() == 7 and ys.max() - ys.min() == 7
+
+
+def test_permute_tokens_round_trip_and_attention_equivariance():
+    """Un-permuting undoes permuting; full attention commutes with a common permutation of
+    the tokens (fp64 torch SDPA), which is what lets the attention path run on the reordered
+    sequence and map its output back."""
+    q, k, v = _rand_qkv(1, 2, 64, 16, 16, seed=4)
+    perm = oracle.hilbert_order(8, 8)
+    qp = oracle.permute_tokens(q, perm)
+    assert torch.equal(oracle.permute_tokens(qp, perm, inverse=True), q)
+    assert torch.equal(qp[0, 1, 5], q[0, 1, perm[5]])
+    kp, vp = oracle.permute_tokens(k, perm), oracle.permute_tokens(v, perm)
+    o = _sdpa64(q, k, v, 16)
+    op = _sdpa64(qp, kp, vp, 16)
+    back = op.reshape(1, 2, 64, 16)[..., torch.as_tensor(np.argsort(perm)), :]
+    assert torch.allclose(back.reshape(o.shape), o, atol=1e-13)

@@ -29,6 +29,8 @@ __all__ = [
     "library_path",
     "load_library",
     "rt_build_block_mask",
+    "rt_build_block_mask_exact",
+    "rt_exact_mask_workspace_bytes",
     "rt_attn_full_capture",
     "rt_attn_sparse_reshape",
     "rt_pair_query_blocks",
@@ -92,6 +94,8 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
                                                        vp]
             lib.rt_pair_query_blocks.argtypes = [shp, vp, vp, vp, vp, sz, vp]
             lib.rt_workspace_bytes.argtypes = [shp, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+            lib.rt_build_block_mask_exact.argtypes = [shp, vp, vp, vp, f32, i32, i32, vp, vp, vp, vp, sz, vp]
+            lib.rt_exact_mask_workspace_bytes.argtypes = [shp, ctypes.POINTER(sz)]
             lib.rt_status_string.argtypes = [ctypes.c_int]
             lib.rt_status_string.restype = ctypes.c_char_p
             lib.rt_abi_version.argtypes = []
@@ -102,6 +106,7 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.rt_build_block_mask_static.restype = ctypes.c_int
             for fn in ("rt_build_block_mask", "rt_attn_full_capture", "rt_attn_sparse_reshape",
                        "rt_attn_full_capture_u16", "rt_attn_sparse_reshape_u16",
+                       "rt_build_block_mask_exact", "rt_exact_mask_workspace_bytes",
                        "rt_pair_query_blocks", "rt_workspace_bytes", "rt_take_device_error",
                        "rt_selftest_wait_timeout"):
                 getattr(lib, fn).restype = ctypes.c_int
@@ -231,6 +236,51 @@ def rt_build_block_mask(q: torch.Tensor, k: torch.Tensor, *, head_dim: int, bloc
                                                  _ptr(col_idx), _ptr(block_scores), _stream_handle(dev, stream)),
               name)
     return (row_ptr, col_idx, block_scores) if want_scores else (row_ptr, col_idx)
+
+
+def rt_build_block_mask_exact(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, head_dim: int,
+                              block_size: int, scale: float, keep_blocks: int, forced_prefix_tokens: int = 0,
+                              row_ptr: torch.Tensor | None = None, col_idx: torch.Tensor | None = None,
+                              block_mass: torch.Tensor | bool | None = None, workspace: torch.Tensor | None = None,
+                              stream=None):
+    """Kept key blocks chosen by exact block attention mass (CSR).  Returns (row_ptr, col_idx[, block_mass])."""
+    name = "rt_build_block_mask_exact"
+    dims = _check_qkv(name, q, k, v)
+    B, H, N, D = dims
+    nb = -(-N // block_size) if block_size > 0 else 0
+    dev = q.device
+    if row_ptr is None:
+        row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        col_idx = torch.empty(B * H * nb * max(keep_blocks, 0), dtype=torch.int32, device=dev)
+    _check_buf(name, "row_ptr", row_ptr, torch.int32, dev, min_numel=B * H * nb + 1)
+    _check_buf(name, "col_idx", col_idx, torch.int32, dev, min_numel=B * H * nb * max(keep_blocks, 0))
+    want_mass = block_mass is True
+    if want_mass:
+        block_mass = torch.empty(B, H, nb, nb, dtype=torch.float32, device=dev)
+    elif block_mass is False:
+        block_mass = None
+    if block_mass is not None:
+        _check_buf(name, "block_mass", block_mass, torch.float32, dev, min_numel=B * H * nb * nb)
+    if workspace is not None:
+        _check_buf(name, "workspace", workspace, torch.uint8, dev)
+    shape = _shape(dims, head_dim, block_size)
+    with torch.cuda.device(dev):
+        _call(load_library().rt_build_block_mask_exact(
+            ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), float(scale), int(keep_blocks),
+            int(forced_prefix_tokens), _ptr(row_ptr), _ptr(col_idx), _ptr(block_mass), _ptr(workspace),
+            _nbytes(workspace), _stream_handle(dev, stream)), name)
+    return (row_ptr, col_idx, block_mass) if want_mass else (row_ptr, col_idx)
+
+
+def rt_exact_mask_workspace_bytes(batch: int, heads: int, seq_len: int, *, head_dim: int, head_dim_padded: int,
+                                  block_size: int) -> int:
+    """Workspace bytes rt_build_block_mask_exact needs for this shape."""
+    shape = RtShape(batch, heads, seq_len, head_dim, head_dim_padded, block_size)
+    n = ctypes.c_size_t(0)
+    _call(load_library().rt_exact_mask_workspace_bytes(ctypes.byref(shape), ctypes.byref(n)),
+          "rt_exact_mask_workspace_bytes")
+    return int(n.value)
 
 
 def rt_attn_full_capture(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, head_dim: int, block_size: int,

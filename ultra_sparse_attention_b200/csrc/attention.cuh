@@ -100,6 +100,9 @@ struct AttnArgs {
   float* out_u;
   uint16_t* out_u16;     // compressed cache out (instead of out_u)
   float* out_u_scale;
+  // capture step, optional: per 64-key tile t and row i, log2 of the row's exponential sum over
+  // the tile (units of s * scale * log2 e), fp32 [B*H][ceil(N/64)][N]
+  float* out_block_lse;
   __nv_bfloat16* out;
   // sparse step: the query blocks of each 128-row tile, int32 [B*H][n_tiles][2]
   // (-1: empty half); null = the neighbouring blocks
@@ -1178,6 +1181,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
       if (kept) zk += zt;
       else zm += zt;
+      if (a.out_block_lse != nullptr && valid)  // coalesced: a warp's 32 rows are consecutive
+        a.out_block_lse[(static_cast<size_t>(bh) * Tn + j) * a.N + i] = m_run + __log2f(zt) - kPBias;
       if (!masked_any) {
         tmem_st32(sbuf, pk);  // kept by every row
       } else {
@@ -1251,7 +1256,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
           for (int c = 0; c < 16; ++c) ouv[c] = 0.f;
         }
-        if (valid) {
+        if (valid && a.out != nullptr) {  // no O and U in the block-mass pass
           uint32_t w[8];
           float uo[16];
 #pragma unroll

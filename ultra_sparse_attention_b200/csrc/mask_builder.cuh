@@ -100,72 +100,18 @@ __device__ __forceinline__ bool sel_better(float sa, int ka, float sb, int kb) {
   return sa > sb || (sa == sb && ka < kb);
 }
 
-// grid (ceil(n_blocks / kSelWarps), B*H), 32*kSelWarps threads.
-template <int D>
-__global__ void __launch_bounds__(32 * kSelWarps)
-    score_select_kernel(const float* __restrict__ pooled_q, const float* __restrict__ pooled_k, int n_blocks,
-                        int bs, float scale, int keep, int forced_tokens, int32_t* __restrict__ row_ptr,
-                        int32_t* __restrict__ col_idx, float* __restrict__ block_scores) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  constexpr int kS = sel_stride<D>();
-  static_assert(D % 4 == 0, "pooled rows are read as float4");
-  float* pk = reinterpret_cast<float*>(smem_raw);                 // [kSelChunk][D+4]
-  float* pq = pk + kSelChunk * kS;                                // [kSelWarps][D]
-  float* sc = pq + kSelWarps * D;                                 // [kSelWarps][n_blocks]
-  uint32_t* taken = reinterpret_cast<uint32_t*>(sc + kSelWarps * n_blocks);  // [kSelWarps][words]
-  __shared__ int skip;
-  if (threadIdx.x == 0) skip = device_status_set() ? 1 : 0;
-  __syncthreads();
-  if (skip) return;  // an earlier kernel failed (block-uniform)
-
-  const int bh = blockIdx.y;
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int qb = blockIdx.x * kSelWarps + warp;
-  const bool have_row = qb < n_blocks;
+// One query block's selection by a warp: the top `keep` key blocks of my_sc[0, n_blocks) in the
+// (score desc, index asc) order, the forced prefix blocks first -- up to 8 by rounds of a warp
+// arg-max, more by a threshold found with a binary search over order-preserving score keys --
+// then a ballot scan that writes CSR row `row` ascending (row_ptr[row], and row_ptr[row + 1]
+// for the last row).  my_taken: select_words(n_blocks) words of scratch, cleared here.
+__device__ __forceinline__ void select_row(const float* my_sc, uint32_t* my_taken, int n_blocks, int bs, int keep,
+                                           int forced_tokens, size_t row, bool last_row,
+                                           int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
+                                           int lane) {
   const int words = select_words(n_blocks);
-  const size_t head = static_cast<size_t>(bh) * n_blocks;
-
-  for (int i = threadIdx.x; i < kSelWarps * (D / 4); i += blockDim.x) {
-    const int w = i / (D / 4), c4 = i % (D / 4);
-    const int qq = blockIdx.x * kSelWarps + w;
-    reinterpret_cast<float4*>(pq + w * D)[c4] =
-        qq < n_blocks ? reinterpret_cast<const float4*>(pooled_q + (head + qq) * D)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  for (int i = threadIdx.x; i < kSelWarps * words; i += blockDim.x) taken[i] = 0u;
-
-  float* my_sc = sc + warp * n_blocks;
-  for (int kb0 = 0; kb0 < n_blocks; kb0 += kSelChunk) {
-    __syncthreads();
-    const int nch = min(kSelChunk, n_blocks - kb0);
-    for (int i = threadIdx.x; i < nch * (D / 4); i += blockDim.x) {
-      const int r = i / (D / 4), c4 = i % (D / 4);
-      reinterpret_cast<float4*>(pk + r * kS)[c4] = reinterpret_cast<const float4*>(pooled_k + (head + kb0 + r) * D)[c4];
-    }
-    __syncthreads();
-    if (have_row) {
-      const float4* a = reinterpret_cast<const float4*>(pq + warp * D);
-      for (int r = lane; r < nch; r += 32) {
-        const float4* b = reinterpret_cast<const float4*>(pk + r * kS);
-        // Four partial sums (one per float4 lane) keep four FMA chains in flight.
-        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll
-        for (int c4 = 0; c4 < D / 4; ++c4) {
-          const float4 x = a[c4], y = b[c4];
-          acc0 = fmaf(x.x, y.x, acc0);
-          acc1 = fmaf(x.y, y.y, acc1);
-          acc2 = fmaf(x.z, y.z, acc2);
-          acc3 = fmaf(x.w, y.w, acc3);
-        }
-        float s = scale * ((acc0 + acc1) + (acc2 + acc3));
-        if (s != s) s = -INFINITY;  // a NaN never wins
-        my_sc[kb0 + r] = s;
-      }
-    }
-  }
+  for (int w = lane; w < words; w += 32) my_taken[w] = 0u;
   __syncwarp();
-  if (!have_row) return;
-
-  uint32_t* my_taken = taken + warp * words;
   const int forced = min(n_blocks, forced_tokens > 0 ? (forced_tokens + bs - 1) / bs : 0);
   for (int kb = lane; kb < forced; kb += 32) atomicOr(&my_taken[kb / 32], 1u << (kb % 32));
   __syncwarp();
@@ -214,7 +160,6 @@ __global__ void __launch_bounds__(32 * kSelWarps)
     __syncwarp();
   }
 
-  const size_t row = head + qb;
   int32_t* out = col_idx + row * keep;
   int written = 0;
   for (int base = 0; base < n_blocks; base += 32) {
@@ -227,11 +172,146 @@ __global__ void __launch_bounds__(32 * kSelWarps)
   }
   if (lane == 0) {
     row_ptr[row] = static_cast<int32_t>(row * keep);
-    if (row + 1 == static_cast<size_t>(gridDim.y) * n_blocks)
-      row_ptr[row + 1] = static_cast<int32_t>((row + 1) * keep);
+    if (last_row) row_ptr[row + 1] = static_cast<int32_t>((row + 1) * keep);
   }
+}
+
+// grid (ceil(n_blocks / kSelWarps), B*H), 32*kSelWarps threads.
+template <int D>
+__global__ void __launch_bounds__(32 * kSelWarps)
+    score_select_kernel(const float* __restrict__ pooled_q, const float* __restrict__ pooled_k, int n_blocks,
+                        int bs, float scale, int keep, int forced_tokens, int32_t* __restrict__ row_ptr,
+                        int32_t* __restrict__ col_idx, float* __restrict__ block_scores) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  constexpr int kS = sel_stride<D>();
+  static_assert(D % 4 == 0, "pooled rows are read as float4");
+  float* pk = reinterpret_cast<float*>(smem_raw);                 // [kSelChunk][D+4]
+  float* pq = pk + kSelChunk * kS;                                // [kSelWarps][D]
+  float* sc = pq + kSelWarps * D;                                 // [kSelWarps][n_blocks]
+  uint32_t* taken = reinterpret_cast<uint32_t*>(sc + kSelWarps * n_blocks);  // [kSelWarps][words]
+  __shared__ int skip;
+  if (threadIdx.x == 0) skip = device_status_set() ? 1 : 0;
+  __syncthreads();
+  if (skip) return;  // an earlier kernel failed (block-uniform)
+
+  const int bh = blockIdx.y;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int qb = blockIdx.x * kSelWarps + warp;
+  const bool have_row = qb < n_blocks;
+  const int words = select_words(n_blocks);
+  const size_t head = static_cast<size_t>(bh) * n_blocks;
+
+  for (int i = threadIdx.x; i < kSelWarps * (D / 4); i += blockDim.x) {
+    const int w = i / (D / 4), c4 = i % (D / 4);
+    const int qq = blockIdx.x * kSelWarps + w;
+    reinterpret_cast<float4*>(pq + w * D)[c4] =
+        qq < n_blocks ? reinterpret_cast<const float4*>(pooled_q + (head + qq) * D)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+
+  float* my_sc = sc + warp * n_blocks;
+  for (int kb0 = 0; kb0 < n_blocks; kb0 += kSelChunk) {
+    __syncthreads();
+    const int nch = min(kSelChunk, n_blocks - kb0);
+    for (int i = threadIdx.x; i < nch * (D / 4); i += blockDim.x) {
+      const int r = i / (D / 4), c4 = i % (D / 4);
+      reinterpret_cast<float4*>(pk + r * kS)[c4] = reinterpret_cast<const float4*>(pooled_k + (head + kb0 + r) * D)[c4];
+    }
+    __syncthreads();
+    if (have_row) {
+      const float4* a = reinterpret_cast<const float4*>(pq + warp * D);
+      for (int r = lane; r < nch; r += 32) {
+        const float4* b = reinterpret_cast<const float4*>(pk + r * kS);
+        // Four partial sums (one per float4 lane) keep four FMA chains in flight.
+        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll
+        for (int c4 = 0; c4 < D / 4; ++c4) {
+          const float4 x = a[c4], y = b[c4];
+          acc0 = fmaf(x.x, y.x, acc0);
+          acc1 = fmaf(x.y, y.y, acc1);
+          acc2 = fmaf(x.z, y.z, acc2);
+          acc3 = fmaf(x.w, y.w, acc3);
+        }
+        float s = scale * ((acc0 + acc1) + (acc2 + acc3));
+        if (s != s) s = -INFINITY;  // a NaN never wins
+        my_sc[kb0 + r] = s;
+      }
+    }
+  }
+  __syncwarp();
+  if (!have_row) return;
+  const size_t row = head + qb;
+  select_row(my_sc, taken + warp * words, n_blocks, bs, keep, forced_tokens, row,
+             row + 1 == static_cast<size_t>(gridDim.y) * n_blocks, row_ptr, col_idx, lane);
   if (block_scores != nullptr)
     for (int kb = lane; kb < n_blocks; kb += 32) block_scores[row * n_blocks + kb] = my_sc[kb];
+}
+
+// Exact-mass selection.  block_lse [B*H][n_tiles][N] holds, per key tile of 64 keys and row i,
+// log2 of the row's exponential sum over the tile in the units of s*scale*log2(e); with the
+// row's log-sum-exp lse2_i = m_i*log2(e) + log2(Z_full_i) (m natural, from the same pass)
+//   mass[qb][kb] = sum over rows i of qb, tiles t of kb of 2^(block_lse[t][i] - lse2_i),
+// the softmax probability the block's rows give the key block.  One warp per query block:
+// the masses go to shared memory, then select_row keeps the largest.  grid
+// (ceil(n_blocks / kSelWarps), B*H), 32*kSelWarps threads.
+__host__ __device__ constexpr size_t mass_select_smem_bytes(int n_blocks) {
+  return sizeof(float) * static_cast<size_t>(kSelWarps) * n_blocks +
+         sizeof(uint32_t) * kSelWarps * select_words(n_blocks);
+}
+
+__global__ void __launch_bounds__(32 * kSelWarps)
+    mass_select_kernel(const float* __restrict__ block_lse, const float* __restrict__ stat_m,
+                       const float* __restrict__ stat_zfull, int N, int n_blocks, int bs, int keep,
+                       int forced_tokens, int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
+                       float* __restrict__ block_mass) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* sc = reinterpret_cast<float*>(smem_raw);                            // [kSelWarps][n_blocks]
+  uint32_t* taken = reinterpret_cast<uint32_t*>(sc + kSelWarps * n_blocks);  // [kSelWarps][words]
+  __shared__ int skip;
+  if (threadIdx.x == 0) skip = device_status_set() ? 1 : 0;
+  __syncthreads();
+  if (skip) return;  // an earlier kernel failed (block-uniform)
+  const int bh = blockIdx.y;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int qb = blockIdx.x * kSelWarps + warp;
+  if (qb >= n_blocks) return;  // no block-wide synchronisation below
+  const int n_tiles = (N + 63) / 64;
+  const int tiles_per_block = bs / 64;
+  const int i0 = qb * bs;
+  // Up to four rows per lane (block size 128): their log-sum-exp in log2 units.
+  float lse2[4];
+  int rows[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int r = lane + 32 * t;
+    rows[t] = (r < bs && i0 + r < N) ? i0 + r : -1;
+    lse2[t] = 0.f;
+    if (rows[t] >= 0) {
+      const size_t g = static_cast<size_t>(bh) * N + rows[t];
+      lse2[t] = __ldg(stat_m + g) * 1.4426950408889634f + __log2f(__ldg(stat_zfull + g));
+    }
+  }
+  float* my_sc = sc + warp * n_blocks;
+#pragma unroll 4
+  for (int kb = 0; kb < n_blocks; ++kb) {
+    float acc = 0.f;
+    for (int tt = 0; tt < tiles_per_block; ++tt) {
+      const int kt = kb * tiles_per_block + tt;
+      if (kt >= n_tiles) break;
+      const float* src = block_lse + (static_cast<size_t>(bh) * n_tiles + kt) * N;
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        if (rows[t] >= 0) acc += ex2_approx(__ldg(src + rows[t]) - lse2[t]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) my_sc[kb] = acc;
+  }
+  __syncwarp();
+  const size_t row = static_cast<size_t>(bh) * n_blocks + qb;
+  select_row(my_sc, taken + warp * select_words(n_blocks), n_blocks, bs, keep, forced_tokens, row,
+             row + 1 == static_cast<size_t>(gridDim.y) * n_blocks, row_ptr, col_idx, lane);
+  if (block_mass != nullptr)
+    for (int kb = lane; kb < n_blocks; kb += 32) block_mass[row * n_blocks + kb] = my_sc[kb];
 }
 
 }  // namespace rt

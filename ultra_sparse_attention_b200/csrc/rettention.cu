@@ -325,9 +325,64 @@ size_t capture_workspace_bytes(const Dims& d) {
   return static_cast<size_t>(d.bh) * d.N * d.D * 2 + static_cast<size_t>(d.bh) * 4;
 }
 
+// Workspace of rt_build_block_mask_exact, in 256-byte aligned parts: the capture pass's
+// workspace, an all-empty CSR row_ptr, the pass's m, Z_full, Z_kept and the per-tile
+// log-sum-exp of every row.
+struct ExactMaskLayout {
+  size_t capture, row_ptr, m, zfull, zkept, block_lse, total;
+};
+
+ExactMaskLayout exact_mask_layout(const Dims& d) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t rows = static_cast<size_t>(d.bh) * d.N;
+  ExactMaskLayout l;
+  l.capture = 0;
+  l.row_ptr = up(capture_workspace_bytes(d));
+  l.m = l.row_ptr + up((static_cast<size_t>(d.bh) * d.n_blocks + 1) * 4);
+  l.zfull = l.m + up(rows * 4);
+  l.zkept = l.zfull + up(rows * 4);
+  l.block_lse = l.zkept + up(rows * 4);
+  l.total = l.block_lse + up(rows * rt::key_tiles(static_cast<int>(d.N)) * 4);
+  return l;
+}
+
 // Workspace of rt_pair_query_blocks: the candidates of step 1 (none at block size 128).
 size_t pairing_workspace_bytes(const Dims& d) {
   return d.bs == 64 ? static_cast<size_t>(d.bh) * d.n_blocks * rt::kPairCands * 2 : 0;
+}
+
+// One capture-kernel pass with its V prologue: the max |v| per head and the scaled f16 copy of
+// V into `ws` (capture_workspace_bytes), then the capture kernel with the outputs set in `a`.
+rt_status capture_pass(const Dims& d, const void* q, const void* k, const void* v, float scale,
+                       const int32_t* row_ptr, const int32_t* col_idx, AttnArgs a, bool u16, void* ws,
+                       cudaStream_t s) {
+  const size_t per_head8 = static_cast<size_t>(d.N) * d.D / 8;  // D is a multiple of 16
+  const size_t v16_bytes = static_cast<size_t>(d.bh) * per_head8 * 16;
+  void* v16 = ws;
+  uint32_t* amax = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + v16_bytes);
+  Maps m;
+  // The output map is encoded on q when there is no output (the block-mass pass); it is unused.
+  if (!make_maps(&m, d, q, k, v16, a.out != nullptr ? static_cast<const void*>(a.out) : q, rt::kBM, true))
+    return RT_ERR_CUDA;
+  const size_t per_head_blocks = (per_head8 + 255) / 256;
+  const size_t want = (8 * static_cast<size_t>(sm_count()) + d.bh - 1) / d.bh;
+  const dim3 cgrid(static_cast<unsigned>(std::max<size_t>(1, std::min(per_head_blocks, want))),
+                   static_cast<unsigned>(d.bh));
+  if (cudaMemsetAsync(amax, 0, static_cast<size_t>(d.bh) * 4, s) != cudaSuccess) return RT_ERR_CUDA;
+  rt::v_absmax_kernel<<<cgrid, 256, 0, s>>>(static_cast<const uint4*>(v), per_head8, amax);
+  if (launch_status() != RT_OK) return RT_ERR_CUDA;
+  rt::convert_v_f16_kernel<<<cgrid, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), per_head8,
+                                                 amax);
+  if (launch_status() != RT_OK) return RT_ERR_CUDA;
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.v_amax = amax;
+  a.N = static_cast<int>(d.N);
+  a.d = static_cast<int>(d.d);
+  a.n_blocks = static_cast<int>(d.n_blocks);
+  a.n_heads = static_cast<int>(d.bh);
+  a.scale_log2 = scale * rt::kLog2e;
+  return dispatch_attention<true>(d, m, a, u16, s);
 }
 
 // The capture call behind rt_attn_full_capture (fp32 U) and rt_attn_full_capture_u16
@@ -352,36 +407,10 @@ rt_status full_capture_impl(const rt_shape* shape, const void* q, const void* k,
     return RT_ERR_INVALID_ARGUMENT;
   // The PV products run on f16 P and an f16 copy of V scaled per head by a power of two
   // (workspace: the copy, then the per-head max |v|; the caller's, or from the pool).
-  const size_t per_head8 = static_cast<size_t>(d.N) * d.D / 8;  // D is a multiple of 16
-  const size_t v16_bytes = static_cast<size_t>(d.bh) * per_head8 * 16;
   const bool own = workspace == nullptr;
   void* ws = workspace;
   if (own && !workspace_alloc(&ws, capture_workspace_bytes(d), s)) return RT_ERR_CUDA;
-  void* v16 = ws;
-  uint32_t* amax = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + v16_bytes);
-  Maps m;
-  if (!make_maps(&m, d, q, k, v16, out, rt::kBM, true)) {
-    if (own) cudaFreeAsync(ws, s);
-    return RT_ERR_CUDA;
-  }
-  const size_t per_head_blocks = (per_head8 + 255) / 256;
-  const size_t want = (8 * static_cast<size_t>(sm_count()) + d.bh - 1) / d.bh;
-  const dim3 cgrid(static_cast<unsigned>(std::max<size_t>(1, std::min(per_head_blocks, want))),
-                   static_cast<unsigned>(d.bh));
-  st = cudaMemsetAsync(amax, 0, static_cast<size_t>(d.bh) * 4, s) == cudaSuccess ? RT_OK : RT_ERR_CUDA;
-  if (st == RT_OK) {
-    rt::v_absmax_kernel<<<cgrid, 256, 0, s>>>(static_cast<const uint4*>(v), per_head8, amax);
-    st = launch_status();
-  }
-  if (st == RT_OK) {
-    rt::convert_v_f16_kernel<<<cgrid, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16),
-                                                   per_head8, amax);
-    st = launch_status();
-  }
   AttnArgs a{};
-  a.row_ptr = row_ptr;
-  a.col_idx = col_idx;
-  a.v_amax = amax;
   a.out_m = stat_m;
   a.out_zfull = stat_zfull;
   a.out_zkept = stat_zkept;
@@ -389,12 +418,7 @@ rt_status full_capture_impl(const rt_shape* shape, const void* q, const void* k,
   a.out_u16 = stat_u16;
   a.out_u_scale = stat_u_scale;
   a.out = static_cast<__nv_bfloat16*>(out);
-  a.N = static_cast<int>(d.N);
-  a.d = static_cast<int>(d.d);
-  a.n_blocks = static_cast<int>(d.n_blocks);
-  a.n_heads = static_cast<int>(d.bh);
-  a.scale_log2 = scale * rt::kLog2e;
-  if (st == RT_OK) st = dispatch_attention<true>(d, m, a, u16, s);
+  st = capture_pass(d, q, k, v, scale, row_ptr, col_idx, a, u16, ws, s);
   if (own && cudaFreeAsync(ws, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
   return st;
 }
@@ -598,6 +622,75 @@ rt_status rt_build_block_mask_static(const rt_shape* shape, const void* q, const
   if (st != RT_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   return mask_for_dim(d, q, k, scale, keep_blocks, forced_prefix_tokens, row_ptr, col_idx, block_scores, pooled, s);
+}
+
+rt_status rt_exact_mask_workspace_bytes(const rt_shape* shape, size_t* bytes) {
+  Dims d;
+  rt_status st = check_shape(shape, &d);
+  if (st != RT_OK) return st;
+  if (!bytes) return RT_ERR_INVALID_ARGUMENT;
+  *bytes = exact_mask_layout(d).total;
+  return RT_OK;
+}
+
+rt_status rt_build_block_mask_exact(const rt_shape* shape, const void* q, const void* k, const void* v, float scale,
+                                    int32_t keep_blocks, int32_t forced_prefix_tokens, int32_t* row_ptr,
+                                    int32_t* col_idx, float* block_mass, void* workspace, size_t workspace_bytes,
+                                    rt_stream_t stream) {
+  Dims d;
+  rt_status st = check_shape(shape, &d);
+  if (st != RT_OK) return st;
+  if (!q || !k || !v || !row_ptr || !col_idx) return RT_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(row_ptr, 4) || !aligned(col_idx, 4) ||
+      !aligned(block_mass, 4))
+    return RT_ERR_INVALID_ARGUMENT;
+  if (!scale_ok(scale) || forced_prefix_tokens < 0) return RT_ERR_INVALID_ARGUMENT;
+  if (keep_blocks < 1 || keep_blocks > d.n_blocks) return RT_ERR_INVALID_ARGUMENT;
+  const int64_t forced = std::min<int64_t>(d.n_blocks, (int64_t(forced_prefix_tokens) + d.bs - 1) / d.bs);
+  if (forced > keep_blocks) return RT_ERR_INVALID_ARGUMENT;
+  if (d.bh * d.n_blocks * keep_blocks > (int64_t(1) << 31) - 1) return RT_ERR_UNSUPPORTED;
+  const ExactMaskLayout l = exact_mask_layout(d);
+  if (workspace && (!aligned(workspace, 256) || workspace_bytes < l.total)) return RT_ERR_INVALID_ARGUMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool own = workspace == nullptr;
+  void* ws = workspace;
+  if (own && !workspace_alloc(&ws, l.total, s)) return RT_ERR_CUDA;
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  int32_t* empty_rp = reinterpret_cast<int32_t*>(base + l.row_ptr);
+  float* m = reinterpret_cast<float*>(base + l.m);
+  float* zf = reinterpret_cast<float*>(base + l.zfull);
+  float* zk = reinterpret_cast<float*>(base + l.zkept);
+  float* lse = reinterpret_cast<float*>(base + l.block_lse);
+  // Pass 1: full attention statistics of every row with no key block kept (every tile goes
+  // to the masked sum; O and U are not stored), and each row's per-tile log-sum-exp.
+  st = cudaMemsetAsync(empty_rp, 0, (static_cast<size_t>(d.bh) * d.n_blocks + 1) * 4, s) == cudaSuccess
+           ? RT_OK
+           : RT_ERR_CUDA;
+  if (st == RT_OK) {
+    AttnArgs a{};
+    a.out_m = m;
+    a.out_zfull = zf;
+    a.out_zkept = zk;
+    a.out_block_lse = lse;
+    st = capture_pass(d, q, k, v, scale, empty_rp, empty_rp, a, false, base + l.capture, s);
+  }
+  // Pass 2: block masses from the log-sum-exps, then the top-k selection per query block.
+  if (st == RT_OK) {
+    const size_t smem = rt::mass_select_smem_bytes(static_cast<int>(d.n_blocks));
+    if (cudaFuncSetAttribute(rt::mass_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess) {
+      st = RT_ERR_CUDA;
+    } else {
+      dim3 grid(static_cast<unsigned>((d.n_blocks + rt::kSelWarps - 1) / rt::kSelWarps),
+                static_cast<unsigned>(d.bh));
+      rt::mass_select_kernel<<<grid, 32 * rt::kSelWarps, smem, s>>>(
+          lse, m, zf, static_cast<int>(d.N), static_cast<int>(d.n_blocks), static_cast<int>(d.bs), keep_blocks,
+          forced_prefix_tokens, row_ptr, col_idx, block_mass);
+      st = launch_status();
+    }
+  }
+  if (own && cudaFreeAsync(ws, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
+  return st;
 }
 
 rt_status rt_take_device_error(int32_t* code) {
