@@ -475,6 +475,46 @@ def run_sweep(args, device, checker=None) -> list:
                      "what": "rt_build_block_mask_exact (one full-attention pass, block masses, top-k) "
                              "instead of the pooled mask; same capture and sparse kernels"}
             del rpx, cix, tbx, stx, reshx, plainx
+        # The image grids with their tokens in Hilbert order (each 64-token block an 8 x 8 patch
+        # square): the permutation's cost and the reshape's distance to full attention.
+        hilbert = None
+        if w.kind in ("smooth", "smooth_outliers"):
+            perm = usa.rt_hilbert_order(w.grid, w.grid).to(device)
+            pq0 = torch.empty_like(q0)
+            pm_ms = []
+            for it in range(args.sweep_warmup + 5):
+                flush.zero_()
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                e[0].record(stream)
+                usa.rt_permute_tokens(q0, perm, out=pq0, head_dim=w.head_dim)
+                e[1].record(stream)
+                if it >= args.sweep_warmup:
+                    pm_ms.append((e[0], e[1]))
+            hp0 = [usa.rt_permute_tokens(x, perm, head_dim=w.head_dim) for x in (q0, k0, v0)]
+            hp1 = [usa.rt_permute_tokens(x, perm, head_dim=w.head_dim) for x in (q1, k1, v1)]
+            rph, cih = usa.rt_build_block_mask(hp0[0], hp0[1], keep_blocks=keep,
+                                               forced_prefix_tokens=w.forced_prefix_tokens, **kw)
+            tbh = usa.rt_pair_query_blocks(hp0[0], rph, cih, head_dim=w.head_dim, block_size=w.block_size)
+            _, sth = usa.rt_attn_full_capture(*hp0, row_ptr=rph, col_idx=cih, **kw)
+            resh = usa.rt_permute_tokens(usa.rt_attn_sparse_reshape(*hp1, row_ptr=rph, col_idx=cih, stats=sth,
+                                                                    tile_blocks=tbh, **kw), perm, inverse=True,
+                                         head_dim=w.head_dim)
+            plainh = usa.rt_permute_tokens(usa.rt_attn_sparse_reshape(*hp1, row_ptr=rph, col_idx=cih, stats=None,
+                                                                      tile_blocks=tbh, **kw), perm, inverse=True,
+                                           head_dim=w.head_dim)
+            torch.cuda.synchronize()
+            if usa.rt_take_device_error() != 0:
+                raise RuntimeError(f"a kernel reported a device error in the Hilbert cycle ({name})")
+            pm = statistics.mean(a.elapsed_time(b) for a, b in pm_ms)
+            hilbert = {"permute_ms_per_tensor": pm,
+                       "permute_gbs": 2 * q0.numel() * 2 / (pm / 1e3) / 1e9,
+                       "reshape_rel_l2_vs_full": torch.linalg.vector_norm(resh.float() - full1.float()).item() / ref_norm,
+                       "plain_sparse_rel_l2_vs_full":
+                           torch.linalg.vector_norm(plainh.float() - full1.float()).item() / ref_norm,
+                       "what": "Q/K/V of both steps reordered along the Hilbert curve of the patch grid "
+                               "(rt_hilbert_order, rt_permute_tokens), the pooled mask and the same kernels on "
+                               "the reordered tokens, the output mapped back"}
+            del perm, pq0, hp0, hp1, rph, cih, tbh, sth, resh, plainh
         del full1
         ms = {k: statistics.mean(a.elapsed_time(b) for a, b in v) for k, v in times.items()}
         nums = workload_numbers(w, keep, rp.cpu().numpy(), ci.cpu().numpy())
@@ -491,7 +531,7 @@ def run_sweep(args, device, checker=None) -> list:
                     "sparse_tensor_frac_of_bf16_peak": exe / peaks["bf16_tflops"],
                     "capture_tflops": cap, "capture_frac_of_bf16_peak": cap / peaks["bf16_tflops"],
                     "reshape_rel_l2_vs_full": err_r, "plain_sparse_rel_l2_vs_full": err_p,
-                    "exact_mass_mask": exact,
+                    "exact_mass_mask": exact, "hilbert_order": hilbert,
                     "steps": args.sweep_steps, "warmup": args.sweep_warmup, "l2": "flushed between cycles"})
         if checker is not None:
             out[-1]["oracle_check"] = checker.check(w, keep, host0, host1, rp, ci, out0, st, out1)

@@ -280,6 +280,40 @@ rt_status rt_build_block_mask_exact(const rt_shape *shape, const void *q, const 
 rt_status rt_exact_mask_workspace_bytes(const rt_shape *shape, size_t *bytes);
 
 /*
+ * rt_hilbert_order, rt_permute_tokens -- Hilbert-curve token order.
+ *
+ * HilbertA blog page, "Introducing HilbertA", first component (Reordering):
+ * tokens are put in the order of a Hilbert curve over the patch grid, so
+ * tokens that are close on the grid stay close in the sequence.  Run the
+ * attention path on Q, K, V permuted this way and map the output back with
+ * the inverse: a 64-token block of a 64 x 64 image grid is then an 8 x 8 patch
+ * square instead of one patch row, so the block mask pools and keeps
+ * spatially coherent blocks.  The results of every call are those of the same
+ * calls on the permuted tensors (attention commutes with a common permutation
+ * of its tokens); the cached statistics stay in the permuted order.
+ *
+ * rt_hilbert_order (host only, no CUDA call) writes perm[t], int32, for
+ * t < prefix_tokens + frames*grid_h*grid_w: position t of the reordered
+ * sequence takes token perm[t] of the row-major one, where cell (x, y) of
+ * frame f is token prefix_tokens + f*grid_h*grid_w + y*grid_w + x.  The
+ * prefix tokens (text) keep their places; each frame's cells follow the
+ * Hilbert curve of the smallest power-of-two square holding the grid
+ * (starting at (0, 0), ending at (2^k - 1, 0)), the square's cells outside
+ * the grid skipped.  grid sides up to 32768.  perm: host memory.
+ *
+ * rt_permute_tokens copies a bf16 [B,H,N,D] tensor: inverse = 0 gathers
+ * dst[b,h,t] = src[b,h,perm[t]], inverse != 0 scatters dst[b,h,perm[t]] =
+ * src[b,h,t].  perm: int32 [N] device, a permutation of 0..N-1 (entries
+ * outside [0, N) are skipped; a gather writes that row as zeros).  src and
+ * dst are distinct, 16-byte aligned device buffers.  HBM-bound: one read and
+ * one write of the tensor.
+ */
+rt_status rt_hilbert_order(int32_t prefix_tokens, int32_t frames, int32_t grid_h, int32_t grid_w,
+                           int32_t *perm);
+rt_status rt_permute_tokens(const rt_shape *shape, const void *src, const int32_t *perm,
+                            int32_t inverse, void *dst, rt_stream_t stream);
+
+/*
  * rt_pair_query_blocks -- group the query blocks of each head into the
  * sparse kernel's 128-row tiles.
  *

@@ -264,3 +264,46 @@ def test_full_size_exact_mask_cycle(cuda_device, name):
     err_reshape = np.linalg.norm(g_rows - full) / np.linalg.norm(full)
     err_plain = np.linalg.norm(p_rows - full) / np.linalg.norm(full)
     assert err_reshape < 0.5 * err_plain, (name, err_reshape, err_plain)
+
+
+# ------------------------------------------------------------------ Hilbert token order, full size
+@pytest.mark.parametrize("name", ["image", "long"])
+def test_full_size_hilbert_cycle(cuda_device, name):
+    """The image workloads with their tokens in Hilbert order: mask, capture and sparse step on
+    the reordered tokens, outputs mapped back, on sampled rows against the oracle doing the
+    same; the reshape stays much closer to full attention than plain sparse attention."""
+    w, h0, h1 = _host_inputs(name)
+    d, bs, D = w.head_dim, w.block_size, w.head_dim_padded
+    bh, N = w.batch * w.heads, w.seq_len
+    keep = w.keep_blocks()
+    perm = usa.rt_hilbert_order(w.grid, w.grid)
+    pd = perm.to(cuda_device)
+    p0 = [usa.rt_permute_tokens(x.to(cuda_device), pd, head_dim=d) for x in h0]
+    p1 = [usa.rt_permute_tokens(x.to(cuda_device), pd, head_dim=d) for x in h1]
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale)
+    rp, ci = usa.rt_build_block_mask(p0[0], p0[1], keep_blocks=keep, **kw)
+    tiles = usa.rt_pair_query_blocks(p0[0], rp, ci, head_dim=d, block_size=bs)
+    _, st = usa.rt_attn_full_capture(*p0, row_ptr=rp, col_idx=ci, **kw)
+    out1 = usa.rt_permute_tokens(usa.rt_attn_sparse_reshape(*p1, row_ptr=rp, col_idx=ci, stats=st, tile_blocks=tiles,
+                                                            **kw), pd, inverse=True, head_dim=d)
+    plain = usa.rt_permute_tokens(usa.rt_attn_sparse_reshape(*p1, row_ptr=rp, col_idx=ci, stats=None, **kw), pd,
+                                  inverse=True, head_dim=d)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    rp_h, ci_h = rp.cpu().numpy(), ci.cpu().numpy()
+    ph0 = [oracle.permute_tokens(x, perm.numpy()) for x in h0]
+    ph1 = [oracle.permute_tokens(x, perm.numpy()) for x in h1]
+    rows = sample_rows(bh, N, SAMPLE_ROWS, seed=17)            # rows of the original order
+    pos = np.argsort(perm.numpy())                             # where each original token sits
+    prow = (rows // N) * N + pos[rows % N]
+    orc = oracle.full_capture(*ph0, d, bs, w.scale, rp_h, ci_h, rows=prow)
+    want = oracle.sparse_reshape(*ph1, d, bs, w.scale, rp_h, ci_h, orc, rows=prow)
+    sel = torch.as_tensor(rows, device=cuda_device)
+    got = out1.reshape(-1, D)[sel]
+    compare_out(got, want, d, f"{name} Hilbert sparse O")
+    full = oracle.full_capture(*ph1, d, bs, w.scale, rp_h, ci_h, rows=prow)["o"]
+    g_rows = got.double().cpu().numpy()[:, :d]
+    p_rows = plain.reshape(-1, D)[sel].double().cpu().numpy()[:, :d]
+    err_reshape = np.linalg.norm(g_rows - full) / np.linalg.norm(full)
+    err_plain = np.linalg.norm(p_rows - full) / np.linalg.norm(full)
+    assert err_reshape < 0.5 * err_plain, (name, err_reshape, err_plain)

@@ -794,3 +794,68 @@ def test_exact_mask_keeps_a_dominant_block(cuda_device):
     assert torch.all(ci == 777 // bs)
     rp_o, ci_o = oracle.build_block_mask_exact(q, k, d, bs, 0.125, 1, 0)
     assert np.array_equal(ci.cpu().numpy(), ci_o)
+
+
+# ------------------------------------------------------------------ Hilbert token order
+@pytest.mark.parametrize("D,d", [(64, 64), (80, 72), (128, 112)])
+def test_permute_tokens_matches_oracle(cuda_device, D, d):
+    """Gather and scatter by the Hilbert order equal the oracle's reindexing bit for bit and
+    undo each other; an entry outside [0, N) gathers a zero row."""
+    B, H, gh, gw = 2, 3, 24, 40
+    N = gh * gw
+    x = torch.zeros(B, H, N, D, dtype=torch.bfloat16)
+    x[..., :d] = torch.randn(B, H, N, d, generator=torch.Generator().manual_seed(D)).to(torch.bfloat16)
+    perm = usa.rt_hilbert_order(gh, gw)
+    pd = perm.to(cuda_device)
+    xd = x.to(cuda_device)
+    fwd = usa.rt_permute_tokens(xd, pd, head_dim=d)
+    back = usa.rt_permute_tokens(fwd, pd, inverse=True, head_dim=d)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    want = oracle.permute_tokens(x, perm.numpy())
+    assert torch.equal(fwd.cpu().view(torch.int16), want.view(torch.int16))
+    assert torch.equal(back.cpu().view(torch.int16), x.view(torch.int16))
+    bad = perm.clone()
+    bad[7] = -1
+    g = usa.rt_permute_tokens(xd, bad.to(cuda_device), head_dim=d)
+    torch.cuda.synchronize()
+    assert torch.all(g[:, :, 7] == 0) and torch.equal(g[:, :, 8].cpu(), want[:, :, 8])
+
+
+@pytest.mark.parametrize("gh,gw,d,D,bs", [(32, 32, 72, 80, 64), (24, 40, 64, 64, 64), (32, 32, 72, 80, 128)])
+def test_hilbert_cycle_matches_oracle(cuda_device, gh, gw, d, D, bs):
+    """Q, K, V reordered along the Hilbert curve, then mask, capture and sparse step on the
+    reordered tokens, the outputs mapped back: against the oracle doing the same steps."""
+    N = gh * gw
+    w = Workload(name="case", batch=1, heads=2, seq_len=N, head_dim=d, head_dim_padded=D, block_size=bs,
+                 keep=(Fraction(1, 8),), forced_prefix_tokens=0, steps=2, capture_every=2, drift_sigma=0.05,
+                 kind="iid", iid_std=1.2, seed=gh + gw + bs)
+    (h0, h1), (d0, d1) = _inputs(w, cuda_device)
+    perm = usa.rt_hilbert_order(gh, gw)
+    pd = perm.to(cuda_device)
+    p0 = [usa.rt_permute_tokens(x, pd, head_dim=d) for x in d0]
+    p1 = [usa.rt_permute_tokens(x, pd, head_dim=d) for x in d1]
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale)
+    keep = w.keep_blocks()
+    rp, ci, sc = usa.rt_build_block_mask(p0[0], p0[1], keep_blocks=keep, block_scores=True, **kw)
+    out0p, st = usa.rt_attn_full_capture(*p0, row_ptr=rp, col_idx=ci, **kw)
+    out1p = usa.rt_attn_sparse_reshape(*p1, row_ptr=rp, col_idx=ci, stats=st, **kw)
+    out0 = usa.rt_permute_tokens(out0p, pd, inverse=True, head_dim=d)
+    out1 = usa.rt_permute_tokens(out1p, pd, inverse=True, head_dim=d)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    # oracle: the same steps on its own reordering of the host tensors
+    ph0 = [oracle.permute_tokens(x, perm.numpy()) for x in h0]
+    ph1 = [oracle.permute_tokens(x, perm.numpy()) for x in h1]
+    _, _, s64 = oracle.build_block_mask(ph0[0], ph0[1], d, bs, w.scale, keep, 0, return_scores=True)
+    tol = score_tol(s64)
+    assert np.max(np.abs(sc.double().cpu().numpy().reshape(s64.shape) - s64)) <= tol
+    rp_h, ci_h = rp.cpu().numpy(), ci.cpu().numpy()
+    assert check_mask(rp_h, ci_h, s64, keep, bs, 0, tol) <= 1
+    orc = oracle.full_capture(*ph0, d, bs, w.scale, rp_h, ci_h)
+    want1 = oracle.sparse_reshape(*ph1, d, bs, w.scale, rp_h, ci_h, orc)
+    inv = np.argsort(perm.numpy())
+    bh = w.batch * w.heads
+    to_orig = lambda a: a.reshape(bh, N, -1)[:, inv].reshape(bh * N, -1)
+    compare_out(out0.reshape(-1, D), to_orig(orc["o"]), d, "Hilbert capture O")
+    compare_out(out1.reshape(-1, D), to_orig(want1), d, "Hilbert sparse O")

@@ -31,6 +31,8 @@ __all__ = [
     "rt_build_block_mask",
     "rt_build_block_mask_exact",
     "rt_exact_mask_workspace_bytes",
+    "rt_hilbert_order",
+    "rt_permute_tokens",
     "rt_attn_full_capture",
     "rt_attn_sparse_reshape",
     "rt_pair_query_blocks",
@@ -96,6 +98,8 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.rt_workspace_bytes.argtypes = [shp, ctypes.POINTER(sz), ctypes.POINTER(sz)]
             lib.rt_build_block_mask_exact.argtypes = [shp, vp, vp, vp, f32, i32, i32, vp, vp, vp, vp, sz, vp]
             lib.rt_exact_mask_workspace_bytes.argtypes = [shp, ctypes.POINTER(sz)]
+            lib.rt_hilbert_order.argtypes = [i32, i32, i32, i32, vp]
+            lib.rt_permute_tokens.argtypes = [shp, vp, vp, i32, vp, vp]
             lib.rt_status_string.argtypes = [ctypes.c_int]
             lib.rt_status_string.restype = ctypes.c_char_p
             lib.rt_abi_version.argtypes = []
@@ -107,6 +111,7 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
             for fn in ("rt_build_block_mask", "rt_attn_full_capture", "rt_attn_sparse_reshape",
                        "rt_attn_full_capture_u16", "rt_attn_sparse_reshape_u16",
                        "rt_build_block_mask_exact", "rt_exact_mask_workspace_bytes",
+                       "rt_hilbert_order", "rt_permute_tokens",
                        "rt_pair_query_blocks", "rt_workspace_bytes", "rt_take_device_error",
                        "rt_selftest_wait_timeout"):
                 getattr(lib, fn).restype = ctypes.c_int
@@ -281,6 +286,35 @@ def rt_exact_mask_workspace_bytes(batch: int, heads: int, seq_len: int, *, head_
     _call(load_library().rt_exact_mask_workspace_bytes(ctypes.byref(shape), ctypes.byref(n)),
           "rt_exact_mask_workspace_bytes")
     return int(n.value)
+
+
+def rt_hilbert_order(grid_h: int, grid_w: int, *, frames: int = 1, prefix_tokens: int = 0) -> torch.Tensor:
+    """Hilbert-curve token order (host int32 [prefix + frames*grid_h*grid_w]): position t of the
+    reordered sequence takes token perm[t] of the row-major one."""
+    n = prefix_tokens + frames * grid_h * grid_w
+    perm = torch.empty(max(n, 0), dtype=torch.int32)
+    _call(load_library().rt_hilbert_order(int(prefix_tokens), int(frames), int(grid_h), int(grid_w),
+                                          ctypes.c_void_p(perm.data_ptr())), "rt_hilbert_order")
+    return perm
+
+
+def rt_permute_tokens(x: torch.Tensor, perm: torch.Tensor, *, inverse: bool = False, head_dim: int | None = None,
+                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Token-reordered copy of bf16 [B, H, N, D] ``x``: out[..., t, :] = x[..., perm[t], :], or with
+    ``inverse`` out[..., perm[t], :] = x[..., t, :].  ``perm``: int32 [N] on x's device."""
+    name = "rt_permute_tokens"
+    dims = _check_qkv(name, x)
+    B, H, N, D = dims
+    dev = x.device
+    _check_buf(name, "perm", perm, torch.int32, dev, shape=(N,))
+    if out is None:
+        out = torch.empty_like(x)
+    _check_buf(name, "out", out, torch.bfloat16, dev, shape=dims)
+    shape = _shape(dims, head_dim or D, 64)
+    with torch.cuda.device(dev):
+        _call(load_library().rt_permute_tokens(ctypes.byref(shape), _ptr(x), _ptr(perm), 1 if inverse else 0,
+                                               _ptr(out), _stream_handle(dev, stream)), name)
+    return out
 
 
 def rt_attn_full_capture(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, head_dim: int, block_size: int,

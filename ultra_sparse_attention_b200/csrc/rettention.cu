@@ -8,16 +8,20 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "rettention.h"
 #include "ptx.cuh"
 #include "mask_builder.cuh"
 #include "attention.cuh"
 #include "pairing.cuh"
+#include "hilbert.cuh"
 
 namespace {
 
@@ -691,6 +695,43 @@ rt_status rt_build_block_mask_exact(const rt_shape* shape, const void* q, const 
   }
   if (own && cudaFreeAsync(ws, s) != cudaSuccess && st == RT_OK) st = RT_ERR_CUDA;
   return st;
+}
+
+rt_status rt_hilbert_order(int32_t prefix_tokens, int32_t frames, int32_t grid_h, int32_t grid_w, int32_t* perm) {
+  if (!perm || prefix_tokens < 0 || frames < 1 || grid_h < 1 || grid_w < 1) return RT_ERR_INVALID_ARGUMENT;
+  if (grid_h > (1 << 15) || grid_w > (1 << 15)) return RT_ERR_UNSUPPORTED;
+  const int64_t cells = int64_t(grid_h) * grid_w;
+  if (prefix_tokens + frames * cells > (int64_t(1) << 31) - 1) return RT_ERR_UNSUPPORTED;
+  int k = 0;
+  while ((1 << k) < std::max(grid_h, grid_w)) ++k;
+  // The grid's cells in the order of the enclosing square's curve (cells outside are skipped).
+  std::vector<std::pair<uint64_t, int32_t>> order(static_cast<size_t>(cells));
+  for (int32_t y = 0; y < grid_h; ++y)
+    for (int32_t x = 0; x < grid_w; ++x)
+      order[static_cast<size_t>(y) * grid_w + x] = {rt::hilbert_index(k, x, y), y * grid_w + x};
+  std::sort(order.begin(), order.end());
+  for (int32_t t = 0; t < prefix_tokens; ++t) perm[t] = t;
+  for (int32_t f = 0; f < frames; ++f) {
+    const int64_t base = prefix_tokens + f * cells;
+    for (int64_t c = 0; c < cells; ++c) perm[base + c] = static_cast<int32_t>(base + order[static_cast<size_t>(c)].second);
+  }
+  return RT_OK;
+}
+
+rt_status rt_permute_tokens(const rt_shape* shape, const void* src, const int32_t* perm, int32_t inverse, void* dst,
+                            rt_stream_t stream) {
+  Dims d;
+  rt_status st = check_shape(shape, &d);
+  if (st != RT_OK) return st;
+  if (!src || !perm || !dst || src == dst) return RT_ERR_INVALID_ARGUMENT;
+  if (!aligned(src, 16) || !aligned(dst, 16) || !aligned(perm, 4)) return RT_ERR_INVALID_ARGUMENT;
+  const int chunks = static_cast<int>(d.D / 8);  // 16-byte chunks of a bf16 row
+  const size_t per_head = static_cast<size_t>(d.N) * chunks;
+  const dim3 grid(static_cast<unsigned>((per_head + 255) / 256), static_cast<unsigned>(d.bh));
+  rt::permute_rows_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(src), perm, static_cast<uint4*>(dst), static_cast<int>(d.N), chunks,
+      inverse ? 1 : 0);
+  return launch_status();
 }
 
 rt_status rt_take_device_error(int32_t* code) {
