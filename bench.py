@@ -605,8 +605,11 @@ class OracleChecker:
         def errs(got, want):
             g = got.reshape(-1, D)[sel].double().cpu().numpy()[:, :d]
             e = np.abs(g - want)
+            big = np.abs(want) > 1.0  # where the unit-scale reading of the max-abs bound differs
             return {"max_abs_unit_scale": float(np.max(e / np.maximum(1.0, np.abs(want)))),
-                    "mean_abs": float(e.mean())}
+                    "mean_abs": float(e.mean()), "max_abs_raw": float(e.max()),
+                    "max_abs_where_above_1": float(e[big].max()) if big.any() else None,
+                    "max_rel_where_above_1": float((e[big] / np.abs(want[big])).max()) if big.any() else None}
 
         zf = st.zfull.reshape(-1)[sel].double().cpu().numpy()
         zk = st.zkept.reshape(-1)[sel].double().cpu().numpy()
