@@ -859,3 +859,40 @@ def test_hilbert_cycle_matches_oracle(cuda_device, gh, gw, d, D, bs):
     to_orig = lambda a: a.reshape(bh, N, -1)[:, inv].reshape(bh * N, -1)
     compare_out(out0.reshape(-1, D), to_orig(orc["o"]), d, "Hilbert capture O")
     compare_out(out1.reshape(-1, D), to_orig(want1), d, "Hilbert sparse O")
+
+
+def test_hilbert_cycle_on_a_video_grid_with_text_prefix(cuda_device):
+    """Video token layout (text tokens in front, frames of a patch grid that is not a power of
+    two): the text keeps its place, each frame follows the enclosing curve; the cycle on the
+    reordered tokens against the oracle doing the same steps."""
+    T, F, gh, gw = 70, 3, 10, 13
+    N = T + F * gh * gw
+    d, D, bs = 64, 64, 64
+    w = Workload(name="case", batch=1, heads=2, seq_len=N, head_dim=d, head_dim_padded=D, block_size=bs,
+                 keep=(Fraction(1, 4),), forced_prefix_tokens=T, steps=2, capture_every=2, drift_sigma=0.05,
+                 kind="iid", iid_std=1.2, seed=5)
+    (h0, h1), (d0, d1) = _inputs(w, cuda_device)
+    perm = usa.rt_hilbert_order(gh, gw, frames=F, prefix_tokens=T)
+    assert np.array_equal(perm.numpy(), oracle.hilbert_order(gh, gw, frames=F, prefix=T))
+    pd = perm.to(cuda_device)
+    p0 = [usa.rt_permute_tokens(x, pd, head_dim=d) for x in d0]
+    p1 = [usa.rt_permute_tokens(x, pd, head_dim=d) for x in d1]
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale)
+    keep = w.keep_blocks()
+    rp, ci, sc = usa.rt_build_block_mask(p0[0], p0[1], keep_blocks=keep, forced_prefix_tokens=T, block_scores=True,
+                                         **kw)
+    _, st = usa.rt_attn_full_capture(*p0, row_ptr=rp, col_idx=ci, **kw)
+    out1 = usa.rt_permute_tokens(usa.rt_attn_sparse_reshape(*p1, row_ptr=rp, col_idx=ci, stats=st, **kw), pd,
+                                 inverse=True, head_dim=d)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    ph0 = [oracle.permute_tokens(x, perm.numpy()) for x in h0]
+    ph1 = [oracle.permute_tokens(x, perm.numpy()) for x in h1]
+    _, _, s64 = oracle.build_block_mask(ph0[0], ph0[1], d, bs, w.scale, keep, T, return_scores=True)
+    tol = score_tol(s64)
+    rp_h, ci_h = rp.cpu().numpy(), ci.cpu().numpy()
+    assert check_mask(rp_h, ci_h, s64, keep, bs, T, tol) <= 1
+    orc = oracle.full_capture(*ph0, d, bs, w.scale, rp_h, ci_h)
+    want1 = oracle.sparse_reshape(*ph1, d, bs, w.scale, rp_h, ci_h, orc)
+    inv = np.argsort(perm.numpy())
+    compare_out(out1.reshape(-1, D), want1.reshape(2, N, d)[:, inv].reshape(2 * N, d), d, "Hilbert video sparse O")
