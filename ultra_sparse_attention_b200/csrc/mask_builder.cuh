@@ -10,12 +10,15 @@
 // Two kernels, both bound by memory or latency, not by arithmetic:
 //   pool_blocks_kernel   reads Q and K once (HBM-bound), writes fp32 block
 //                        means [BH, n_blocks, D] (pad columns zero);
-//   score_select_kernel  one warp per query block: scores against every key
-//                        block from shared memory, then the top k in the
-//                        (score desc, index asc) order -- up to 8 by rounds of
-//                        a warp arg-max, more by a threshold found with a
-//                        binary search over order-preserving score keys --
-//                        then a ballot scan that writes the row ascending.
+//   score_select_kernel  eight query blocks per CTA: their scores against every
+//                        key block (pooled K staged in shared memory, each
+//                        thread scoring one key block against four query
+//                        blocks), then one warp per query block selects the
+//                        top k in the (score desc, index asc) order -- up to 8
+//                        by rounds of a warp arg-max, more by a threshold found
+//                        with a binary search over order-preserving score keys
+//                        -- and a ballot scan writes the row ascending.
+//   mass_select_kernel   the same selection on exact block attention masses.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -70,7 +73,7 @@ __global__ void __launch_bounds__(D / 8 * kPoolRowGroups)
 }
 
 constexpr int kSelWarps = 8;      // query blocks per CTA
-constexpr int kSelChunk = 64;     // key blocks staged in shared memory at a time
+constexpr int kSelChunk = 128;    // key blocks staged in shared memory at a time
 
 __host__ __device__ constexpr int select_words(int n_blocks) { return (n_blocks + 31) / 32; }
 
@@ -208,6 +211,11 @@ __global__ void __launch_bounds__(32 * kSelWarps)
         qq < n_blocks ? reinterpret_cast<const float4*>(pooled_q + (head + qq) * D)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 
+  // Thread t scores key block t % kSelChunk of each staged chunk against four of the CTA's query
+  // blocks, 4 * (t / kSelChunk) .. +3: one pooled K row read from shared memory serves four dot
+  // products (the query rows are the same for the whole warp, a broadcast).
+  static_assert(kSelWarps == 8 && kSelChunk * 2 == 32 * kSelWarps, "two groups of four query blocks");
+  const int kbl = threadIdx.x % kSelChunk, q0 = 4 * (threadIdx.x / kSelChunk);
   float* my_sc = sc + warp * n_blocks;
   for (int kb0 = 0; kb0 < n_blocks; kb0 += kSelChunk) {
     __syncthreads();
@@ -217,27 +225,32 @@ __global__ void __launch_bounds__(32 * kSelWarps)
       reinterpret_cast<float4*>(pk + r * kS)[c4] = reinterpret_cast<const float4*>(pooled_k + (head + kb0 + r) * D)[c4];
     }
     __syncthreads();
-    if (have_row) {
-      const float4* a = reinterpret_cast<const float4*>(pq + warp * D);
-      for (int r = lane; r < nch; r += 32) {
-        const float4* b = reinterpret_cast<const float4*>(pk + r * kS);
-        // Four partial sums (one per float4 lane) keep four FMA chains in flight.
-        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+    if (kbl < nch) {
+      const float4* b = reinterpret_cast<const float4*>(pk + kbl * kS);
+      // Two FMA chains per query block keep eight chains in flight.
+      float acc[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-        for (int c4 = 0; c4 < D / 4; ++c4) {
-          const float4 x = a[c4], y = b[c4];
-          acc0 = fmaf(x.x, y.x, acc0);
-          acc1 = fmaf(x.y, y.y, acc1);
-          acc2 = fmaf(x.z, y.z, acc2);
-          acc3 = fmaf(x.w, y.w, acc3);
+      for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 y = b[c4];
+#pragma unroll
+        for (int qi = 0; qi < 4; ++qi) {
+          const float4 x = reinterpret_cast<const float4*>(pq + (q0 + qi) * D)[c4];
+          acc[qi][0] = fmaf(x.x, y.x, acc[qi][0]);
+          acc[qi][1] = fmaf(x.y, y.y, acc[qi][1]);
+          acc[qi][0] = fmaf(x.z, y.z, acc[qi][0]);
+          acc[qi][1] = fmaf(x.w, y.w, acc[qi][1]);
         }
-        float s = scale * ((acc0 + acc1) + (acc2 + acc3));
+      }
+#pragma unroll
+      for (int qi = 0; qi < 4; ++qi) {
+        if (blockIdx.x * kSelWarps + q0 + qi >= n_blocks) continue;
+        float s = scale * (acc[qi][0] + acc[qi][1]);
         if (s != s) s = -INFINITY;  // a NaN never wins
-        my_sc[kb0 + r] = s;
+        sc[(q0 + qi) * n_blocks + kb0 + kbl] = s;
       }
     }
   }
-  __syncwarp();
+  __syncthreads();  // each row's scores were written by other threads
   if (!have_row) return;
   const size_t row = head + qb;
   select_row(my_sc, taken + warp * words, n_blocks, bs, keep, forced_tokens, row,
