@@ -37,7 +37,7 @@ def _worker(rank, world, port, out):
 
 def test_two_rank_max_and_reference_on_rank0_only():
     port = _free_port()
-    manager = mp.Manager()
+    manager = mp.get_context("spawn").Manager()  # no fork of this multi-threaded process
     out = manager.dict()
     mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
     for rank in (0, 1):

@@ -108,11 +108,13 @@ def _brute_topk(scores, keep, forced):
 def test_select_equals_brute_force(keep, forced_tokens, bs, ties):
     nkb = 8
     forced = min(nkb, -(-forced_tokens // bs)) if forced_tokens > 0 else 0
-    if forced > keep:
-        pytest.skip("forced blocks exceed keep (rejected input)")
     rng = np.random.default_rng(keep * 100 + forced_tokens + ties)
     rows = 12
     s = rng.integers(-2, 3, size=(rows, nkb)).astype(np.float64) if ties else rng.normal(size=(rows, nkb))
+    if forced > keep:  # more forced blocks than kept ones: the input is rejected, not truncated
+        with pytest.raises(RuntimeError, match="select failed"):
+            oracle.select_blocks(s, keep, bs, forced_tokens)
+        return
     row_ptr, col_idx = oracle.select_blocks(s, keep, bs, forced_tokens)
     assert list(row_ptr) == [r * keep for r in range(rows + 1)]
     for r in range(rows):
