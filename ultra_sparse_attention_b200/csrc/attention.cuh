@@ -13,8 +13,9 @@
 //                          statistics cached across denoising steps).
 //
 // Shared design (a 128-row query tile of one (batch, head) at a time):
-//  * warp 0 issues TMA loads, warp 1 issues tcgen05.mma, warps 2..5 own one
-//    query row per thread (TMEM lane = row) for the softmax and the epilogue.
+//  * warp 0 issues TMA loads, warp 1 issues tcgen05.mma (the two swapped in the
+//    second of two CTAs on an SM), warps 2..5 own one query row per thread
+//    (TMEM lane = row) for the softmax and the epilogue.
 //  * S = Q K^T lands in TMEM; the softmax writes P as bf16 back into the first
 //    32 columns of the same buffer and the PV product reads A = P straight from
 //    TMEM (no shared-memory round trip).
@@ -456,13 +457,17 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
+  // Two CTAs share an SM, one holding TMEM columns 0-255 and the other 256-511.  The second swaps
+  // the producer and MMA roles of warps 0 and 1, so that the two MMA warps sit on different SM
+  // sub-partitions (a warp's sub-partition is its index mod 4) and slow different softmax warps.
+  const int prod_w = (tmem & 256u) ? 1 : 0;
   volatile int* abort_flag = &sh.abort_flag;
   const bool run = sh.abort_flag == 0;  // block-uniform
   auto tile_of = [&](int i) { return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x); };
 
   if (!run) {
     // an earlier kernel failed: leave the outputs untouched
-  } else if (warp == 0) {
+  } else if (warp == prod_w) {
     // ---------------- producer (the whole warp; lane 0 issues the copies)
     int lists_built = 0, stores_issued = 0, q_loads = 0, g = 0, kslot = 0, vslot = 0;
     bool ok = true;
@@ -594,7 +599,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 1 - prod_w) {
     // ---------------- MMA issuer (the whole warp; one elected lane issues)
     struct Item { int i, j, T, e; bool valid; };  // query tile, key tile in it, its count, non-empty ordinal
     Item q0{-1, 0, 0, 0, false}, q1{-1, 0, 0, 0, false};  // key tiles g-2 and g-1, while their PV is pending
@@ -1029,6 +1034,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
+  // Two CTAs share an SM, one holding TMEM columns 0-255 and the other 256-511.  The second swaps
+  // the producer and MMA roles of warps 0 and 1, so that the two MMA warps sit on different SM
+  // sub-partitions (a warp's sub-partition is its index mod 4) and slow different softmax warps.
+  const int prod_w = (tmem & 256u) ? 1 : 0;
   const bool ok_any = sh.ok_any != 0, ou_any = sh.ou_any != 0;
   volatile int* abort_flag = &sh.abort_flag;
 
@@ -1045,7 +1054,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 
   if (!run) {
     // an earlier kernel failed: leave the outputs untouched
-  } else if (warp == 0) {
+  } else if (warp == prod_w) {
     if (lane == 0) {
       load_q<D>(smem + L::kOffQ, &tq, &tq_tail, &sh.q_full, q_row0, bh);
       int issued = 0;
@@ -1063,7 +1072,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           mbar_wait(&sh.kv_full[j % NS], (j / NS) & 1, &no_abort, kDrainLimitNs);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 - prod_w) {
     // MMA issuer: the whole warp, one elected lane issues.
     bool ok = warp_wait(&sh.q_full, 0, abort_flag);
     bool ok_started = false, ou_started = false;
