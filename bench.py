@@ -761,11 +761,11 @@ def build_line(args, r: dict, world: int, peaks: dict, peak_src: str, sweep, cpu
                    "algorithmic_bytes": nums["sparse_bytes"], "target_frac": 0.5}
     kept_tokens = nums["executed_flops"] / nums["dense_flops"]
     claims = [
-        {"claim": "full-attention quality with as few as 3.1% of the tokens", "source":
+        {"claim": "quality on par with full attention while attending to 3.1% of the tokens", "source":
          "Re-ttention project page, Abstract", "hardware": "not stated",
          "here": f"{r['keep']}/{w.n_blocks} key blocks per query block = {100.0 * r['keep'] / w.n_blocks:.2f}% of the "
                  f"keys; {100.0 * kept_tokens:.2f}% of the dense score work executed"},
-        {"claim": "over 95% of the attention computation skipped", "source": "Re-ttention project page, teaser",
+        {"claim": "more than 95% of the attention compute avoided", "source": "Re-ttention project page, teaser",
          "hardware": "not stated", "here": f"{100.0 * (1.0 - kept_tokens):.2f}% of the dense QK^T and PV flops skipped "
                                            "in the sparse step"},
     ]

@@ -128,8 +128,8 @@ rt_status rt_build_block_mask(const rt_shape *shape, const void *q, const void *
  *
  * The teaser corrects sparse attention with statistics kept from an earlier
  * denoising step; the mechanism highlight names the cached quantities: the
- * stable ratio between sparse and full softmax denominators and the residual
- * contribution of the masked-out tokens.  For every query row i, with
+ * ratio of the two softmax denominators (sparse over full), which stays
+ * nearly constant across steps, and what the masked keys add to the output.  For every query row i, with
  * s_ij = scale * q_i . k_j over all keys j < N and K(i) the keys of the blocks
  * that i's query block keeps:
  *   m_i      = max_j s_ij
@@ -170,9 +170,9 @@ rt_status rt_attn_full_capture(const rt_shape *shape, const void *q, const void 
 /*
  * rt_attn_sparse_reshape -- block-sparse attention with the statistical reshape.
  *
- * The Abstract reshapes the sparse attention scores with the prior softmax
- * distribution history to overcome the normalisation shift of a softmax over
- * a subset of keys; the mechanism highlight reconstructs the full
+ * The Abstract reshapes the sparse attention scores using the softmax
+ * statistics of an earlier step, to undo the shift in normalisation that a
+ * softmax over part of the keys causes; the mechanism highlight reconstructs the full
  * distribution from the reused denominator ratio and the cached residual.
  * For every query row i, over the kept keys K(i) of the current Q, K, V:
  *   m'_i = max_{j in K(i)} s_ij,  Z'_i = sum_{K(i)} exp(s_ij - m'_i),

@@ -10,7 +10,7 @@
  *   - teaser: sparse attention is corrected with statistics kept from an
  *     earlier denoising step, so that it recovers the full attention
  *     distribution;
- *   - Abstract: only a subset of tokens enters the sparse step, and the
+ *   - Abstract: the sparse step sees a small part of the tokens, and the
  *     reshape undoes the shift that normalising over that subset causes,
  *     using the softmax statistics of an earlier step;
  *   - mechanism highlight: the full/sparse softmax-denominator ratio is reused

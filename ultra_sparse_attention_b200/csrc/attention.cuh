@@ -4,9 +4,9 @@
 //                          emits the statistics the later sparse steps reuse:
 //                          row max m, Z_full, Z_kept and the fp32 residual
 //                          numerator U of the masked-out keys (project page,
-//                          mechanism highlight: the reused ratio of the sparse
-//                          and full softmax denominators, and the cached residual
-//                          contribution of the masked-out tokens).
+//                          mechanism highlight: the ratio of the two softmax
+//                          denominators, sparse over full, is reused, and what
+//                          the masked keys add to the output is cached).
 //   sparse_reshape_kernel  attention over the kept key blocks only, then the
 //                          reshape o = (N' + e^{m_c - m'} U) / (Z' * Z_full / Z_kept)
 //                          in the epilogue (teaser: sparse attention reshaped with

@@ -9,8 +9,8 @@ of CogVideoX and PixArt DiTs.  Trained weights and prompts are not available
 here, so each workload below is a synthetic stand-in with the attention
 shapes of those models: batch, heads, tokens, head dim, block size, keep
 ratio and the denoising-step schedule (full capture every k-th step, sparse
-steps in between; project page, teaser: "cached statistics across denoising
-steps").
+steps in between; project page, teaser: the statistics are cached at one
+denoising step and reused by the following ones).
 
 Every tensor is built in fp32 on the host from one ``torch.Generator``
 seeded with the workload's seed, rounded to bf16 (round-to-nearest-even) and
