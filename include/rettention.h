@@ -129,14 +129,25 @@ rt_status rt_build_block_mask(const rt_shape *shape, const void *q, const void *
  * The teaser corrects sparse attention with statistics kept from an earlier
  * denoising step; the mechanism highlight names the cached quantities: the
  * ratio of the two softmax denominators (sparse over full), which stays
- * nearly constant across steps, and what the masked keys add to the output.  For every query row i, with
- * s_ij = scale * q_i . k_j over all keys j < N and K(i) the keys of the blocks
- * that i's query block keeps:
- *   m_i      = max_j s_ij
+ * nearly constant across steps, and what the masked keys add to the output.
+ * For every query row i, with s_ij = scale * q_i . k_j over all keys j < N and
+ * K(i) the keys of the blocks that i's query block keeps:
+ *   m_i      = max_j s_ij                  (the cache's reference, see below)
  *   Z_full_i = sum_j exp(s_ij - m_i)
  *   Z_kept_i = sum_{j in K(i)} exp(s_ij - m_i)
  *   U_i      = sum_{j not in K(i)} exp(s_ij - m_i) * v_j
  *   out_i    = sum_j exp(s_ij - m_i) * v_j / Z_full_i       (full attention, bf16)
+ *
+ * m_i is the reference the three cached sums share, and the reshape does not
+ * depend on it.  It is the row max, except on a row whose kept keys carry less
+ * than 2^-64 of the mass at the max (a masked key far above every kept one):
+ * there Z_kept_i would leave fp32's range, and m_i is lowered by the integer
+ * number of binades that balances the exponents of Z_kept_i and Z_full_i (by
+ * at most 100 binades).  A kept part below ~2^-226 of the mass at the max
+ * still reads Z_kept_i = 0; the sparse step then takes that row's kept mass as
+ * unchanged since the capture (see rt_attn_sparse_reshape).  Ratios such as
+ * Z_full/Z_kept, m + log Z_full and U/Z_full are what to compare across
+ * implementations.
  *
  * The P V products take the probabilities in f16 with an f16 copy of V, made
  * by the call in a device workspace of B*H*N*D*2 + B*H*4 bytes (see
@@ -181,7 +192,12 @@ rt_status rt_attn_full_capture(const rt_shape *shape, const void *q, const void 
  * with m, Z_full, Z_kept, U from the latest capture step (same CSR).  If all
  * four statistics pointers are NULL the call computes plain block-sparse
  * attention out_i = N'_i / Z'_i.  A row whose query block keeps no key block
- * gets out_i = 0.
+ * gets out_i = 0.  The product is formed so that no intermediate leaves fp32's
+ * range when the kept keys lie far below the cached reference (where
+ * exp(m_i - m'_i) * U_i and Z_full_i / Z_kept_i can each exceed it); a row that
+ * keeps keys but has a cached Z_kept_i of 0 (a kept mass below the capture's
+ * range, see rt_attn_full_capture) gets out_i = U_i / Z_full_i, the reshape
+ * with its kept mass taken as unchanged, exact when the inputs are.
  *
  * q, k, v       bf16 [B,H,N,D] device (the current step's inputs).
  * row_ptr, col_idx  the CSR used at the capture step.

@@ -307,3 +307,39 @@ def test_full_size_hilbert_cycle(cuda_device, name):
     err_reshape = np.linalg.norm(g_rows - full) / np.linalg.norm(full)
     err_plain = np.linalg.norm(p_rows - full) / np.linalg.norm(full)
     assert err_reshape < 0.5 * err_plain, (name, err_reshape, err_plain)
+
+
+def test_long_workload_rows_led_by_masked_outlier_keys(cuda_device):
+    """The long workload's heavy-tailed outlier keys, on a 2-head draw of it: some query rows
+    score an outlier key in a masked block ~90-115 nats above every key they keep, so their
+    kept sum relative to the row max lies below fp32's range.  On the rows whose cached
+    log(Z_full / Z_kept) is largest the capture statistics and the first sparse step must
+    match the oracle, and the whole sparse step must be finite."""
+    import dataclasses
+    w = dataclasses.replace(WORKLOADS["long"], heads=2)
+    steps = denoising_inputs(w, 2)
+    h0, h1 = next(steps)[1:], next(steps)[1:]
+    d, bs = w.head_dim, w.block_size
+    kw = dict(head_dim=d, block_size=bs, scale=w.scale)
+    x0 = [t.to(cuda_device) for t in h0]
+    x1 = [t.to(cuda_device) for t in h1]
+    rp, ci = usa.rt_build_block_mask(x0[0], x0[1], keep_blocks=w.keep_blocks(), forced_prefix_tokens=0, **kw)
+    tiles = usa.rt_pair_query_blocks(x0[0], rp, ci, head_dim=d, block_size=bs)
+    _, st = usa.rt_attn_full_capture(*x0, row_ptr=rp, col_idx=ci, **kw)
+    got = usa.rt_attn_sparse_reshape(*x1, row_ptr=rp, col_idx=ci, stats=st, tile_blocks=tiles, **kw)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    assert torch.isfinite(got).all(), "non-finite sparse output"
+    log_ratio = (st.zfull.log() - st.zkept.log()).reshape(-1)
+    assert torch.isfinite(log_ratio).all()
+    rows = np.sort(torch.topk(log_ratio, 48).indices.cpu().numpy().astype(np.int64))
+    assert float(log_ratio[rows].min()) > 60.0  # the draw has the rows this test is about
+    rp_h, ci_h = rp.cpu().numpy(), ci.cpu().numpy()
+    orc = oracle.full_capture(*h0, d, bs, w.scale, rp_h, ci_h, rows=rows)
+    orc_abs = oracle.full_capture(h0[0], h0[1], h0[2].abs(), d, bs, w.scale, rp_h, ci_h, rows=rows)["u"]
+    assert np.log(orc["zfull"] / orc["zkept"]).max() > 88.0  # beyond fp32 relative to the row max
+    compare_stats(st, rows, orc, orc_abs, d, "long, 2 heads: capture stats")
+    want = oracle.sparse_reshape(*h1, d, bs, w.scale, rp_h, ci_h, orc, rows=rows)
+    D = w.head_dim_padded
+    compare_out(got.reshape(-1, D)[torch.as_tensor(rows, device=cuda_device)], want, d,
+                "long, 2 heads: sparse step on the rows led by masked outliers")

@@ -534,6 +534,106 @@ def test_capture_peaked_rows(cuda_device, N, d, D, bs, peak, gap):
     _capture_vs_oracle(cuda_device, (pad(q), pad(k), pad(v)), d, bs, scale, rp, ci, f"peak gap {gap:g} nats")
 
 
+def _csr_without_block(bh, nb, keep, seed, block):
+    """Random kept sets that never contain `block` (sorted): int32 row_ptr, col_idx."""
+    rng = np.random.default_rng(seed)
+    others = np.array([b for b in range(nb) if b != block])
+    sets = [sorted(int(x) for x in rng.choice(others, size=keep, replace=False)) for _ in range(bh * nb)]
+    row_ptr = np.array([0] + list(np.cumsum([len(s) for s in sets])), np.int32)
+    col_idx = np.array([kb for s in sets for kb in s], np.int32)
+    return row_ptr, col_idx
+
+
+@pytest.mark.parametrize("compressed", [False, True])
+@pytest.mark.parametrize("gap", [30.0, 70.0, 95.0, 115.0, 130.0])
+@pytest.mark.parametrize("N,d,D,bs,peak", [(2000, 64, 64, 64, 1500), (2000, 72, 80, 128, 700)])
+def test_masked_dominant_rows(cuda_device, N, d, D, bs, peak, gap, compressed):
+    """The mirror of the peaked rows: the row maximum sits on one key (token `peak`) in a
+    block that no query block keeps, `gap` nats above every kept key.  Relative to the row
+    max the kept sum is about e^-gap, beyond fp32 from ~87 nats on, so the cache has to
+    hold it at another reference; the statistics (through the reference-free ratio,
+    log-sum-exp and U / Z_full), the capture output and the reshaped sparse step -- on the
+    same inputs and on drifted ones -- must all meet the tolerances against the oracle,
+    with no non-finite value."""
+    g = torch.Generator().manual_seed(int(gap) + N + peak + 7)
+    B, H = 1, 2
+    scale = 1.0 / np.sqrt(d)
+    u = torch.randn(d, generator=g)
+    q = u + 0.3 * torch.randn(B, H, N, d, generator=g)
+    k = 0.5 * torch.randn(B, H, N, d, generator=g)
+    c = gap / (scale * float(u @ u))
+    k[:, :, peak] = c * u
+    v = torch.randn(B, H, N, d, generator=g)
+
+    def pad(x):
+        out = torch.zeros(B, H, N, D)
+        out[..., :d] = x
+        return out.to(torch.bfloat16)
+
+    nb = -(-N // bs)
+    rp, ci = _csr_without_block(B * H, nb, max(2, nb // 4), seed=N + peak, block=peak // bs)
+    h0 = (pad(q), pad(k), pad(v))
+    h1 = (pad(q + 0.05 * torch.randn(B, H, N, d, generator=g)), pad(k + 0.05 * torch.randn(B, H, N, d, generator=g)),
+          pad(v + 0.05 * torch.randn(B, H, N, d, generator=g)))
+    q0, k0, v0 = (x.to(cuda_device) for x in h0)
+    rp_d, ci_d = to_dev(rp, cuda_device), to_dev(ci, cuda_device)
+    out, st = usa.rt_attn_full_capture(q0, k0, v0, head_dim=d, block_size=bs, scale=scale, row_ptr=rp_d,
+                                       col_idx=ci_d, compressed=compressed)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    orc = oracle.full_capture(*h0, d, bs, scale, rp, ci)
+    orc_abs = oracle.full_capture(h0[0], h0[1], h0[2].abs(), d, bs, scale, rp, ci)["u"]
+    assert np.log(orc["zfull"] / orc["zkept"]).max() > gap - 10.0  # the case is what it claims
+    what = f"masked max {gap:g} nats up"
+    compare_out(out.reshape(-1, D), orc["o"], d, f"{what}: capture O")
+    st32 = usa.Stats(st.m, st.zfull, st.zkept, st.residual())
+    for t in (st.m, st.zfull, st.zkept, st32.u):
+        assert torch.isfinite(t).all(), f"{what}: non-finite statistics"
+    compare_stats(st32, np.arange(B * H * N), orc, orc_abs, d, f"{what}: capture stats")
+    for name, h in (("same inputs", h0), ("drifted inputs", h1)):
+        x = [t.to(cuda_device) for t in h]
+        got = usa.rt_attn_sparse_reshape(*x, head_dim=d, block_size=bs, scale=scale, row_ptr=rp_d, col_idx=ci_d,
+                                         stats=st)
+        torch.cuda.synchronize()
+        assert usa.rt_take_device_error() == 0
+        want = oracle.sparse_reshape(*h, d, bs, scale, rp, ci, orc)
+        compare_out(got.reshape(-1, D), want, d, f"{what}: sparse step, {name}")
+
+
+def test_masked_dominant_rows_beyond_the_cache_range(cuda_device):
+    """A masked maximum ~200 nats above every kept key: the kept sum lies below what the fp32
+    cache holds even at a shifted reference (its Z_kept reads 0).  The capture output is
+    still exact, and the sparse step on unchanged inputs falls back to U / Z_full -- exact
+    there, because the kept mass is negligible -- with every value finite."""
+    N, d, D, bs, peak, gap = 1000, 64, 64, 64, 600, 200.0
+    g = torch.Generator().manual_seed(99)
+    B, H = 1, 2
+    scale = 1.0 / np.sqrt(d)
+    u = torch.randn(d, generator=g)
+    q = u + 0.3 * torch.randn(B, H, N, d, generator=g)
+    k = 0.5 * torch.randn(B, H, N, d, generator=g)
+    k[:, :, peak] = gap / (scale * float(u @ u)) * u
+    v = torch.randn(B, H, N, d, generator=g)
+    h = tuple(x.to(torch.bfloat16) for x in (q, k, v))
+    nb = -(-N // bs)
+    rp, ci = _csr_without_block(B * H, nb, 4, seed=5, block=peak // bs)
+    x = [t.to(cuda_device) for t in h]
+    rp_d, ci_d = to_dev(rp, cuda_device), to_dev(ci, cuda_device)
+    out, st = usa.rt_attn_full_capture(*x, head_dim=d, block_size=bs, scale=scale, row_ptr=rp_d, col_idx=ci_d)
+    got = usa.rt_attn_sparse_reshape(*x, head_dim=d, block_size=bs, scale=scale, row_ptr=rp_d, col_idx=ci_d,
+                                     stats=st)
+    torch.cuda.synchronize()
+    assert usa.rt_take_device_error() == 0
+    orc = oracle.full_capture(*h, d, bs, scale, rp, ci)
+    assert np.log(orc["zfull"] / orc["zkept"]).min() > 170.0
+    assert (st.zkept == 0).float().mean().item() > 0.5  # most rows are beyond the range
+    for t in (st.m, st.zfull, st.u):
+        assert torch.isfinite(t).all()
+    compare_out(out.reshape(-1, D), orc["o"], d, "capture O, masked max 200 nats up")
+    compare_out(got.reshape(-1, D), oracle.sparse_reshape(*h, d, bs, scale, rp, ci, orc), d,
+                "sparse step beyond the cache range, same inputs")
+
+
 # ------------------------------------------------------------------ maximum size
 def test_cycle_at_the_block_limit(cuda_device):
     """One mask + capture + sparse cycle at the largest supported block count (2048 blocks

@@ -54,6 +54,8 @@ constexpr float kRescaleDown = 64.f; // log2 units
 constexpr float kSumUp = 0x1p8f;      // 2^kRescaleUp
 constexpr float kSumDown = 0x1p-64f;  // 2^-kRescaleDown
 constexpr float kPBias = 7.f;         // capture: f16 P carries p * 2^7 (p <= 2^8, so <= 2^15)
+constexpr float kCacheShiftBelow = 64.f;  // capture: Z_kept below 2^-64 of the row max moves the cache reference
+constexpr int kCacheShiftMax = 100;       // ... by at most 2^100 (Z_full <= 2^114.2, U <= 2^114.2 max|v|)
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 
 // Tile byte sizes for head dim D (bf16 Q/K/V tiles).  A tile is its 64-column
@@ -760,7 +762,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
               // Rescaling O needs PV(g-1) done: step g+1 (the previous tile's O is already read when j == 0).
               if (j > 0 && !warp_wait(&sh.step[(g + 1) & 7], ((g + 1) >> 3) & 1, abort_flag)) { ok = false; break; }
               tc_fence_after();
-              const float f = need ? ex2_approx(m_run - ref) : 1.f;
+              // Moving the reference down (the row so far far below the cached max) multiplies
+              // by up to 2^126 while anything has been summed (a term >= 2^-126 bounds the gap);
+              // with nothing summed yet O and z are zero and the factor could overflow, so 0.
+              const float f = need ? (z > 0.f ? ex2_approx(m_run - ref) : 0.f) : 1.f;
               tmem_row_scale<D>(tmem + lane_off + kOCol, f);
               z *= f;
             }
@@ -818,7 +823,20 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         fu = ex2_approx(mc2 - m_run) * us_c;  // us_c: U's power-of-two scale (1 for fp32 U)
       }
       const float denom = has_stats ? z * (zf_c / zk_c) : z;
-      const float inv = z > 0.f ? 1.f / denom : 0.f;
+      float inv = z > 0.f ? 1.f / denom : 0.f;
+      // o = (N' + e^{m_c - m'} U) * inv.  On a row whose kept keys lie far below its masked
+      // maximum, inv can underflow and e^{m_c - m'} U overflow although their product is of
+      // the order of |v|; there inv is raised to 2^-100 (N' * inv stays negligible, as the
+      // true value is smaller still) and U's coefficient is formed in the log domain with
+      // 2^100 taken out.  A cached Z_kept of 0 there means a kept mass below the cache's
+      // range (under ~2^-226 of the row's): the row is reshaped as if it had not changed
+      // since the capture, o = U / Z_full.
+      if (has_u && z > 0.f && !(inv >= 0x1p-100f && mc2 - m_run < 120.f)) {
+        inv = 0x1p-100f;
+        fu = (zk_c > 0.f ? ex2_approx(mc2 - m_run + __log2f(zk_c) - __log2f(zf_c) - __log2f(z) + 100.f)
+                         : __fdividef(0x1p100f, zf_c)) *
+             us_c;
+      }
       unsigned char* stg = smem + L::kOffQ + (i & 1) * T::kQBytes;
       if (Tn > 0) {
         if (!warp_wait(&sh.o_full, e & 1, abort_flag)) break;
@@ -1229,9 +1247,25 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       const float M = fmaxf(seen_k, seen_u);
       const float adjk = ex2_approx(m_k - kPBias - M);
       const float adju = ex2_approx(m_u - kPBias - M);
-      const float zkept = zk * adjk, zfull = zkept + zm * adju;
-      const float inv = zfull > 0.f ? unscale / zfull : 0.f;
-      float adj = adju * unscale;
+      const float zkept_m = zk * adjk, zfull_m = zkept_m + zm * adju;
+      const float inv = zfull_m > 0.f ? unscale / zfull_m : 0.f;
+      // Reference of the cache.  The row max M, unless the kept keys carry less than 2^-64
+      // of the row's mass: relative to M their sum may then fall below fp32's range (a masked
+      // key far above every kept one), so the cache takes a reference 2^sh lower, sh the
+      // integer that balances the two sums' exponents (Z_kept 2^-(g+f)/2, Z_full 2^(g+f)/2 for
+      // a gap of g binades and a full sum of 2^f).  The reshape formula does not depend on the
+      // reference, as long as m, Z_full, Z_kept and U share it.
+      int sh = 0;
+      float zkept = zkept_m;
+      if (zk > 0.f) {
+        const float lk = __log2f(zk) + (m_k - kPBias - M);  // log2 Z_kept relative to M
+        if (lk < -kCacheShiftBelow) {
+          sh = min(static_cast<int>(-0.5f * (lk + __log2f(zfull_m))), kCacheShiftMax);
+          zkept = ex2_approx(lk + static_cast<float>(sh));
+        }
+      }
+      const float zfull = zfull_m * exp2_int(sh);
+      float adj = adju * unscale * exp2_int(sh);
       float u_scale = 1.f;
       if constexpr (kU16) {
         // Compressed cache: the row's U as f16 times a power of two 2^-k, with k chosen so
@@ -1297,7 +1331,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
       if (valid) {  // the sums carry no V scale
         if constexpr (kU16) a.out_u_scale[row_g] = u_scale;
-        a.out_m[row_g] = M * kLn2;
+        a.out_m[row_g] = (M - static_cast<float>(sh)) * kLn2;
         a.out_zfull[row_g] = zfull;
         a.out_zkept[row_g] = zkept;
       }
