@@ -310,6 +310,13 @@ __device__ __forceinline__ float exp_row64(const float (&s)[64], float m, uint64
   return z0 + z1;
 }
 
+// U's coefficient in the sparse epilogue, times 2^100, on a row led by masked keys:
+// e^{m_c - m'} Z_kept / (Z_full Z') from logarithms, or 1 / Z_full when Z_kept is 0.  Rare, and
+// kept out of line: inlined, it costs the common epilogue ~2% (register pressure at the cap).
+__device__ __noinline__ float far_row_u_coef(float gap, float zk, float zf, float z) {
+  return zk > 0.f ? ex2_approx(gap + __log2f(zk) - __log2f(zf) - __log2f(z) + 100.f) : __fdividef(0x1p100f, zf);
+}
+
 __device__ __forceinline__ bool bitmap_has(const uint32_t* bm, int kb) { return (bm[kb / 32] >> (kb % 32)) & 1u; }
 
 // Set the bits of the kept key blocks of query block `qb` of head `bh` (threads `t0, t0+stride, ...`).
@@ -833,9 +840,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       // since the capture, o = U / Z_full.
       if (has_u && z > 0.f && !(inv >= 0x1p-100f && mc2 - m_run < 120.f)) {
         inv = 0x1p-100f;
-        fu = (zk_c > 0.f ? ex2_approx(mc2 - m_run + __log2f(zk_c) - __log2f(zf_c) - __log2f(z) + 100.f)
-                         : __fdividef(0x1p100f, zf_c)) *
-             us_c;
+        fu = far_row_u_coef(mc2 - m_run, zk_c, zf_c, z) * us_c;
       }
       unsigned char* stg = smem + L::kOffQ + (i & 1) * T::kQBytes;
       if (Tn > 0) {
