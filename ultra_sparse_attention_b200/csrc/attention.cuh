@@ -972,7 +972,8 @@ struct alignas(8) CaptureShared {
 
 template <int D>
 __host__ __device__ constexpr size_t capture_smem_bytes(int n_blocks) {
-  const size_t s = 1024 + CaptureLayout<D>::kOffShared + sizeof(CaptureShared) + 2 * sizeof(uint32_t) * attn_words(n_blocks);
+  const size_t s = 1024 + CaptureLayout<D>::kOffShared + sizeof(CaptureShared) + 2 * sizeof(uint32_t) * attn_words(n_blocks) +
+                   2 * static_cast<size_t>(n_blocks);
   return s > CaptureLayout<D>::kMinSmem ? s : CaptureLayout<D>::kMinSmem;
 }
 
@@ -1014,6 +1015,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   CaptureShared& sh = *reinterpret_cast<CaptureShared*>(smem + L::kOffShared);
   const int words = attn_words(a.n_blocks);
   uint32_t* bitmaps = reinterpret_cast<uint32_t*>(&sh + 1);
+  uint8_t* kinds = reinterpret_cast<uint8_t*>(bitmaps + 2 * attn_words(a.n_blocks));  // [key tiles]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.y;
@@ -1050,10 +1052,16 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   if (run)
     for (int t = threadIdx.x; t < Tn; t += blockDim.x) {
       const int kb = t * kBN / BS;
+      uint8_t kind = 0;
       for (int g = 0; g < nqb_here; ++g) {
-        if (bitmap_has(bitmaps + g * words, kb)) sh.ok_any = 1;
-        else sh.ou_any = 1;
+        if (bitmap_has(bitmaps + g * words, kb)) {
+          sh.ok_any = 1;
+          kind |= static_cast<uint8_t>(1u << g);
+        } else {
+          sh.ou_any = 1;
+        }
       }
+      kinds[t] = kind;
     }
   tc_fence_before();
   __syncthreads();
@@ -1066,15 +1074,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   const bool ok_any = sh.ok_any != 0, ou_any = sh.ou_any != 0;
   volatile int* abort_flag = &sh.abort_flag;
 
-  // Per key tile: does some row keep it / mask it?
+  // Per key tile: does some row keep it / mask it?  From the byte written above (bit g: query
+  // block g of the tile keeps it): evaluating the bitmaps here instead, once per key tile in
+  // the MMA and softmax warps, cost the capture ~12%.
+  const uint32_t all_kept = (1u << nqb_here) - 1u;
   auto tile_kind = [&](int j, bool& kept_any, bool& masked_any) {
-    const int kb = j * kBN / BS;
-    kept_any = false;
-    masked_any = false;
-    for (int g = 0; g < nqb_here; ++g) {
-      if (bitmap_has(bitmaps + g * words, kb)) kept_any = true;
-      else masked_any = true;
-    }
+    const uint32_t k = kinds[j];
+    kept_any = k != 0u;
+    masked_any = k != all_kept;
   };
 
   if (!run) {
@@ -1151,7 +1158,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const bool valid = i < a.N;
     const size_t row_g = static_cast<size_t>(bh) * a.N + (valid ? i : 0);
     const float C = a.scale_log2;
-    const uint32_t* my_bm = bitmaps + (grp < nqb_here ? grp : 0) * words;
     // The kept keys (O_kept, Z_kept) and the masked keys (U, the masked sum) are two online
     // softmaxes with references of their own (log2 units): each set's p stays within 2^8 of
     // its own largest term, so the f16 P of the masked rows keeps its precision even when the
@@ -1166,7 +1172,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       tc_fence_after();
       bool kept_any, masked_any;
       tile_kind(j, kept_any, masked_any);
-      const bool kept = grp < nqb_here && bitmap_has(my_bm, j * kBN / BS);  // warp-uniform
+      const bool kept = (kinds[j] >> grp) & 1u;  // warp-uniform (0 for a query block beyond the end)
       const uint32_t sbuf = tmem + lane_off + (j & 1) * 64;
       float s[64];
       tmem_ld64(sbuf, s);
