@@ -733,9 +733,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       float m_seen = -INFINITY, z = 0.f;
       bool ok = true;
       for (int j = 0; j < Tn; ++j, ++g) {
+        const uint32_t ent = lst[j];  // the list is complete: read it while S(g) is computed
         if (!warp_wait(&sh.step[g & 7], (g >> 3) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t ent = lst[j];
         const bool active = (ent >> grp) & 1u;  // warp-uniform
         const uint32_t pt = tmem + lane_off + (g & 1) * 64;
         uint32_t pk[32];
@@ -1117,10 +1117,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       return true;
     };
     auto pv = [&](int j) -> bool {
-      if (!warp_wait(&sh.p_full[j & 1], (j >> 1) & 1, abort_flag)) return false;
-      tc_fence_after();
       bool kept_any, masked_any;
       tile_kind(j, kept_any, masked_any);
+      if (!warp_wait(&sh.p_full[j & 1], (j >> 1) & 1, abort_flag)) return false;
+      tc_fence_after();
       const uint32_t v_base = sbase + L::kOffStage0 + (j % NS) * T::kStageBytes + T::kKVBytes;
       const uint32_t sbuf = tmem + (j & 1) * 64;
       if (!masked_any) {  // kept by every row: P in the S buffer
@@ -1168,11 +1168,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     bool ok = true;
     int mixed = 0;  // mixed key tiles so far
     for (int j = 0; j < Tn; ++j) {
-      if (!warp_wait(&sh.s_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
       bool kept_any, masked_any;
       tile_kind(j, kept_any, masked_any);
       const bool kept = (kinds[j] >> grp) & 1u;  // warp-uniform (0 for a query block beyond the end)
+      if (!warp_wait(&sh.s_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
       const uint32_t sbuf = tmem + lane_off + (j & 1) * 64;
       float s[64];
       tmem_ld64(sbuf, s);
