@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define RT_ABI_VERSION 6
+#define RT_ABI_VERSION 7
 
 typedef enum rt_status {
     RT_OK = 0,
@@ -155,8 +155,10 @@ rt_status rt_build_block_mask(const rt_shape *shape, const void *q, const void *
  * two separate online softmaxes, each against a reference of its own, and p
  * enters f16 as p * 2^7 with p <= 2^8: every term of U down to 2^-21 of the
  * row's largest masked term keeps 11 mantissa bits (a relative error below
- * 2^-12), smaller ones an absolute error below 2^-32 of that term, however
- * far the row's maximum lies above its masked scores.  The copy is scaled per
+ * 2^-12, plus at most 7.5e-5 for the one exponential in eight computed on the
+ * FMA pipe, see rt_selftest_exp2_poly), smaller ones an absolute error below
+ * 2^-32 of that term, however far the row's maximum lies above its masked
+ * scores.  The copy is scaled per
  * (batch, head) by the power of two that puts max |v| in [2^14, 2^15) and the
  * scale is taken out exactly afterwards, so any finite V keeps 11 mantissa
  * bits down to 2^-30 of its head's largest |v|.
@@ -397,6 +399,17 @@ rt_status rt_take_device_error(int32_t *code);
  * status word and returns.  Faults nothing and leaves the context usable.
  */
 rt_status rt_selftest_wait_timeout(int64_t timeout_ns, rt_stream_t stream);
+
+/*
+ * rt_selftest_exp2_poly -- evaluates, for the tests, the FMA-pipe 2^x that the
+ * capture kernel uses for one exponential pair in eight (Cody-Waite range
+ * reduction and a degree-3 minimax polynomial on [-1/2, 1/2]; maximum relative
+ * error 7.5e-5; inputs below -125, -inf included, give 2^-125).
+ *
+ * x  in, fp32 [n] device.   y  out, fp32 [n] device (y[i] = 2^x[i]).
+ * n = 0 does nothing; a NULL or misaligned pointer is RT_ERR_INVALID_ARGUMENT.
+ */
+rt_status rt_selftest_exp2_poly(const float *x, float *y, int32_t n, rt_stream_t stream);
 
 /*
  * rt_build_block_mask_static -- rt_build_block_mask for callers that must not

@@ -32,7 +32,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    assert usa.rt_abi_version() == 6
+    assert usa.rt_abi_version() == 7
     for code in range(5):
         s = usa.rt_status_string(code)
         assert s.startswith("RT_")
@@ -194,3 +194,13 @@ def test_exact_mask_argument_validation():
     assert ex(ws=ctypes.c_void_p(0x10010), ws_bytes=n.value) == usa.RT_ERR_INVALID_ARGUMENT  # 256-byte alignment
     assert ex(ws=ctypes.c_void_p(0x10000), ws_bytes=n.value - 1) == usa.RT_ERR_INVALID_ARGUMENT
     assert ex(shape=RtShape(1, 2, 512, 64, 64, 32)) == usa.RT_ERR_UNSUPPORTED
+
+
+def test_exp2_selftest_argument_validation():
+    """Rejected before any launch (no GPU needed); n = 0 does nothing."""
+    lib = usa.load_library()
+    assert lib.rt_selftest_exp2_poly(None, None, 0, None) == usa.RT_OK
+    assert lib.rt_selftest_exp2_poly(A16, A16, -1, None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert lib.rt_selftest_exp2_poly(None, A16, 4, None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert lib.rt_selftest_exp2_poly(A16, None, 4, None) == usa.RT_ERR_INVALID_ARGUMENT
+    assert lib.rt_selftest_exp2_poly(ctypes.c_void_p(0x10002), A16, 4, None) == usa.RT_ERR_INVALID_ARGUMENT

@@ -41,6 +41,7 @@ __all__ = [
     "rt_abi_version",
     "rt_take_device_error",
     "rt_selftest_wait_timeout",
+    "rt_selftest_exp2_poly",
     "rt_build_block_mask_static",
     "STATIC_POOL_FLOATS",
 ]
@@ -106,6 +107,7 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
             lib.rt_abi_version.restype = i32
             lib.rt_take_device_error.argtypes = [ctypes.POINTER(i32)]
             lib.rt_selftest_wait_timeout.argtypes = [i64, vp]
+            lib.rt_selftest_exp2_poly.argtypes = [vp, vp, i32, vp]
             lib.rt_build_block_mask_static.argtypes = [shp, vp, vp, f32, i32, i32, vp, vp, vp, vp]
             lib.rt_build_block_mask_static.restype = ctypes.c_int
             for fn in ("rt_build_block_mask", "rt_attn_full_capture", "rt_attn_sparse_reshape",
@@ -113,7 +115,7 @@ def load_library(build_if_needed: bool = True) -> ctypes.CDLL:
                        "rt_build_block_mask_exact", "rt_exact_mask_workspace_bytes",
                        "rt_hilbert_order", "rt_permute_tokens",
                        "rt_pair_query_blocks", "rt_workspace_bytes", "rt_take_device_error",
-                       "rt_selftest_wait_timeout"):
+                       "rt_selftest_wait_timeout", "rt_selftest_exp2_poly"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -447,6 +449,17 @@ def rt_selftest_wait_timeout(timeout_ns: int, stream=None):
     dev = torch.device("cuda", torch.cuda.current_device())
     _call(load_library().rt_selftest_wait_timeout(int(timeout_ns), _stream_handle(dev, stream)),
           "rt_selftest_wait_timeout")
+
+
+def rt_selftest_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """2^x by the capture kernel's FMA-pipe exponential (fp32 CUDA tensor in, same shape out)."""
+    if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("rt_selftest_exp2_poly: x must be a contiguous fp32 CUDA tensor")
+    y = torch.empty_like(x)
+    with torch.cuda.device(x.device):
+        _call(load_library().rt_selftest_exp2_poly(_ptr(x), _ptr(y), int(x.numel()),
+                                                   _stream_handle(x.device, stream)), "rt_selftest_exp2_poly")
+    return y
 
 
 def rt_build_block_mask_static(q: torch.Tensor, k: torch.Tensor, *, head_dim: int, block_size: int, scale: float,

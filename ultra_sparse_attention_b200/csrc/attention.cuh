@@ -1209,9 +1209,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), C2, nref), x0, x1);
-          s[c] = ex2_approx(x0);
-          s[c + 1] = ex2_approx(x1);
+          const uint64_t xx = f2_fma(f2_pack(s[c], s[c + 1]), C2, nref);
+          if (c % 16 == 14) {  // one pair in eight on the FMA pipe: the MUFU is the busier unit
+            f2_unpack(f2_exp2_poly(xx), s[c], s[c + 1]);
+          } else {
+            f2_unpack(xx, x0, x1);
+            s[c] = ex2_approx(x0);
+            s[c + 1] = ex2_approx(x1);
+          }
           zz = f2_add(zz, f2_pack(s[c], s[c + 1]));
           pk[c / 2] = pack_f16x2(s[c], s[c + 1]);
         }
@@ -1358,6 +1363,17 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
+}
+
+// Evaluates f2_exp2_poly on n inputs (pairs of lanes), for the tests of that function.
+__global__ void exp2_poly_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i], b = i + 1 < n ? x[i + 1] : 0.f;
+  float ya, yb;
+  f2_unpack(f2_exp2_poly(f2_pack(a, b)), ya, yb);
+  y[i] = ya;
+  if (i + 1 < n) y[i + 1] = yb;
 }
 
 // Per (batch, head) max |v| into amax (float bits, atomic max; zeroed before).  grid (x, B*H).

@@ -307,6 +307,32 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+// 2^x for two floats on the FMA pipe instead of the MUFU, so that a softmax can move part of
+// its exponentials off the MUFU.  Cody-Waite range reduction: x = j + f with j = rint(x) (the
+// 1.5 * 2^23 shift trick) and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial whose
+// coefficients were fitted for least maximum relative error on that interval by linear
+// programming over 20001 points (maximum relative error 7.5e-5 in fp32 Horner form, below
+// half an f16 unit, 2.4e-4); j is then added to the result's exponent field.  x is clamped to
+// [-125, 126] first so the exponent arithmetic cannot wrap: inputs below -125 (and -inf) give
+// 2^-125, not 0.  rt_selftest_exp2_poly evaluates it for the tests.
+__device__ __forceinline__ uint64_t f2_exp2_poly(uint64_t x) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x = f2_pack(fminf(fmaxf(x0, -125.f), 126.f), fminf(fmaxf(x1, -125.f), 126.f));
+  const uint64_t t = f2_add(x, f2_pack(kShift, kShift));
+  const uint64_t j = f2_add(t, f2_pack(-kShift, -kShift));
+  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x);  // exact
+  uint64_t q = f2_fma(f, f2_pack(0x1.c3f78cp-5f, 0x1.c3f78cp-5f), f2_pack(0x1.f0de34p-3f, 0x1.f0de34p-3f));
+  q = f2_fma(q, f, f2_pack(0x1.62f31ap-1f, 0x1.62f31ap-1f));
+  q = f2_fma(q, f, f2_pack(0x1.fff692p-1f, 0x1.fff692p-1f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

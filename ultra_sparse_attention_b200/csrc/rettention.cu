@@ -744,6 +744,15 @@ rt_status rt_take_device_error(int32_t* code) {
   return RT_OK;
 }
 
+rt_status rt_selftest_exp2_poly(const float* x, float* y, int32_t n, rt_stream_t stream) {
+  if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return RT_ERR_INVALID_ARGUMENT;
+  if (!aligned(x, 4) || !aligned(y, 4)) return RT_ERR_INVALID_ARGUMENT;
+  if (n == 0) return RT_OK;
+  const int pairs = (n + 1) / 2;
+  rt::exp2_poly_selftest_kernel<<<(pairs + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return launch_status();
+}
+
 rt_status rt_selftest_wait_timeout(int64_t timeout_ns, rt_stream_t stream) {
   if (timeout_ns <= 0 || timeout_ns > 10000000000ll) return RT_ERR_INVALID_ARGUMENT;
   rt::wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
