@@ -2,8 +2,10 @@
 //
 //   full_capture_kernel    full attention at a capture step; per row it also
 //                          emits the statistics the later sparse steps reuse:
-//                          row max m, Z_full, Z_kept and the fp32 residual
-//                          numerator U of the masked-out keys (project page,
+//                          the reference m (the row max, lowered on rows led by
+//                          masked keys so Z_kept stays in fp32), Z_full, Z_kept
+//                          and the residual numerator U of the masked-out keys
+//                          (project page,
 //                          mechanism highlight: the ratio of the two softmax
 //                          denominators, sparse over full, is reused, and what
 //                          the masked keys add to the output is cached).
@@ -16,9 +18,11 @@
 //  * warp 0 issues TMA loads, warp 1 issues tcgen05.mma (the two swapped in the
 //    second of two CTAs on an SM), warps 2..5 own one query row per thread
 //    (TMEM lane = row) for the softmax and the epilogue.
-//  * S = Q K^T lands in TMEM; the softmax writes P as bf16 back into the first
-//    32 columns of the same buffer and the PV product reads A = P straight from
-//    TMEM (no shared-memory round trip).
+//  * S = Q K^T lands in TMEM; the softmax writes P (bf16 in the sparse step, f16
+//    scaled by 2^7 in the capture) back into the first 32 columns of the same
+//    buffer and the PV product reads A = P straight from TMEM (no shared-memory
+//    round trip).  The capture computes one exponential pair in eight on the
+//    FMA pipe (f2_exp2_poly), the rest on the MUFU.
 //  * With 64-token blocks the 128-row tile holds two query blocks, each with
 //    its own kept list; the sparse kernel walks the union of both lists and a
 //    row whose block does not keep a tile writes P = 0 for it.  (An M = 64 MMA
