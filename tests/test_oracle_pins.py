@@ -252,6 +252,23 @@ def test_reshape_unchanged_inputs_recover_full_attention_with_max_in_masked_bloc
     assert np.any(np.abs(s_kept_max[:bs] - st["o"][:bs]) > 1e-3)
 
 
+@pytest.mark.parametrize("delta", [-40.0, 7.5, 60.0])
+def test_reshape_is_independent_of_the_cache_reference(delta):
+    """The cached m is only the reference the three sums share: m + delta with Z_full,
+    Z_kept and U scaled by e^-delta gives the same reshaped output (the GPU cache lowers m
+    on rows led by masked keys and relies on this)."""
+    N, d, D, bs = 256, 64, 64, 64
+    q0, k0, v0 = _rand_qkv(1, 2, N, d, D, seed=4)
+    q1, k1, v1 = _rand_qkv(1, 2, N, d, D, seed=5)
+    q, k, v, (row_ptr, col_idx) = _sparse_case(N, d, D, bs, seed=6)
+    st = oracle.full_capture(q0, k0, v0, d, bs, 1 / 8, row_ptr, col_idx)
+    f = math.exp(-delta)
+    moved = {"m": st["m"] + delta, "zfull": st["zfull"] * f, "zkept": st["zkept"] * f, "u": st["u"] * f}
+    want = oracle.sparse_reshape(q1, k1, v1, d, bs, 1 / 8, row_ptr, col_idx, st)
+    got = oracle.sparse_reshape(q1, k1, v1, d, bs, 1 / 8, row_ptr, col_idx, moved)
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-12)
+
+
 def test_reshape_uniform_kept_shift_closed_form():
     """Ratio reading pinned by a closed form.
 
